@@ -1,0 +1,88 @@
+"""The quantized attention method end to end, in float32 on the CPU.
+
+Test infrastructure only (see the package docstring).  This is a diagnostic:
+it predicts the error the method itself makes against exact attention, so a
+test can tell a kernel bug from the cost of 8-bit arithmetic.
+
+Steps, per (batch, query head, 128-row query block), over the 128-key tiles
+in increasing order (the blockwise online softmax the fused kernels use;
+SageAttention README, "Current Features"; qwbw.cn article, pitfalls, for the
+``pv_accum_dtype`` options):
+
+1. S = Q8 . K8^T exactly in integers (K8 holds codes of K - mean(K)).
+2. Dequantize in the log2 domain: s = S * f with
+   f = (qs * ks) * (sm_scale * log2(e)), all float32.  Keys j >= N, and
+   j > i under the causal mask, are excluded.
+3. Online softmax: m' = max(m, row max of s); p = 2^(s - m');
+   alpha = 2^(m - m'); l = l * alpha + sum(p).
+4. P is stored as E4M3(p * 448).
+5. PV: mode 0 (fp32 accumulation) O = O * alpha + P8 . V8;
+   mode 1 (fp16+fp32, "two-level accumulation") the tile's P8 . V8 is first
+   rounded to float16 (a fresh fp16 accumulator per tile), then
+   O = O * alpha + T.
+6. out = O * vs / (448 * l), rounded to the output dtype by the caller.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import fp8
+from .quant import BLOCK, P_SCALE, F32
+
+LOG2E = 1.4426950408889634
+
+
+def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None):
+    """Emulated output float32 (len(heads), len(q_blocks) * 128, d) in HND row order.
+
+    ``qz`` is the dict from ``quant.quantize``.  ``heads`` lists (b, hq) pairs
+    (default: all), ``q_blocks`` the 128-row query blocks (default: all).
+    Rows beyond N are returned as NaN.
+    """
+    B, Hq, Hkv, N, d = qz["B"], qz["Hq"], qz["Hkv"], qz["N"], qz["d"]
+    G = Hq // Hkv
+    nb = (N + BLOCK - 1) // BLOCK
+    mode = qz["pv_mode"]
+    hs = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
+    qbs = list(range(nb)) if q_blocks is None else list(q_blocks)
+    c = F32(F32(sm_scale) * F32(LOG2E))
+    out = np.full((len(hs), len(qbs) * BLOCK, d), np.nan, F32)
+    for n, (b, h) in enumerate(hs):
+        hk = h // G
+        v8 = fp8.decode(qz["v8"][b, hk]).astype(np.float64)     # (Np, dp)
+        for r, qb in enumerate(qbs):
+            rows = qb * BLOCK + np.arange(BLOCK)
+            q8 = qz["q8"][b, h, qb * BLOCK:(qb + 1) * BLOCK].astype(np.int64)
+            m = np.full(BLOCK, -np.inf, F32)
+            l = np.zeros(BLOCK, F32)
+            O = np.zeros((BLOCK, qz["dp"]), F32)
+            last = qb if causal else nb - 1
+            for j in range(last + 1):
+                keys = j * BLOCK + np.arange(BLOCK)
+                k8 = qz["k8"][b, hk, j * BLOCK:(j + 1) * BLOCK].astype(np.int64)
+                S = q8 @ k8.T
+                valid = (keys[None, :] < N) & np.ones((BLOCK, 1), bool)
+                if causal:
+                    valid &= keys[None, :] <= rows[:, None]
+                f = F32(F32(qz["qs"][b, h, qb]) * F32(qz["ks"][b, hk, j])) * c
+                smax = np.where(valid, S, np.iinfo(np.int64).min).max(axis=1)
+                has = valid.any(axis=1)
+                tmax = np.where(has, smax.astype(F32) * f, F32(-np.inf)).astype(F32)
+                m_new = np.maximum(m, tmax)
+                with np.errstate(invalid="ignore"):
+                    arg = (S.astype(np.float64) * np.float64(f) - m_new[:, None].astype(np.float64)).astype(F32)
+                p = np.where(valid, np.exp2(arg), F32(0)).astype(F32)
+                alpha = np.where(np.isneginf(m), F32(0), np.exp2((m - m_new).astype(F32))).astype(F32)
+                alpha = np.where(np.isneginf(m_new), F32(1), alpha).astype(F32)
+                l = (l * alpha + p.sum(axis=1, dtype=F32)).astype(F32)
+                p8 = fp8.decode(fp8.encode((p * F32(P_SCALE)).astype(F32)))
+                pv = p8 @ v8[j * BLOCK:(j + 1) * BLOCK]                  # exact in float64
+                if mode == 1:
+                    pv = pv.astype(np.float16)
+                O = (O * alpha[:, None] + pv.astype(F32)).astype(F32)
+                m = m_new
+            vs = qz["vs"][b, hk].astype(F32)
+            o = (O * vs[None, :] / (F32(P_SCALE) * l[:, None])).astype(F32)
+            ok = rows < N
+            out[n, r * BLOCK:(r + 1) * BLOCK][ok] = o[ok, :d]
+    return out

@@ -1,0 +1,166 @@
+"""Quantization step of SageAttention-style attention, emulated on the CPU.
+
+Test infrastructure only (see the package docstring).
+
+What the pages fix (SageAttention README, "Current Features"; qwbw.cn
+article, pitfalls section):
+
+* Q K^T runs on INT8 codes, with "smoothing" of K and scales at "varying
+  granularities";
+* P V runs in FP8;
+* head_dim is zero-padded to 64, 128 or 256 when it is none of those.
+
+Readings adopted where the pages give no formula or number (each one is a
+choice a reader can check here, and the CUDA path implements the same one):
+
+* Smoothing subtracts the per-channel mean of K over all N tokens of a
+  (batch, kv-head) (softmax is invariant to it: every score of query row i
+  shifts by q_i . mean(K)).  The mean is summed in float32 in a fixed order:
+  each 128-token block is summed token by token from its lowest token
+  (starting from +0.0, skipping tokens >= N), then the block partial sums are
+  added one by one in block order starting from +0.0, and the total is
+  divided by float(N) with one IEEE division.
+* Q and K - mean(K) get symmetric INT8 codes per (batch, head, 128-token
+  block) over all channels: amax = max |x| over the block's real tokens and
+  channels; inv = 127 / amax (one IEEE float32 division; 0 when amax = 0);
+  code = clamp(rint(x * inv), -127, 127) with rint rounding half to even;
+  scale = amax / 127.  Padded tokens and channels get code 0.
+* V gets FP8 E4M3 codes per (batch, kv-head, channel) over all tokens:
+  inv = VMAX / amax, code = E4M3_rne_satfinite(v * inv), scale = amax / VMAX.
+  VMAX is 448 for fp32 PV accumulation and 1 for the fp16+fp32 (two-level)
+  accumulation, so that one 128-key tile's fp16 partial sum is bounded by
+  128 * 448 * 1 = 57344 < 65504 and cannot overflow.
+* All float arithmetic is IEEE float32 with round-to-nearest-even and no
+  fused multiply-add; numpy float32 operations satisfy this.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from . import fp8
+
+BLOCK = 128              # tokens per Q/K scale block and per KV tile
+P_SCALE = 448.0          # p in [0, 1] is stored as E4M3(p * 448)
+VMAX = {0: 448.0, 1: 1.0}  # V code range per PV accumulation mode
+F32 = np.float32
+
+
+def padded_dim(d: int) -> int:
+    """Smallest of 64, 128, 256 that holds d (qwbw.cn article, pitfalls: pad_qkv)."""
+    for p in (64, 128, 256):
+        if d <= p:
+            return p
+    raise ValueError(f"head_dim {d} > 256 is not supported")
+
+
+def n_blocks(n: int) -> int:
+    return (n + BLOCK - 1) // BLOCK
+
+
+def to_hnd(x, layout: str) -> np.ndarray:
+    """Any fp16/bf16 tensor or array -> float32 numpy (B, H, N, d); widening is exact."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            x = x.float().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x, dtype=np.float32)
+    if layout == "NHD":
+        x = x.transpose(0, 2, 1, 3)
+    elif layout != "HND":
+        raise ValueError(layout)
+    return np.ascontiguousarray(x)
+
+
+def k_token_mean(k: np.ndarray) -> np.ndarray:
+    """Per-channel mean of K over tokens, in the fixed float32 order described above.
+
+    k: float32 (B, H, N, d) -> float32 (B, H, d).
+    """
+    B, H, N, d = k.shape
+    nb = n_blocks(N)
+    kp = np.zeros((B, H, nb * BLOCK, d), F32)
+    kp[:, :, :N] = k
+    kb = kp.reshape(B, H, nb, BLOCK, d)
+    part = np.zeros((B, H, nb, d), F32)
+    for t in range(BLOCK):
+        valid = (np.arange(nb) * BLOCK + t) < N          # skip tokens beyond N
+        part = np.where(valid[None, None, :, None], part + kb[:, :, :, t, :], part)
+    total = np.zeros((B, H, d), F32)
+    for b in range(nb):
+        total = total + part[:, :, b, :]
+    return total / F32(N)
+
+
+def int8_per_block(x: np.ndarray, dp: int):
+    """Symmetric per-(b, h, 128-token block) INT8 codes of x (float32 (B,H,N,d)).
+
+    Returns codes int8 (B, H, N_pad, dp) and scales float32 (B, H, nblocks).
+    """
+    B, H, N, d = x.shape
+    nb = n_blocks(N)
+    xp = np.zeros((B, H, nb * BLOCK, dp), F32)
+    xp[:, :, :N, :d] = x                               # padding is exact zeros
+    xb = xp.reshape(B, H, nb, BLOCK, dp)
+    amax = np.abs(xb).max(axis=(3, 4))                 # zeros cannot raise the max
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, F32(127.0) / amax, F32(0.0)).astype(F32)
+    prod = (xb * inv[:, :, :, None, None]).astype(F32)
+    codes = np.clip(np.rint(prod), -127, 127).astype(np.int8)
+    scale = (amax / F32(127.0)).astype(F32)
+    return codes.reshape(B, H, nb * BLOCK, dp), scale
+
+
+def fp8_per_channel(v: np.ndarray, dp: int, vmax: float):
+    """Per-(b, h, channel) E4M3 codes of v (float32 (B,H,N,d)) over all tokens.
+
+    Returns codes uint8 (B, H, N_pad, dp) and scales float32 (B, H, dp).
+    """
+    B, H, N, d = v.shape
+    nb = n_blocks(N)
+    amax = np.zeros((B, H, dp), F32)
+    amax[:, :, :d] = np.abs(v).max(axis=2)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, F32(vmax) / amax, F32(0.0)).astype(F32)
+    vp = np.zeros((B, H, nb * BLOCK, dp), F32)
+    vp[:, :, :N, :d] = v
+    prod = (vp * inv[:, :, None, :]).astype(F32)
+    codes = fp8.encode(prod)
+    # padded tokens are +0.0 * inv = +0.0 -> code 0; padded channels have inv 0
+    scale = (amax / F32(vmax)).astype(F32)
+    return codes, scale
+
+
+def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
+    """The whole quantization step for one attention call.
+
+    q: (B, Hq, N, d), k and v: (B, Hkv, N, d) in ``layout`` (fp16/bf16 torch
+    tensors or arrays).  Returns a dict of numpy arrays:
+      q8 int8 (B,Hq,Np,dp), qs f32 (B,Hq,nb), k8 int8 (B,Hkv,Np,dp),
+      ks f32 (B,Hkv,nb), km f32 (B,Hkv,dp), v8 uint8 (B,Hkv,Np,dp) E4M3 codes,
+      vs f32 (B,Hkv,dp), plus the sizes.
+    """
+    qf, kf, vf = (to_hnd(t, layout) for t in (q, k, v))
+    B, Hq, N, d = qf.shape
+    Hkv = kf.shape[1]
+    dp = padded_dim(d)
+    km = k_token_mean(kf)
+    ksm = (kf - km[:, :, None, :]).astype(F32)        # one float32 subtraction
+    q8, qs = int8_per_block(qf, dp)
+    k8, ks = int8_per_block(ksm, dp)
+    v8, vs = fp8_per_channel(vf, dp, VMAX[pv_mode])
+    kmp = np.zeros((B, Hkv, dp), F32)
+    kmp[:, :, :d] = km
+    return dict(q8=q8, qs=qs, k8=k8, ks=ks, km=kmp, v8=v8, vs=vs,
+                B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, dp=dp, pv_mode=pv_mode)
+
+
+def qk_int32(q8: np.ndarray, k8: np.ndarray) -> np.ndarray:
+    """Exact integer scores S = Q8 . K8^T for one head: (Nq, dp) x (Nk, dp) -> int32.
+
+    |S| <= 256 * 127^2 < 2^31, so int32 holds every value exactly.
+    """
+    s = q8.astype(np.int64) @ k8.astype(np.int64).T
+    assert np.abs(s).max(initial=0) < 2 ** 31
+    return s.astype(np.int32)

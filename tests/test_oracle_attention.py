@@ -1,0 +1,140 @@
+"""Pins for the oracle's exact float64 attention (CPU only).
+
+Brute force on tiny inputs, closed forms, invariants, and torch's SDPA in
+float64 as an independent library routine.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import attention, emulate, fp8, quant
+
+
+def _brute(q, k, v, causal, scale):
+    # pure-python loops, no numpy linear algebra
+    N, d = len(q), len(q[0])
+    out = []
+    for i in range(N):
+        js = [j for j in range(N) if (j <= i or not causal)]
+        s = [scale * sum(q[i][c] * k[j][c] for c in range(d)) for j in js]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = sum(e)
+        out.append([sum(e[t] * v[js[t]][c] for t in range(len(js))) / z for c in range(d)])
+    return out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_brute_force_tiny(causal):
+    rng = np.random.default_rng(0)
+    q, k, v = (rng.standard_normal((1, 1, 7, 3)).astype(np.float32) for _ in range(3))
+    got = attention.attention_f64(q, k, v, "HND", causal, 0.7)[0, 0]
+    ref = _brute(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, 0.7)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_closed_forms():
+    rng = np.random.default_rng(1)
+    v = rng.standard_normal((1, 1, 9, 4)).astype(np.float32)
+    k = rng.standard_normal((1, 1, 9, 4)).astype(np.float32)
+    q0 = np.zeros_like(k)
+    vf = v[0, 0].astype(np.float64)
+    # Q = 0: uniform weights -> mean of V; causal -> prefix means
+    assert np.allclose(attention.attention_f64(q0, k, v, causal=False)[0, 0], vf.mean(0)[None, :].repeat(9, 0))
+    pref = np.cumsum(vf, 0) / np.arange(1, 10)[:, None]
+    assert np.allclose(attention.attention_f64(q0, k, v, causal=True)[0, 0], pref)
+    # row 0 under the causal mask sees only key 0
+    q = rng.standard_normal((1, 1, 9, 4)).astype(np.float32)
+    assert np.allclose(attention.attention_f64(q, k, v, causal=True)[0, 0, 0], vf[0])
+    # sm_scale -> 0 gives the mean; a huge sm_scale picks the argmax key
+    assert np.allclose(attention.attention_f64(q, k, v, sm_scale=1e-12)[0, 0], vf.mean(0)[None].repeat(9, 0))
+    s = q[0, 0].astype(np.float64) @ k[0, 0].astype(np.float64).T
+    hard = vf[s.argmax(1)]
+    assert np.allclose(attention.attention_f64(q, k, v, sm_scale=1e4)[0, 0], hard, atol=1e-6)
+
+
+def test_rows_sum_and_matches_torch_sdpa_f64():
+    w = W.TINY.with_(N=100, d=24, Hq=4, Hkv=2)
+    q, k, v = W.make_inputs(w)
+    for causal in (False, True):
+        got = attention.attention_f64(q, k, v, "HND", causal, 0.3)
+        kk = k.double().repeat_interleave(2, dim=1)
+        vv = v.double().repeat_interleave(2, dim=1)
+        ref = torch.nn.functional.scaled_dot_product_attention(q.double(), kk, vv, is_causal=causal, scale=0.3)
+        assert np.allclose(got, ref.numpy(), rtol=1e-10, atol=1e-12)
+    # V = 1 gives 1 everywhere: the weights of every row sum to one
+    ones = torch.ones_like(v)
+    assert np.allclose(attention.attention_f64(q, k, ones, "HND", True, 0.3), 1.0)
+
+
+def test_invariances():
+    w = W.TINY.with_(N=64, d=16, Hq=4, Hkv=2)
+    q, k, v = (t.double().numpy() for t in W.make_inputs(w))
+    base = attention.attention_f64(q, k, v, "HND", False, 0.25)
+    # permuting keys together with values changes nothing without the mask
+    perm = np.random.default_rng(2).permutation(64)
+    assert np.allclose(attention.attention_f64(q, k[:, :, perm], v[:, :, perm], "HND", False, 0.25), base)
+    # subtracting the token mean of K changes nothing (each row of scores shifts)
+    km = k.mean(axis=2, keepdims=True)
+    for causal in (False, True):
+        assert np.allclose(attention.attention_f64(q, k - km, v, "HND", causal, 0.25),
+                           attention.attention_f64(q, k, v, "HND", causal, 0.25))
+    # GQA equals MHA with K and V repeated per group
+    mha = attention.attention_f64(q, np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1), "HND", False, 0.25)
+    assert np.allclose(mha, base)
+    # NHD storage of the same tensors gives the same result
+    nhd = attention.attention_f64(*(t.transpose(0, 2, 1, 3) for t in (q, k, v)), "NHD", False, 0.25)
+    assert np.allclose(nhd, base)
+    # zero-padding d to 128 with sm_scale 1/sqrt(96) equals the unpadded result
+    w2 = W.TINY.with_(N=50, d=96)
+    q2, k2, v2 = (t.double().numpy() for t in W.make_inputs(w2))
+    pad = lambda t: np.concatenate([t, np.zeros(t.shape[:3] + (32,))], axis=3)
+    a = attention.attention_f64(q2, k2, v2, "HND", True, 1 / math.sqrt(96))
+    b = attention.attention_f64(pad(q2), pad(k2), pad(v2), "HND", True, 1 / math.sqrt(96))
+    assert np.allclose(b[..., :96], a) and np.allclose(b[..., 96:], 0)
+    # rows/heads selection returns the same numbers as the full call
+    sel = attention.attention_f64(q, k, v, "HND", False, 0.25, heads=[(0, 3)], rows=[5, 60])
+    assert np.allclose(sel[0], base[0, 3, [5, 60]])
+
+
+def test_emulation_constant_scores_give_mean_of_v():
+    # Q = 0 makes every score 0, so every p is exactly 1 and P8 = 448 exactly;
+    # V values +-1, +-0.5 with amax 1 are exact in E4M3 after scaling by 448.
+    rng = np.random.default_rng(3)
+    N = 300
+    q = np.zeros((1, 1, N, 8), np.float32)
+    k = rng.standard_normal((1, 1, N, 8)).astype(np.float32)
+    v = rng.choice([-1.0, -0.5, 0.5, 1.0], size=(1, 1, N, 8)).astype(np.float32)
+    v[0, 0, 0] = 1.0
+    qz = quant.quantize(q, k, v, "HND", 0)
+    em = emulate.emulate(qz, False, 0.35)[0, :N]
+    assert np.allclose(em, v[0, 0].mean(0)[None].repeat(N, 0), rtol=1e-6, atol=1e-7)
+    emc = emulate.emulate(qz, True, 0.35)[0, :N]
+    pref = np.cumsum(v[0, 0].astype(np.float64), 0) / np.arange(1, N + 1)[:, None]
+    assert np.allclose(emc, pref, rtol=1e-6, atol=1e-7)
+
+
+def test_emulation_causal_row0_is_dequantized_v0():
+    w = W.TINY.with_(causal=True)
+    q, k, v = W.make_inputs(w)
+    for mode in (0, 1):
+        qz = quant.quantize(q, k, v, "HND", mode)
+        em = emulate.emulate(qz, True, 0.125, heads=[(0, 1)], q_blocks=[0])[0, 0]
+        vhat = fp8.decode(qz["v8"][0, 1, 0, :64]) * qz["vs"][0, 1, :64]
+        assert np.allclose(em, vhat, rtol=1e-6)
+
+
+def test_emulation_tracks_exact_attention():
+    # The method's own error on the tiny workload: cosine similarity >= 0.999
+    # and max abs error inside the 1e-1 bound the 9070XT bench reports.
+    w = W.TINY
+    q, k, v = W.make_inputs(w)
+    for mode in (0, 1):
+        qz = quant.quantize(q, k, v, "HND", mode)
+        em = emulate.emulate(qz, False, 0.125).reshape(1, 2, 256, 64).astype(np.float64)
+        ref = attention.attention_f64(q, k, v, "HND", False, 0.125)
+        cos = (em * ref).sum() / np.sqrt((em ** 2).sum() * (ref ** 2).sum())
+        assert cos >= 0.999 and np.abs(em - ref).max() < 0.1

@@ -1,0 +1,130 @@
+"""Seeded synthetic inputs for the quantized-attention path.
+
+This module only draws random numbers and arranges them in the shapes and
+layouts of the attention workloads; it holds none of the method's
+arithmetic.  Both the CPU oracle (through the tests) and the CUDA path (through
+the tests and the bench) are fed from here, so the two always see identical
+fp16/bf16 bits.
+
+Recipe (every draw is fp32 from a torch CPU generator, then rounded to the
+workload dtype with round-to-nearest-even):
+
+* ``normal``         Q, K, V i.i.d. N(0, 1).
+* ``normal_koffset`` as ``normal``, plus one per-channel offset vector
+  o ~ N(0, 3^2) of shape (d,) added to every K token of every batch and head
+  (the "K has a channel-wise bias" case that mean-smoothing targets).
+* ``normal_koutlier`` as ``normal``, then round(0.01 * Hkv * d) distinct
+  (kv-head, channel) pairs, chosen by the seed, have K multiplied by 8 on all
+  tokens and batches (outlier channels).
+* ``uniform2``       Q, K, V i.i.d. U(-2, 2).
+
+Each tensor has its own generator stream so that changing one tensor's shape
+never changes another's values: stream 0 = Q, 1 = K, 2 = V, 3 = K offset,
+4 = outlier choice.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Iterator
+
+import torch
+
+STREAM_Q, STREAM_K, STREAM_V, STREAM_OFFSET, STREAM_OUTLIER = 0, 1, 2, 3, 4
+
+DTYPES = {"fp16": torch.float16, "bf16": torch.bfloat16}
+
+
+@dataclasses.dataclass(frozen=True)
+class Workload:
+    """One attention problem: shapes, dtype, layout, mask and value recipe."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    dtype: str = "fp16"           # "fp16" | "bf16"
+    layout: str = "HND"           # "HND" = (B,H,N,d), "NHD" = (B,N,H,d)
+    causal: bool = False
+    dist: str = "normal"          # see module docstring
+    pv_mode: int = 0              # 0 = FP8 PV with fp32 accumulation, 1 = fp16+fp32
+    seed: int = 0
+    sm_scale: float | None = None  # None -> 1/sqrt(d)
+
+    def ops(self) -> float:
+        """Algorithmic attention operations 4*B*Hq*N^2*d, halved under the causal mask."""
+        v = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+        return v / 2 if self.causal else v
+
+    def with_(self, **kw) -> "Workload":
+        return dataclasses.replace(self, **kw)
+
+
+# The five workloads the method is exercised on (image/video DiT self-attention,
+# causal LLM prefill with GQA, head-dim padding sweep) plus the tiny one.
+TINY = Workload("tiny_b1_h2_n256_d64", 1, 2, 2, 256, 64, "fp16", "HND", False, "normal", 0, 0, 1.0 / 8.0)
+IMAGE_DIT = Workload("image_dit_b2_h24_n4096_d64", 2, 24, 24, 4096, 64, "bf16", "HND", False, "normal_koffset", 0, 2)
+VIDEO_DIT = Workload("video_dit_b1_h24_n32768_d128_nhd", 1, 24, 24, 32768, 128, "bf16", "NHD", False,
+                     "normal_koffset", 1, 3)
+LLM_GQA = Workload("llm_causal_gqa_b4_hq32_hkv8_n8192_d128", 4, 32, 8, 8192, 128, "fp16", "HND", True,
+                   "normal_koutlier", 0, 4)
+
+
+def pad_sweep() -> Iterator[Workload]:
+    """B=8, H=16, N in {1K,2K,4K,16K}, d in {96, 64}, causal and not, U(-2,2)."""
+    for n in (1024, 2048, 4096, 16384):
+        for d in (96, 64):
+            for causal in (False, True):
+                yield Workload(f"pad_sweep_b8_h16_n{n}_d{d}_{'causal' if causal else 'full'}",
+                               8, 16, 16, n, d, "fp16", "HND", causal, "uniform2", 0, 5)
+
+
+ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep())
+BY_NAME = {w.name: w for w in ALL}
+
+
+def _gen(w: Workload, stream: int) -> torch.Generator:
+    # One independent, reproducible stream per (workload seed, shape, tensor).
+    key = (w.seed * 1_000_003 + stream * 7919 + w.N * 31 + w.d * 131 + w.B * 17 + w.Hq * 3
+           + w.Hkv * 5 + (1 if w.causal else 0))
+    return torch.Generator().manual_seed(key & 0x7FFF_FFFF_FFFF)
+
+
+def _draw(w: Workload, stream: int, shape) -> torch.Tensor:
+    g = _gen(w, stream)
+    if w.dist == "uniform2":
+        return torch.rand(shape, generator=g, dtype=torch.float32) * 4.0 - 2.0
+    return torch.randn(shape, generator=g, dtype=torch.float32)
+
+
+def make_inputs(w: Workload):
+    """Return (q, k, v) as contiguous CPU tensors of w.dtype in w.layout.
+
+    Logical shapes are (B, Hq, N, d) for q and (B, Hkv, N, d) for k, v; for
+    the NHD layout the same logical tensors are stored as (B, N, H, d).
+    """
+    if w.dist not in ("normal", "normal_koffset", "normal_koutlier", "uniform2"):
+        raise ValueError(f"unknown value recipe {w.dist!r}")
+    q = _draw(w, STREAM_Q, (w.B, w.Hq, w.N, w.d))
+    k = _draw(w, STREAM_K, (w.B, w.Hkv, w.N, w.d))
+    v = _draw(w, STREAM_V, (w.B, w.Hkv, w.N, w.d))
+    if w.dist == "normal_koffset":
+        off = torch.randn((w.d,), generator=_gen(w, STREAM_OFFSET), dtype=torch.float32) * 3.0
+        k += off
+    elif w.dist == "normal_koutlier":
+        n_out = max(1, round(0.01 * w.Hkv * w.d))
+        pick = torch.randperm(w.Hkv * w.d, generator=_gen(w, STREAM_OUTLIER))[:n_out]
+        for p in pick.tolist():
+            k[:, p // w.d, :, p % w.d] *= 8.0
+    dt = DTYPES[w.dtype]
+    out = []
+    for t in (q, k, v):
+        t = t.to(dt)
+        if w.layout == "NHD":
+            t = t.transpose(1, 2)
+        out.append(t.contiguous())
+    return tuple(out)
+
+
+def sm_scale_of(w: Workload) -> float:
+    return w.sm_scale if w.sm_scale is not None else 1.0 / (w.d ** 0.5)
