@@ -1,0 +1,312 @@
+"""Throughput of the quantized attention path on B200, one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+A step is one pass of the whole path over one batch of synthetic input:
+the quantize/smooth pass plus the fused INT8-QK / FP8-PV attention kernel
+(``sage_attn``).  The default workload is the image-DiT self-attention shape
+B=2, H=24, N=4096, d=64, bf16, HND, non-causal, K with a per-channel offset.
+
+* ``value``: whole-job attention TOPS, 4*B*Hq*N^2*d (halved under the causal
+  mask) per step, inputs resident in HBM, per-step CUDA events with an L2
+  flush between steps (outside the events), max over ranks.
+* ``roofline``: the fused attention kernel alone (sage_attn_quantized on the
+  same buffers, per-launch CUDA events, L2 flushed) against the dense INT8/FP8
+  tensor peak (2x the measured bf16 cuBLAS peak, the B200 nominal ratio).
+* ``e2e``: the same metric through the public API with pinned HOST buffers:
+  H2D of q, k, v and D2H of the output inside the timed region.
+* ``cpu_baseline``: the CPU oracle (exact fp64 attention) on a bounded sample
+  of the same workload's heads, on this host's cores.
+* ``--impl reference``: there is no reference implementation to run; the
+  reference arm times the CPU oracle on the same workload instead.
+
+Multi-GPU (torchrun): replicas only, one independent copy of the workload per
+rank, no collective on the data path (weak scaling).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads as W  # noqa: E402
+
+METRIC = "attention TOPS on 1 B200 (N=1K-32K, d=64/128) and % of dense INT8/FP8 tensor peak"
+DEFAULT_WORKLOAD = W.IMAGE_DIT.name
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            m = json.load(f)
+        return dict(bf16=float(m["bf16_tflops"]), bf16_sustained=float(m["bf16_tflops_sustained"]),
+                    hbm=float(m["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+# ------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.dev = device_index
+        self.out_path = os.path.join("/tmp", f"sage_clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            self.f = open(self.out_path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "100",
+                 "-i", str(self.dev)], stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        for line in open(self.out_path):
+            p = [x.strip() for x in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(p[1]), smax=float(p[2]), power=float(p[3]), hw=p[5], hwt=p[6],
+                                 swt=p[7], pcap=p[8]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        load = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in rows:
+            for key, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"), ("swt", "sw_thermal_slowdown"),
+                              ("pcap", "sw_power_cap")):
+                if r[key].lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(r["sm"] for r in load), "sm_max_mhz": max(r["smax"] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows), "samples_under_load": len(load)}
+
+
+# ------------------------------------------------------------------------------------ timing
+def _flush(buf):
+    buf.add_(1)
+
+
+def time_steps(fn, steps, warmup, flush_buf):
+    """Per-step CUDA events on the current stream, L2 flushed before every step."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        _flush(flush_buf)
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        _flush(flush_buf)
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def cpu_oracle_sample(w: W.Workload, budget_s: float):
+    """Exact fp64 attention (the oracle) on successive (b, hq) heads until the time budget is used."""
+    from oracle import attention
+    from oracle.quant import to_hnd
+    q, k, v = W.make_inputs(w.with_(B=1))
+    qf, kf, vf = (to_hnd(t, w.layout) for t in (q, k, v))
+    G = w.Hq // w.Hkv
+    heads, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < budget_s and heads < w.Hq:
+        attention.attention_f64(qf[:, heads:heads + 1], kf[:, heads // G:heads // G + 1],
+                                vf[:, heads // G:heads // G + 1], "HND", w.causal, W.sm_scale_of(w))
+        heads += 1
+    dt = time.perf_counter() - t0
+    ops = w.with_(B=1, Hq=heads, Hkv=heads).ops()
+    try:
+        import threadpoolctl
+        threads = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count()
+    return ops / dt / 1e12, threads, heads, dt
+
+
+# ------------------------------------------------------------------------------------ arms
+def run_reference(args, w):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    budget = 8.0
+    vals = []
+    for i in range(args.warmup + args.steps):
+        tops, threads, heads, dt = cpu_oracle_sample(w, budget / max(1, args.steps))
+        if i >= args.warmup:
+            vals.append((tops, heads, dt))
+    v = statistics.median(t for t, _, _ in vals)
+    ms = statistics.mean(dt for _, _, dt in vals) * 1e3
+    line = {
+        "impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": _config(w),
+        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                         "sample": f"exact fp64 attention of {vals[-1][1]} (b=0, hq) head(s) of the workload per step"},
+        "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "no reference implementation exists for this path; the reference arm is the CPU oracle",
+    }
+    print(json.dumps(line), flush=True)
+
+
+def _config(w):
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "io_dtype": w.dtype,
+            "layout": w.layout, "causal": w.causal, "pv_accum": "fp32" if w.pv_mode == 0 else "fp16+fp32",
+            "values": w.dist, "l2": "flushed between steps (256 MiB write outside the events)"}
+
+
+def run_ours(args, w):
+    import quantized_attention_int8_b200 as qa
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if not qa.sage_device_supported():
+        raise SystemExit("this device is not a B200 (compute capability 10.0)")
+    pv = "fp32" if w.pv_mode == 0 else "fp16+fp32"
+    scale = W.sm_scale_of(w)
+    q, k, v = W.make_inputs(w)
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.empty_like(qd)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    ops = w.ops()
+
+    # ---- whole path (quantize + attention), device-resident inputs
+    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        times = time_steps(step, args.steps, args.warmup, flush)
+    qa.sage_check_status()
+    total_ms = sum(times)
+    if dist:
+        t = torch.tensor([total_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
+
+    # ---- the fused attention kernel alone (roofline)
+    z = qa.sage_quantize(qd, kd, vd, w.layout, pv)
+    kern = lambda: qa.sage_attn_quantized(z, qd.dtype, w.layout, w.causal, scale, pv, out=out)
+    ktimes = time_steps(kern, args.steps, args.warmup, flush)
+    qa.sage_check_status()
+    k_ms = statistics.mean(ktimes)
+    peaks = _peaks()
+    peak_tops = 2.0 * peaks["bf16"]
+    achieved = ops / (k_ms * 1e-3) / 1e12
+
+    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element
+    qtimes = time_steps(lambda: qa.sage_quantize(qd, kd, vd, w.layout, pv), max(3, args.steps // 2), 2, flush)
+    q_ms = statistics.mean(qtimes)
+    q_bytes = 3 * (q.numel() + k.numel() + v.numel())
+
+    # ---- end to end through the public API with pinned host buffers
+    qh, kh, vh = (t.pin_memory() for t in (q, k, v))
+    outh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+
+    def e2e_step():
+        a = qh.to("cuda", non_blocking=True)
+        b = kh.to("cuda", non_blocking=True)
+        c = vh.to("cuda", non_blocking=True)
+        o = qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv)
+        outh.copy_(o, non_blocking=True)
+
+    etimes = time_steps(e2e_step, args.steps, args.warmup, flush)
+    e_ms = sum(etimes)
+    if dist:
+        t = torch.tensor([e_ms], device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e_ms = float(t.item())
+    e2e_value = world * ops * args.steps / (e_ms * 1e-3) / 1e12
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1:
+            tops, threads, heads, dt = cpu_oracle_sample(w, 12.0)
+            cpu = {"value": tops, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                   "sample": f"exact fp64 attention of {heads} (b=0, hq) head(s), {dt:.1f} s"}
+        line = {
+            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8+f8e4m3", "data": "synthetic",
+            "config": _config(w),
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
+                         "frac": achieved / peak_tops, "traffic": None,
+                         "kernel": "sage_fwd_kernel", "kernel_ms": k_ms,
+                         "peak_source": f"2 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s "
+                                        "(dense INT8/FP8 = 2x bf16 on B200)"},
+            "quantize": {"ms": q_ms, "algorithmic_bytes": q_bytes, "GB_per_s": q_bytes / (q_ms * 1e-3) / 1e9,
+                         "hbm_peak_GB_per_s": peaks["hbm"], "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm"]},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": in_bytes,
+                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
+    w = W.BY_NAME[args.workload]
+    if args.impl == "reference":
+        run_reference(args, w)
+    else:
+        run_ours(args, w)
+
+
+if __name__ == "__main__":
+    main()

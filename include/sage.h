@@ -1,0 +1,133 @@
+/*
+ * sage.h -- C ABI of an INT8-QK / FP8-PV quantized attention library for
+ * NVIDIA B200 (sm_100a).
+ *
+ * The operation is scaled-dot-product attention
+ *     out = softmax(Q K^T * sm_scale [+ causal mask]) V
+ * computed the SageAttention way (SageAttention README, "Current Features"):
+ * K is smoothed by subtracting its per-channel token mean, Q and K are
+ * quantized to INT8 with one fp32 scale per 128-token block, Q K^T runs as an
+ * INT8 tensor-core product, the scores go through an online softmax, P is
+ * requantized to FP8 E4M3 and P V runs as an FP8 tensor-core product with
+ * fp32 accumulation or with the two-level fp16+fp32 accumulation.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers owned by the caller.  The library
+ *    never keeps a pointer after the call returns; work is queued on `stream`
+ *    (a cudaStream_t; NULL = the legacy default stream) and may still be
+ *    running when the call returns.
+ *  - Q, K, V and out are dense and contiguous in the given layout
+ *    (SageAttention README, "How to Use", tensor_layout):
+ *        SAGE_HND: (B, H, N, d)      SAGE_NHD: (B, N, H, d)
+ *    with H = Hq for Q and out, H = Hkv for K and V.
+ *  - Inputs are fp16 or bf16 (fp32 is rejected with SAGE_ERR_UNSUPPORTED, as the
+ *    reference API only accepts 16-bit inputs); out has the input dtype.
+ *  - GQA: Hq must be a multiple of Hkv; query head h reads kv head
+ *    h / (Hq / Hkv) (qwbw.cn article, pitfalls section).
+ *  - head dim 1 <= d <= 256; internally it is zero-padded to dp = 64, 128 or
+ *    256, the smallest that holds d (same section, pad_qkv).
+ *  - Causal masking keeps key j for query i iff j <= i (Nq = Nk = N).
+ *  - Errors: argument checks run first and return without touching the GPU or
+ *    writing any output.  A CUDA launch or allocation failure returns
+ *    SAGE_ERR_CUDA / SAGE_ERR_OOM.  Kernel-side timeouts (every wait inside the
+ *    kernels is bounded) are reported later by sage_check_status().
+ *  - A device other than compute capability 10.0 (B200) returns SAGE_ERR_ARCH.
+ */
+#ifndef SAGE_B200_H_
+#define SAGE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,
+  SAGE_ERR_UNSUPPORTED = 2,
+  SAGE_ERR_ARCH = 3,
+  SAGE_ERR_CUDA = 4,
+  SAGE_ERR_OOM = 5,
+  SAGE_ERR_TIMEOUT = 6
+} sage_status;
+
+typedef enum { SAGE_HND = 0, SAGE_NHD = 1 } sage_layout;
+typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype;
+
+/* P.V accumulation (SageAttention README, "Current Features": FP16 accumulator
+ * for FP8 PV and two-level accumulation; qwbw.cn article, pitfalls:
+ * pv_accum_dtype = "fp32" | "fp16+fp32").
+ *   SAGE_PV_FP32      P8.V8 accumulates in fp32 across all key tiles.
+ *   SAGE_PV_FP16_FP32 each 128-key tile's P8.V8 goes to a fresh fp16
+ *                     accumulator, which is then added into an fp32 O.
+ *                     V codes then span [-1, 1] (instead of [-448, 448]) so
+ *                     one tile's fp16 partial (<= 128*448*1) cannot overflow. */
+typedef enum { SAGE_PV_FP32 = 0, SAGE_PV_FP16_FP32 = 1 } sage_pv_mode;
+
+/* Quantized attention, end to end: quantize/smooth pass, then the fused
+ * attention kernel.  q: (B,Hq,N,d), k and v: (B,Hkv,N,d), out: (B,Hq,N,d), all
+ * in `layout`, dtype `dtype`.  sm_scale <= 0 or NaN selects 1/sqrt(d) (the
+ * original d).  The quantized copies of Q/K/V live in a workspace taken with
+ * cudaMallocAsync on `stream` and released stream-ordered before return;
+ * SAGE_ERR_OOM if it cannot be allocated.  out must not overlap q, k or v. */
+sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
+                      sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
+                      void* stream);
+
+/* Bytes of workspace sage_attn takes for these sizes (0 on invalid sizes). */
+size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/* The quantize/smooth pass alone (K token mean, INT8 Q and K - mean(K) codes with
+ * per-128-token-block scales, E4M3 V codes with per-channel scales).  Outputs,
+ * with Np = 128 * ceil(N / 128) and dp the padded head dim, all device memory:
+ *   q8  int8   [B][Hq][Np][dp]     qs  fp32 [B][Hq][Np/128]
+ *   k8  int8   [B][Hkv][Np][dp]    ks  fp32 [B][Hkv][Np/128]    km fp32 [B][Hkv][dp]
+ *   v8t uint8  [B][Hkv][dp][Np]    E4M3 codes, transposed (keys contiguous)
+ *   vs  fp32   [B][Hkv][dp]
+ * Padded tokens and channels hold code 0 (and km 0, vs 0).  Codes and scales
+ * follow: amax over the block's real tokens and channels, inv = 127 / amax,
+ * code = clamp(rint_even(x * inv), -127, 127), scale = amax / 127 (0 when amax
+ * is 0); K is smoothed as x = k - km, km summed in fp32 block by block (tokens
+ * in order inside a block, then the block sums in order) and divided by N;
+ * V: inv = VMAX / amax_channel, code = E4M3_rne_satfinite(v * inv),
+ * vs = amax / VMAX with VMAX = 448 (SAGE_PV_FP32) or 1 (SAGE_PV_FP16_FP32).
+ * Its own small scratch is taken with cudaMallocAsync on `stream`. */
+sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
+                          sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,
+                          int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs, void* stream);
+
+/* The fused attention kernel alone, on buffers in the layouts sage_quantize
+ * writes.  out: (B,Hq,N,d) in `out_layout`, dtype `out_dtype`.  Allocates
+ * nothing. */
+sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t* k8, const float* ks,
+                                const uint8_t* v8t, const float* vs, void* out, int B, int Hq, int Hkv, int N,
+                                int d, sage_dtype out_dtype, sage_layout out_layout, int is_causal, float sm_scale,
+                                sage_pv_mode pv_mode, void* stream);
+
+/* Diagnostic: the exact int32 scores S = Q8 . K8^T of selected 128x128 tiles,
+ * computed by the same TMA + tcgen05 kind::i8 path as the fused kernel.
+ * tiles: DEVICE int32 array of n_tiles records {b, hq, q_tile, k_tile};
+ * s_out: DEVICE int32 [n_tiles][128][128], row = query, column = key.  q8/k8
+ * as written by sage_quantize.  Out-of-range records are skipped and flagged
+ * (sage_check_status returns SAGE_ERR_INVALID_ARG).  Allocates nothing. */
+sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int Hkv, int N, int d,
+                          const int32_t* tiles, int n_tiles, int32_t* s_out, void* stream);
+
+/* Synchronizes `stream`, then reports (and clears) the device-side error word:
+ * SAGE_ERR_TIMEOUT if a kernel gave up on a bounded wait, SAGE_ERR_INVALID_ARG
+ * for a flagged tile record, SAGE_ERR_CUDA for a pending CUDA error. */
+sage_status sage_check_status(void* stream);
+
+/* Static description of a status code. */
+const char* sage_status_string(sage_status s);
+
+/* 1 if the current CUDA device can run this library (compute capability 10.0). */
+int sage_device_supported(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SAGE_B200_H_ */

@@ -1,0 +1,205 @@
+"""INT8-QK / FP8-PV quantized attention for NVIDIA B200 (sm_100a).
+
+Thin Python binding over the C ABI in ``include/sage.h`` (``libsage_b200.so``,
+built in-tree by ``python -m quantized_attention_int8_b200.build_lib``).  The
+functions keep the C entry points' names and only marshal arguments: torch
+supplies device memory and the current CUDA stream, and every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback: if
+the library is missing, importing this package fails.
+
+    from quantized_attention_int8_b200 import sage_attn
+    out = sage_attn(q, k, v, tensor_layout="HND", is_causal=False)
+
+mirrors the ``sageattn(q, k, v, tensor_layout, is_causal, sm_scale)`` call of
+the SageAttention README ("How to Use"); ``pv_accum_dtype`` selects "fp32" or
+"fp16+fp32" accumulation of the FP8 P.V product (qwbw.cn article, pitfalls).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
+    "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
+
+SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_ARCH, SAGE_ERR_CUDA, SAGE_ERR_OOM, \
+    SAGE_ERR_TIMEOUT = range(7)
+SAGE_HND, SAGE_NHD = 0, 1
+SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
+SAGE_PV_FP32, SAGE_PV_FP16_FP32 = 0, 1
+
+_LAYOUTS = {"HND": SAGE_HND, "NHD": SAGE_NHD}
+_DTYPES = {torch.float16: SAGE_FP16, torch.bfloat16: SAGE_BF16, torch.float32: SAGE_FP32}
+_PV = {"fp32": SAGE_PV_FP32, "fp16+fp32": SAGE_PV_FP16_FP32}
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is not built; run `python -m quantized_attention_int8_b200.build_lib` "
+            "(this package has no CPU fallback)")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+    sig = {
+        "sage_attn": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
+        "sage_workspace_bytes": ([I, I, I, I, I], Z),
+        "sage_quantize": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P], I),
+        "sage_attn_quantized": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
+        "sage_qk_int32": ([P, P, I, I, I, I, I, P, I, P, P], I),
+        "sage_check_status": ([P], I),
+        "sage_status_string": ([I], ctypes.c_char_p),
+        "sage_device_supported": ([], I),
+    }
+    for name, (args, res) in sig.items():
+        fn = getattr(lib, name)
+        fn.argtypes, fn.restype = args, res
+    return lib
+
+
+capi = _load()
+
+
+class SageError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {sage_status_string(status)} (status {status})")
+
+
+def sage_status_string(status: int) -> str:
+    return capi.sage_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str) -> None:
+    if status != SAGE_OK:
+        raise SageError(status, where)
+
+
+def _stream() -> int:
+    return torch.cuda.current_stream().cuda_stream
+
+
+def _ptr(t: torch.Tensor | None) -> int | None:
+    return None if t is None else t.data_ptr()
+
+
+def padded_dim(d: int) -> int:
+    if d > 256:
+        raise ValueError("head_dim > 256 is not supported")
+    return 64 if d <= 64 else (128 if d <= 128 else 256)
+
+
+def _shape(q: torch.Tensor, k: torch.Tensor, layout: str):
+    if q.dim() != 4 or k.dim() != 4:
+        raise ValueError("q, k, v must be 4-D")
+    if layout == "HND":
+        B, Hq, N, d = q.shape
+        Hkv = k.shape[1]
+    elif layout == "NHD":
+        B, N, Hq, d = q.shape
+        Hkv = k.shape[2]
+    else:
+        raise ValueError(f"tensor_layout must be 'HND' or 'NHD', got {layout!r}")
+    return B, Hq, Hkv, N, d
+
+
+def _check_inputs(q, k, v, layout):
+    for t in (q, k, v):
+        if not t.is_cuda:
+            raise ValueError("q, k, v must be CUDA tensors (no CPU path exists)")
+        if not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share one dtype")
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    B, Hq, Hkv, N, d = _shape(q, k, layout)
+    kshape = (B, Hkv, N, d) if layout == "HND" else (B, N, Hkv, d)
+    if tuple(k.shape) != kshape:
+        raise ValueError(f"k has shape {tuple(k.shape)}, expected {kshape}")
+    return B, Hq, Hkv, N, d
+
+
+def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None):
+    """Quantized attention of fp16/bf16 q (B,Hq,N,d), k/v (B,Hkv,N,d) (HND; NHD stores (B,N,H,d))."""
+    B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    if out is None:
+        out = torch.empty_like(q)
+    st = capi.sage_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
+                        _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)),
+                        float(sm_scale) if sm_scale is not None else 0.0, _PV[pv_accum_dtype], _stream())
+    _check(st, "sage_attn")
+    return out
+
+
+def sage_workspace_bytes(B, Hq, Hkv, N, d) -> int:
+    return int(capi.sage_workspace_bytes(B, Hq, Hkv, N, d))
+
+
+def sage_quantize(q, k, v, tensor_layout="HND", pv_accum_dtype="fp32") -> dict:
+    """The quantize/smooth pass alone; returns the codes and scales as CUDA tensors.
+
+    Layouts (Np = 128*ceil(N/128), dp = padded head dim): q8 int8 (B,Hq,Np,dp),
+    qs f32 (B,Hq,Np/128), k8 int8 (B,Hkv,Np,dp), ks f32 (B,Hkv,Np/128),
+    km f32 (B,Hkv,dp), v8t uint8 E4M3 (B,Hkv,dp,Np), vs f32 (B,Hkv,dp).
+    """
+    B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
+    dp, nb = padded_dim(d), (N + 127) // 128
+    Np = nb * 128
+    dev = q.device
+    z = dict(
+        q8=torch.empty((B, Hq, Np, dp), dtype=torch.int8, device=dev),
+        qs=torch.empty((B, Hq, nb), dtype=torch.float32, device=dev),
+        k8=torch.empty((B, Hkv, Np, dp), dtype=torch.int8, device=dev),
+        ks=torch.empty((B, Hkv, nb), dtype=torch.float32, device=dev),
+        km=torch.empty((B, Hkv, dp), dtype=torch.float32, device=dev),
+        v8t=torch.empty((B, Hkv, dp, Np), dtype=torch.uint8, device=dev),
+        vs=torch.empty((B, Hkv, dp), dtype=torch.float32, device=dev),
+    )
+    st = capi.sage_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d, _DTYPES[q.dtype],
+                            _LAYOUTS[tensor_layout], _PV[pv_accum_dtype], *(z[n].data_ptr() for n in
+                                                                          ("q8", "qs", "k8", "ks", "km", "v8t", "vs")),
+                            _stream())
+    _check(st, "sage_quantize")
+    z.update(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d)
+    return z
+
+
+def sage_attn_quantized(z: dict, out_dtype=torch.float16, tensor_layout="HND", is_causal=False, sm_scale=None,
+                        pv_accum_dtype="fp32", out=None):
+    """The fused attention kernel alone on quantized buffers (the dict sage_quantize returns)."""
+    B, Hq, Hkv, N, d = (z[n] for n in ("B", "Hq", "Hkv", "N", "d"))
+    if out is None:
+        shape = (B, Hq, N, d) if tensor_layout == "HND" else (B, N, Hq, d)
+        out = torch.empty(shape, dtype=out_dtype, device=z["q8"].device)
+    st = capi.sage_attn_quantized(*(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "v8t", "vs")),
+                                  out.data_ptr(), B, Hq, Hkv, N, d, _DTYPES[out.dtype], _LAYOUTS[tensor_layout],
+                                  int(bool(is_causal)), float(sm_scale) if sm_scale is not None else 0.0,
+                                  _PV[pv_accum_dtype], _stream())
+    _check(st, "sage_attn_quantized")
+    return out
+
+
+def sage_qk_int32(z: dict, tiles) -> torch.Tensor:
+    """int32 Q8.K8^T of 128x128 tiles; tiles = list of (b, hq, q_tile, k_tile)."""
+    t = torch.as_tensor(tiles, dtype=torch.int32).reshape(-1, 4).to(z["q8"].device).contiguous()
+    out = torch.empty((t.shape[0], 128, 128), dtype=torch.int32, device=z["q8"].device)
+    st = capi.sage_qk_int32(z["q8"].data_ptr(), z["k8"].data_ptr(), z["B"], z["Hq"], z["Hkv"], z["N"], z["d"],
+                            t.data_ptr(), t.shape[0], out.data_ptr(), _stream())
+    _check(st, "sage_qk_int32")
+    return out
+
+
+def sage_check_status() -> None:
+    _check(capi.sage_check_status(_stream()), "sage_check_status")
+
+
+def sage_device_supported() -> bool:
+    return bool(capi.sage_device_supported())

@@ -1,0 +1,313 @@
+// C ABI: argument checks, workspace, TMA tensor maps and launches.
+// The operation and the argument contract are documented in include/sage.h.
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "sage_internal.h"
+
+using namespace sage;
+
+namespace {
+
+constexpr size_t kAlign = 1024;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+int padded_dim(int d) { return d <= 64 ? 64 : (d <= 128 ? 128 : 256); }
+
+struct Dims {
+  int B, Hq, Hkv, N, d, dp, Np, nblk, G;
+};
+
+sage_status check_dims(int B, int Hq, int Hkv, int N, int d, Dims* out) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1) return SAGE_ERR_INVALID_ARG;
+  if (d > 256 || Hq % Hkv != 0) return SAGE_ERR_INVALID_ARG;
+  if (B > 65535 || 2L * Hq > 65535 || (long)Hq + 2L * Hkv > 65535 || N > (1 << 30)) return SAGE_ERR_INVALID_ARG;
+  Dims m;
+  m.B = B, m.Hq = Hq, m.Hkv = Hkv, m.N = N, m.d = d;
+  m.dp = padded_dim(d);
+  m.nblk = (N + 127) / 128;
+  m.Np = m.nblk * 128;
+  m.G = Hq / Hkv;
+  // TMA coordinates are 32-bit signed
+  if ((long long)B * Hq * m.Np >= (1LL << 31) || (long long)B * Hkv * m.dp >= (1LL << 31)) return SAGE_ERR_INVALID_ARG;
+  *out = m;
+  return SAGE_OK;
+}
+
+sage_status check_dtype(int dtype) {
+  if (dtype == SAGE_FP32) return SAGE_ERR_UNSUPPORTED;
+  if (dtype != SAGE_FP16 && dtype != SAGE_BF16) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+bool overlaps(const void* a, size_t na, const void* b, size_t nb) {
+  const uintptr_t x = (uintptr_t)a, y = (uintptr_t)b;
+  return x < y + nb && y < x + na;
+}
+
+sage_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return SAGE_OK;
+  return e == cudaErrorMemoryAllocation ? SAGE_ERR_OOM : SAGE_ERR_CUDA;
+}
+
+sage_status check_device() {
+  int dev = 0, major = 0, minor = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  return (major == 10 && minor == 0) ? SAGE_OK : SAGE_ERR_ARCH;
+}
+
+float resolve_scale(float sm_scale, int d) {
+  if (!(sm_scale > 0.f) || std::isnan(sm_scale)) return 1.0f / std::sqrt((float)d);
+  return sm_scale;
+}
+
+// ---------------------------------------------------------------------------------- tensor maps
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D byte tensor: `inner` bytes per row (contiguous), `rows` rows, box {box_inner, box_rows}.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, uint32_t box_inner, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {inner, rows};
+  const cuuint64_t strides[1] = {inner};
+  const cuuint32_t box[2] = {box_inner, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapSwizzle swz = box_inner == 128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B;
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
+
+struct QuantBufs {
+  int8_t* q8;
+  float* qs;
+  int8_t* k8;
+  float* ks;
+  float* km;
+  uint8_t* v8t;
+  float* vs;
+};
+
+sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, int layout, int causal, float sm_scale,
+                    int pv_mode, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
+  const uint32_t ksub = m.dp >= 128 ? 128 : 64;
+  const uint32_t dv = m.dp == 64 ? 64 : 128;
+  if (!make_map(&tq, qb.q8, m.dp, (uint64_t)m.B * m.Hq * m.Np, ksub, 128) ||
+      !make_map(&tk, qb.k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, 128) ||
+      !make_map(&tv, qb.v8t, m.Np, (uint64_t)m.B * m.Hkv * m.dp, 128, dv))
+    return SAGE_ERR_CUDA;
+  FwdParams p;
+  p.qs = qb.qs, p.ks = qb.ks, p.vs = qb.vs, p.out = out;
+  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.N = m.N, p.Np = m.Np, p.nblk = m.nblk, p.d = m.d, p.dp = m.dp, p.G = m.G;
+  p.layout = layout;
+  p.n_vhalves = m.dp == 256 ? 2 : 1;
+  p.vec_out = (m.d % 8 == 0) && aligned16(out);
+  p.scale_log2 = resolve_scale(sm_scale, m.d) * 1.4426950408889634f;
+  return from_cuda(launch_fwd(tq, tk, tv, p, dtype, causal, pv_mode, st));
+}
+
+struct WsLayout {
+  size_t q8, qs, k8, ks, km, v8t, vs, ksum, vmax, vinv, total;
+};
+
+WsLayout ws_layout(const Dims& m) {
+  WsLayout w;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + bytes);
+    return o;
+  };
+  w.q8 = take((size_t)m.B * m.Hq * m.Np * m.dp);
+  w.qs = take((size_t)m.B * m.Hq * m.nblk * 4);
+  w.k8 = take((size_t)m.B * m.Hkv * m.Np * m.dp);
+  w.ks = take((size_t)m.B * m.Hkv * m.nblk * 4);
+  w.km = take((size_t)m.B * m.Hkv * m.dp * 4);
+  w.v8t = take((size_t)m.B * m.Hkv * m.dp * m.Np);
+  w.vs = take((size_t)m.B * m.Hkv * m.dp * 4);
+  w.ksum = take((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
+  w.vmax = take((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
+  w.vinv = take((size_t)m.B * m.Hkv * m.dp * 4);
+  w.total = off;
+  return w;
+}
+
+QuantParams quant_params(const Dims& m, const void* q, const void* k, const void* v, int dtype, int layout,
+                         int pv_mode) {
+  QuantParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = q, p.k = k, p.v = v;
+  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.N = m.N, p.d = m.d, p.dp = m.dp, p.Np = m.Np, p.nblk = m.nblk;
+  p.layout = layout, p.dtype = dtype;
+  p.vec_q = (m.d % 8 == 0) && aligned16(q);
+  p.vec_k = (m.d % 8 == 0) && aligned16(k);
+  p.vec_v = (m.d % 8 == 0) && aligned16(v);
+  p.vmax_code = pv_mode == SAGE_PV_FP16_FP32 ? 1.0f : 448.0f;
+  return p;
+}
+
+sage_status check_common(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
+                         int dtype, int layout, int pv_mode, Dims* m) {
+  if (!q || !k || !v) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_dtype(dtype);
+  if (s != SAGE_OK) return s;
+  if (layout != SAGE_HND && layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
+  if (pv_mode != SAGE_PV_FP32 && pv_mode != SAGE_PV_FP16_FP32) return SAGE_ERR_INVALID_ARG;
+  return check_dims(B, Hq, Hkv, N, d, m);
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  Dims m;
+  if (check_dims(B, Hq, Hkv, N, d, &m) != SAGE_OK) return 0;
+  return ws_layout(m).total;
+}
+
+sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
+                      sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
+                      void* stream) {
+  Dims m;
+  sage_status s = check_common(q, k, v, B, Hq, Hkv, N, d, dtype, layout, pv_mode, &m);
+  if (s != SAGE_OK) return s;
+  if (!out) return SAGE_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
+  if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes))
+    return SAGE_ERR_INVALID_ARG;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const WsLayout w = ws_layout(m);
+  unsigned char* ws = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
+  QuantBufs qb{reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
+               reinterpret_cast<int8_t*>(ws + w.k8), reinterpret_cast<float*>(ws + w.ks),
+               reinterpret_cast<float*>(ws + w.km), ws + w.v8t, reinterpret_cast<float*>(ws + w.vs)};
+  qp.q8 = qb.q8, qp.qs = qb.qs, qp.k8 = qb.k8, qp.ks = qb.ks, qp.km = qb.km, qp.v8t = qb.v8t, qp.vs = qb.vs;
+  qp.ksum_part = reinterpret_cast<float*>(ws + w.ksum);
+  qp.vmax_part = reinterpret_cast<float*>(ws + w.vmax);
+  qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
+  s = from_cuda(launch_quantize(qp, st));
+  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
+  return s;
+}
+
+sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
+                          sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,
+                          int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs, void* stream) {
+  Dims m;
+  sage_status s = check_common(q, k, v, B, Hq, Hkv, N, d, dtype, layout, pv_mode, &m);
+  if (s != SAGE_OK) return s;
+  if (!q8 || !qs || !k8 || !ks || !km || !v8t || !vs) return SAGE_ERR_INVALID_ARG;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_device()) != SAGE_OK) return s;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t part = align_up((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
+  const size_t vinv = align_up((size_t)m.B * m.Hkv * m.dp * 4);
+  unsigned char* scratch = nullptr;
+  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&scratch), 2 * part + vinv, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
+  qp.q8 = q8, qp.qs = qs, qp.k8 = k8, qp.ks = ks, qp.km = km, qp.v8t = v8t, qp.vs = vs;
+  qp.ksum_part = reinterpret_cast<float*>(scratch);
+  qp.vmax_part = reinterpret_cast<float*>(scratch + part);
+  qp.vinv = reinterpret_cast<float*>(scratch + 2 * part);
+  s = from_cuda(launch_quantize(qp, st));
+  const cudaError_t ef = cudaFreeAsync(scratch, st);
+  if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
+  return s;
+}
+
+sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t* k8, const float* ks,
+                                const uint8_t* v8t, const float* vs, void* out, int B, int Hq, int Hkv, int N,
+                                int d, sage_dtype out_dtype, sage_layout out_layout, int is_causal, float sm_scale,
+                                sage_pv_mode pv_mode, void* stream) {
+  if (!q8 || !qs || !k8 || !ks || !v8t || !vs || !out) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_dtype(out_dtype);
+  if (s != SAGE_OK) return s;
+  if (out_layout != SAGE_HND && out_layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
+  if (pv_mode != SAGE_PV_FP32 && pv_mode != SAGE_PV_FP16_FP32) return SAGE_ERR_INVALID_ARG;
+  Dims m;
+  if ((s = check_dims(B, Hq, Hkv, N, d, &m)) != SAGE_OK) return s;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_device()) != SAGE_OK) return s;
+  QuantBufs qb{const_cast<int8_t*>(q8), const_cast<float*>(qs), const_cast<int8_t*>(k8), const_cast<float*>(ks),
+               nullptr, const_cast<uint8_t*>(v8t), const_cast<float*>(vs)};
+  return run_fwd(m, qb, out, out_dtype, out_layout, is_causal ? 1 : 0, sm_scale, pv_mode,
+                 static_cast<cudaStream_t>(stream));
+}
+
+sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int Hkv, int N, int d,
+                          const int32_t* tiles, int n_tiles, int32_t* s_out, void* stream) {
+  if (!q8 || !k8 || !tiles || !s_out || n_tiles < 0) return SAGE_ERR_INVALID_ARG;
+  Dims m;
+  sage_status s = check_dims(B, Hq, Hkv, N, d, &m);
+  if (s != SAGE_OK) return s;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(s_out)) return SAGE_ERR_INVALID_ARG;
+  if (n_tiles == 0) return SAGE_OK;
+  if ((s = check_device()) != SAGE_OK) return s;
+  CUtensorMap tq, tk;
+  const uint32_t ksub = m.dp >= 128 ? 128 : 64;
+  if (!make_map(&tq, q8, m.dp, (uint64_t)m.B * m.Hq * m.Np, ksub, 128) ||
+      !make_map(&tk, k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, 128))
+    return SAGE_ERR_CUDA;
+  QkDumpParams p;
+  p.tiles = tiles, p.n_tiles = n_tiles, p.out = s_out;
+  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.Np = m.Np, p.nblk = m.nblk, p.G = m.G;
+  return from_cuda(launch_qk_dump(tq, tk, p, m.dp, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_check_status(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return SAGE_ERR_CUDA;
+  int flags = 0;
+  if (read_clear_device_error(&flags) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (flags & 1) return SAGE_ERR_TIMEOUT;
+  if (flags & 2) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+const char* sage_status_string(sage_status s) {
+  switch (s) {
+    case SAGE_OK: return "ok";
+    case SAGE_ERR_INVALID_ARG: return "invalid argument";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported (inputs must be fp16 or bf16)";
+    case SAGE_ERR_ARCH: return "device is not compute capability 10.0 (B200, sm_100a)";
+    case SAGE_ERR_CUDA: return "CUDA error";
+    case SAGE_ERR_OOM: return "out of device memory";
+    case SAGE_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+  }
+  return "unknown status";
+}
+
+int sage_device_supported(void) { return check_device() == SAGE_OK ? 1 : 0; }
+
+}  // extern "C"

@@ -1,0 +1,555 @@
+// Fused INT8-QK / FP8-PV attention for sm_100a (tcgen05 + TMA + TMEM).
+//
+// One CTA computes one 128-row query tile of one (batch, query head) and, when
+// the padded head dim is 256, one 128-column half of the output.  Six warps:
+//
+//   warps 0-3  softmax / correction / epilogue; thread t owns query row t
+//              (TMEM lane t), so row max and row sum need no shuffles;
+//   warp 4     TMA producer: Q once, then K and V^T tiles through an
+//              ST-deep ring of shared-memory stages;
+//   warp 5     TMEM allocator and UMMA issuer (one elected thread).
+//
+// Per 128-key tile j (the blockwise online softmax of the method):
+//   S_j  = Q8 . K8_j^T                    tcgen05.mma kind::i8 -> int32 in TMEM
+//   s    = S_j * (qs * ks_j * sm_scale * log2 e), causal / length mask
+//   m'   = max(m, rowmax s), p = 2^(s - m'), alpha = 2^(m - m'), l = l alpha + sum p
+//   P8   = E4M3(p * 448)                  written to shared memory (128B swizzle)
+//   mode 0 (fp32 accumulation):  O = O * alpha (in TMEM) ; O += P8 . V8_j   (kind::f8f6f4, f32)
+//   mode 1 (fp16+fp32):          T = P8 . V8_j (fresh f16 accumulator) ; O = O * alpha + T
+//   out  = O * v_scale / (448 * l)
+//
+// Method: SageAttention README ("Current Features": INT8 QK^T with smoothing,
+// FP8 PV, FP16 accumulator for FP8 PV, two-level accumulation) and the qwbw.cn
+// article (pitfalls: pv_accum_dtype fp32 / fp16+fp32).  The kernel design
+// (tcgen05, TMEM accumulators, TMA ring, warp roles) is this library's own.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+
+#include <climits>
+
+#include "sage_internal.h"
+#include "sm100.cuh"
+
+namespace sage {
+
+template <int DQK, int DV>
+struct FwdCfg {
+  static constexpr int KSUB = DQK >= 128 ? 128 : 64;  // bytes per row of one Q/K sub-tile (= swizzle span)
+  static constexpr int NSUB = DQK / KSUB;
+  static constexpr int Q_BYTES = 128 * DQK;
+  static constexpr int K_BYTES = 128 * DQK;
+  static constexpr int V_BYTES = DV * 128;
+  static constexpr int P_BYTES = 128 * 128;
+  static constexpr int ST = DQK == 64 ? 4 : 3;
+  static constexpr int BAR_BYTES = 256;
+  static constexpr int SMEM = 1024 + Q_BYTES + ST * (K_BYTES + V_BYTES) + 2 * P_BYTES + BAR_BYTES;
+  static constexpr uint32_t TMEM_COLS = 512;
+  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, T_COL = 256 + DV;
+  static_assert(T_COL + DV <= TMEM_COLS, "TMEM plan");
+  static_assert(SMEM <= 227 * 1024, "shared memory plan");
+};
+
+struct FwdBars {
+  uint64_t q_full;
+  uint64_t k_full[4], v_full[4], kv_empty[4];
+  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort;
+};
+
+template <typename OutT>
+__device__ __forceinline__ uint32_t pack2(float a, float b);
+template <>
+__device__ __forceinline__ uint32_t pack2<__half>(float a, float b) {
+  __half2 h = __floats2half2_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+template <>
+__device__ __forceinline__ uint32_t pack2<__nv_bfloat16>(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+__device__ __forceinline__ void store_elem(__half* p, float v) { *p = __float2half_rn(v); }
+__device__ __forceinline__ void store_elem(__nv_bfloat16* p, float v) { *p = __float2bfloat16_rn(v); }
+
+// Warp-uniform bounded wait: every lane waits, and the warp proceeds only if all did.
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  const bool ok = mbar_wait(bar, parity, abort);
+  return __all_sync(0xffffffffu, ok);
+}
+
+// Bounded wait used only while winding down (ignores the abort flag).
+__device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitBudgetCycles) {
+      atomicOr(&g_device_error, SAGE_DEVERR_TIMEOUT);
+      return;
+    }
+  }
+}
+
+template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
+__global__ void __launch_bounds__(192, 1)
+    sage_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                    const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<DQK, DV>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sbase = smem_raw + pad;
+  unsigned char* sQ = sbase;
+  unsigned char* sK = sQ + C::Q_BYTES;
+  unsigned char* sV = sK + C::ST * C::K_BYTES;
+  unsigned char* sP = sV + C::ST * C::V_BYTES;
+  FwdBars* bars = reinterpret_cast<FwdBars*>(sP + 2 * C::P_BYTES);
+  volatile int* abort = &bars->abort;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int qt = blockIdx.x;
+  if (CAUSAL) qt = p.nblk - 1 - qt;  // longest rows first
+  const int hq = blockIdx.y / p.n_vhalves, vh = blockIdx.y - hq * p.n_vhalves;
+  const int b = blockIdx.z;
+  const int hkv = hq / p.G;
+  const int n_kv = CAUSAL ? qt + 1 : p.nblk;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    for (int s = 0; s < C::ST; ++s) {
+      mbar_init(&bars->k_full[s], 1);
+      mbar_init(&bars->v_full[s], 1);
+      mbar_init(&bars->kv_empty[s], 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&bars->s_full[s], 1);
+      mbar_init(&bars->s_empty[s], 4);
+      mbar_init(&bars->p_full[s], 4);
+      mbar_init(&bars->pv_done[s], 1);
+    }
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 4) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const int q_row = (b * p.Hq + hq) * p.Np + qt * 128;
+      const int k_row = (b * p.Hkv + hkv) * p.Np;
+      const int v_row = (b * p.Hkv + hkv) * p.dp + vh * DV;
+      mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
+      for (int s = 0; s < C::NSUB; ++s) tma_load_2d(sQ + s * 128 * C::KSUB, &tmQ, &bars->q_full, s * C::KSUB, q_row);
+      int issued = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % C::ST, u = j / C::ST;
+        if (!mbar_wait(&bars->kv_empty[st], (u & 1) ^ 1, abort)) break;
+        mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
+        for (int s = 0; s < C::NSUB; ++s)
+          tma_load_2d(sK + st * C::K_BYTES + s * 128 * C::KSUB, &tmK, &bars->k_full[st], s * C::KSUB, k_row + j * 128);
+        mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
+        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], j * 128, v_row);
+        issued = j + 1;
+      }
+      // make sure no copy is still landing in shared memory when the CTA exits
+      drain_wait(&bars->q_full, 0);
+      for (int j = issued - C::ST < 0 ? 0 : issued - C::ST; j < issued; ++j) {
+        drain_wait(&bars->k_full[j % C::ST], (j / C::ST) & 1);
+        drain_wait(&bars->v_full[j % C::ST], (j / C::ST) & 1);
+      }
+    }
+  } else if (warp == 5) {
+    // ------------------------------------------------------------------ UMMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*S8*/, 128, 128);
+      constexpr uint32_t idesc_pv = make_idesc(MODE == 0 ? 1 /*F32*/ : 0 /*F16*/, 0 /*E4M3*/, 128, DV);
+      const uint32_t pv_dst = tmem + (MODE == 0 ? C::O_COL : C::T_COL);
+      auto issue_pv = [&](int i) -> bool {
+        const int st = i % C::ST, pb = i & 1;
+        if (!mbar_wait(&bars->v_full[st], (i / C::ST) & 1, abort)) return false;
+        if (!mbar_wait(&bars->p_full[pb], (i >> 1) & 1, abort)) return false;
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sP + pb * C::P_BYTES), va = smem_u32(sV + st * C::V_BYTES);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t acc = MODE == 0 ? (uint32_t)(i > 0 || k > 0) : (uint32_t)(k > 0);
+          umma_f8(pv_dst, smem_desc_kmajor(pa + k * 32, 128), smem_desc_kmajor(va + k * 32, 128), idesc_pv, acc);
+        }
+        umma_commit(&bars->kv_empty[st]);
+        umma_commit(&bars->pv_done[pb]);
+        return true;
+      };
+      bool ok = mbar_wait(&bars->q_full, 0, abort);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t qa = smem_u32(sQ);
+        for (int j = 0; j < n_kv && ok; ++j) {
+          const int st = j % C::ST, sb = j & 1;
+          if (!mbar_wait(&bars->k_full[st], (j / C::ST) & 1, abort)) { ok = false; break; }
+          if (!mbar_wait(&bars->s_empty[sb], ((j >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t ka = smem_u32(sK + st * C::K_BYTES);
+#pragma unroll
+          for (int k = 0; k < DQK / 32; ++k) {
+            const int sub = (k * 32) / C::KSUB, off = (k * 32) % C::KSUB;
+            umma_i8(tmem + (sb ? C::S_COL1 : C::S_COL0),
+                    smem_desc_kmajor(qa + sub * 128 * C::KSUB + off, C::KSUB),
+                    smem_desc_kmajor(ka + sub * 128 * C::KSUB + off, C::KSUB), idesc_qk, (uint32_t)(k > 0));
+          }
+          umma_commit(&bars->s_full[sb]);
+          if (j > 0) ok = issue_pv(j - 1);
+        }
+        if (ok) issue_pv(n_kv - 1);
+      }
+      // every UMMA this thread issued has finished before TMEM is released
+      umma_commit(&bars->mma_done);
+      drain_wait(&bars->mma_done, 0);
+    }
+  } else {
+    // ------------------------------------------------------------------ softmax warps 0-3
+    const int row = warp * 32 + lane;            // query row inside the tile, TMEM lane
+    const int grow = qt * 128 + row;             // query row in the sequence
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const float qsv = p.qs[((size_t)b * p.Hq + hq) * p.nblk + qt];
+    const float* ksp = p.ks + ((size_t)b * p.Hkv + hkv) * p.nblk;
+    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+    bool ok = true;
+    for (int i = 0; i < n_kv; ++i) {
+      const int sb = i & 1, pb = i & 1;
+      if (!warp_wait(&bars->s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t s[128];
+      const uint32_t scol = tmem + lane_base + (sb ? C::S_COL1 : C::S_COL0);
+      tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
+      tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
+      tmem_ld32(scol + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
+      tmem_ld32(scol + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
+
+      // dequantization factor in the log2 domain
+      const float f = __fmul_rn(__fmul_rn(qsv, ksp[i]), p.scale_log2);
+      const int key0 = i * 128;
+      int lim = min(p.N - key0, 128);
+      if (CAUSAL && i == qt) lim = min(lim, row + 1);
+      int mx = INT_MIN;
+#pragma unroll
+      for (int c = 0; c < 128; ++c)
+        if (c < lim) mx = max(mx, (int)s[c]);
+      const float mt = (mx == INT_MIN) ? -INFINITY : __fmul_rn((float)mx, f);
+      const float m_new = fmaxf(m, mt);
+      const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
+      const float neg = (m_new == -INFINITY) ? 0.f : -m_new;
+      float rs = 0.f;
+      uint32_t pk[32];
+#pragma unroll
+      for (int c4 = 0; c4 < 32; ++c4) {
+        float pv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int c = c4 * 4 + e;
+          pv[e] = (c < lim) ? ex2_approx(fmaf((float)(int)s[c], f, neg)) : 0.f;
+          rs += pv[e];
+        }
+        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(pv[0] * 448.f, pv[1] * 448.f), __NV_SATFINITE,
+                                                     __NV_E4M3);
+        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(pv[2] * 448.f, pv[3] * 448.f), __NV_SATFINITE,
+                                                     __NV_E4M3);
+        pk[c4] = (lo & 0xFFFF) | (hi << 16);
+      }
+      l = l * alpha + rs;
+      m = m_new;
+
+      // P tile buffer pb was last read by the P.V MMA of tile i-2
+      if (i >= 2 && !warp_wait(&bars->pv_done[pb], ((i >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+      unsigned char* prow = sP + pb * C::P_BYTES + row * 128;
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
+      fence_proxy_async_smem();
+
+      if (i >= 1) {
+        // the P.V MMA of tile i-1 must be complete before O is touched
+        if (!warp_wait(&bars->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t ocol = tmem + lane_base + C::O_COL;
+        if (MODE == 0) {
+          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll 1
+            for (int cc = 0; cc < DV / 32; ++cc) {
+              uint32_t o[32];
+              tmem_ld32(ocol + cc * 32, o);
+              tmem_wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+              tmem_st32(ocol + cc * 32, o);
+            }
+            tmem_wait_st();
+          }
+        } else {
+          // O = O * alpha_{i-1} + T_{i-1}   (T is the fp16 partial of tile i-1)
+          const uint32_t tcol = tmem + lane_base + C::T_COL;
+#pragma unroll 1
+          for (int cc = 0; cc < DV / 64; ++cc) {
+            uint32_t t[32], o0[32], o1[32];
+            tmem_ld32_pack16(tcol + cc * 64, t);
+            if (i > 1) {
+              tmem_ld32(ocol + cc * 64, o0);
+              tmem_ld32(ocol + cc * 64 + 32, o1);
+            }
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 a = __half22float2(*reinterpret_cast<__half2*>(&t[e]));
+              const float2 bb = __half22float2(*reinterpret_cast<__half2*>(&t[16 + e]));
+              const float o_a = i > 1 ? __uint_as_float(o0[2 * e]) * alpha_prev : 0.f;
+              const float o_b = i > 1 ? __uint_as_float(o0[2 * e + 1]) * alpha_prev : 0.f;
+              const float o_c = i > 1 ? __uint_as_float(o1[2 * e]) * alpha_prev : 0.f;
+              const float o_d = i > 1 ? __uint_as_float(o1[2 * e + 1]) * alpha_prev : 0.f;
+              o0[2 * e] = __float_as_uint(o_a + a.x);
+              o0[2 * e + 1] = __float_as_uint(o_b + a.y);
+              o1[2 * e] = __float_as_uint(o_c + bb.x);
+              o1[2 * e + 1] = __float_as_uint(o_d + bb.y);
+            }
+            tmem_st32(ocol + cc * 64, o0);
+            tmem_st32(ocol + cc * 64 + 32, o1);
+          }
+          tmem_wait_st();
+        }
+      }
+      if (MODE == 1) alpha_prev = alpha;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->p_full[pb]);
+    }
+
+    // ---------------------------------------------------------------- epilogue
+    if (ok) {
+      const int last = n_kv - 1;
+      ok = warp_wait(&bars->pv_done[last & 1], (last >> 1) & 1, abort);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = __fdiv_rn(1.f, 448.f * l);
+        const float* vsp = p.vs + ((size_t)b * p.Hkv + hkv) * p.dp + vh * DV;
+        OutT* out = static_cast<OutT*>(p.out);
+        const size_t orow = (p.layout == SAGE_HND) ? (((size_t)b * p.Hq + hq) * p.N + grow) * p.d
+                                                   : (((size_t)b * p.N + grow) * p.Hq + hq) * p.d;
+        const uint32_t ocol = tmem + lane_base + C::O_COL;
+        const uint32_t tcol = tmem + lane_base + C::T_COL;
+#pragma unroll
+        for (int cc = 0; cc < DV / 32; ++cc) {
+          uint32_t o[32];
+          float of[32];
+          tmem_ld32(ocol + cc * 32, o);
+          if (MODE == 1) {
+            uint32_t t[32];
+            tmem_ld32_pack16(tcol + (cc / 2) * 64, t);
+            tmem_wait_ld();
+            // columns cc*32 .. cc*32+31 are packed pairs 16*(cc&1) .. 16*(cc&1)+15 of this load
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 a = __half22float2(*reinterpret_cast<__half2*>(&t[16 * (cc & 1) + e]));
+              of[2 * e] = (last > 0 ? __uint_as_float(o[2 * e]) * alpha_prev : 0.f) + a.x;
+              of[2 * e + 1] = (last > 0 ? __uint_as_float(o[2 * e + 1]) * alpha_prev : 0.f) + a.y;
+            }
+          } else {
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(o[e]);
+          }
+          if (grow < p.N) {
+            const int c0 = vh * DV + cc * 32;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) of[e] = of[e] * (vsp[cc * 32 + e] * inv_l);
+            if (c0 + 32 <= p.d && p.vec_out) {
+              uint32_t w[16];
+#pragma unroll
+              for (int e = 0; e < 16; ++e) w[e] = pack2<OutT>(of[2 * e], of[2 * e + 1]);
+              uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
+#pragma unroll
+              for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e)
+                if (c0 + e < p.d) store_elem(out + orow + c0 + e, of[e]);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Diagnostic: int32 S = Q8 . K8^T for a list of (b, hq, q_tile, k_tile) tiles, through the
+// same TMA loads, shared-memory descriptors and kind::i8 UMMA as the fused kernel.
+// ------------------------------------------------------------------------------------------------
+template <int DQK>
+__global__ void __launch_bounds__(128, 1)
+    sage_qk_dump_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                        const QkDumpParams p) {
+  using C = FwdCfg<DQK, 64>;
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* sQ = smem_raw + pad;
+  unsigned char* sK = sQ + C::Q_BYTES;
+  FwdBars* bars = reinterpret_cast<FwdBars*>(sK + C::K_BYTES);
+  volatile int* abort = &bars->abort;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x;
+  const int b = p.tiles[4 * t], hq = p.tiles[4 * t + 1], qt = p.tiles[4 * t + 2], kt = p.tiles[4 * t + 3];
+  const bool valid = b >= 0 && b < p.B && hq >= 0 && hq < p.Hq && qt >= 0 && qt < p.nblk && kt >= 0 && kt < p.nblk;
+  if (!valid) {
+    if (threadIdx.x == 0) atomicOr(&g_device_error, SAGE_DEVERR_BAD_ARG);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    mbar_init(&bars->q_full, 1);
+    mbar_init(&bars->mma_done, 1);
+    bars->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&bars->tmem_base, 128);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+  if (threadIdx.x == 32) {
+    const int q_row = (b * p.Hq + hq) * p.Np + qt * 128;
+    const int k_row = (b * p.Hkv + hq / p.G) * p.Np + kt * 128;
+    mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES + C::K_BYTES);
+    for (int s = 0; s < C::NSUB; ++s) {
+      tma_load_2d(sQ + s * 128 * C::KSUB, &tmQ, &bars->q_full, s * C::KSUB, q_row);
+      tma_load_2d(sK + s * 128 * C::KSUB, &tmK, &bars->q_full, s * C::KSUB, k_row);
+    }
+    if (mbar_wait(&bars->q_full, 0, abort)) {
+      tc_fence_after();
+      constexpr uint32_t idesc = make_idesc(2, 1, 128, 128);
+#pragma unroll
+      for (int k = 0; k < DQK / 32; ++k) {
+        const int sub = (k * 32) / C::KSUB, off = (k * 32) % C::KSUB;
+        umma_i8(tmem, smem_desc_kmajor(smem_u32(sQ) + sub * 128 * C::KSUB + off, C::KSUB),
+                smem_desc_kmajor(smem_u32(sK) + sub * 128 * C::KSUB + off, C::KSUB), idesc, (uint32_t)(k > 0));
+      }
+    } else {
+      drain_wait(&bars->q_full, 0);
+    }
+    umma_commit(&bars->mma_done);
+  }
+  if (warp_wait(&bars->mma_done, 0, abort) && !*abort) {
+    tc_fence_after();
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    int32_t* dst = p.out + ((size_t)t * 128 + warp * 32 + lane) * 128;
+#pragma unroll 1
+    for (int cc = 0; cc < 4; ++cc) {
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + cc * 32, r);
+      tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        reinterpret_cast<uint4*>(dst + cc * 32)[e] = make_uint4(r[4 * e], r[4 * e + 1], r[4 * e + 2], r[4 * e + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 128);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
+// launchers
+// ------------------------------------------------------------------------------------------------
+template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
+static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const FwdParams& p, cudaStream_t st) {
+  using C = FwdCfg<DQK, DV>;
+  auto kern = sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.nblk, p.Hq * p.n_vhalves, p.B);
+  kern<<<grid, 192, C::SMEM, st>>>(tq, tk, tv, p);
+  return cudaGetLastError();
+}
+
+template <int DQK, int DV, typename OutT>
+static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const FwdParams& p, int causal, int mode, cudaStream_t st) {
+  if (mode == 0)
+    return causal ? launch_fwd_t<DQK, DV, 0, true, OutT>(tq, tk, tv, p, st)
+                  : launch_fwd_t<DQK, DV, 0, false, OutT>(tq, tk, tv, p, st);
+  return causal ? launch_fwd_t<DQK, DV, 1, true, OutT>(tq, tk, tv, p, st)
+                : launch_fwd_t<DQK, DV, 1, false, OutT>(tq, tk, tv, p, st);
+}
+
+template <typename OutT>
+static cudaError_t launch_fwd_o(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const FwdParams& p, int causal, int mode, cudaStream_t st) {
+  switch (p.dp) {
+    case 64: return launch_fwd_d<64, 64, OutT>(tq, tk, tv, p, causal, mode, st);
+    case 128: return launch_fwd_d<128, 128, OutT>(tq, tk, tv, p, causal, mode, st);
+    case 256: return launch_fwd_d<256, 128, OutT>(tq, tk, tv, p, causal, mode, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const FwdParams& p,
+                       int dtype, int causal, int pv_mode, cudaStream_t st) {
+  return dtype == SAGE_BF16 ? launch_fwd_o<__nv_bfloat16>(tq, tk, tv, p, causal, pv_mode, st)
+                            : launch_fwd_o<__half>(tq, tk, tv, p, causal, pv_mode, st);
+}
+
+cudaError_t read_clear_device_error(int* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_device_error, &zero, sizeof(int));
+}
+
+template <int DQK>
+static cudaError_t launch_qk_dump_t(const CUtensorMap& tq, const CUtensorMap& tk, const QkDumpParams& p,
+                                    cudaStream_t st) {
+  using C = FwdCfg<DQK, 64>;
+  const int smem = 1024 + C::Q_BYTES + C::K_BYTES + C::BAR_BYTES;
+  cudaError_t e = cudaFuncSetAttribute(sage_qk_dump_kernel<DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  sage_qk_dump_kernel<DQK><<<p.n_tiles, 128, smem, st>>>(tq, tk, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_qk_dump(const CUtensorMap& tq, const CUtensorMap& tk, const QkDumpParams& p, int dp,
+                           cudaStream_t st) {
+  switch (dp) {
+    case 64: return launch_qk_dump_t<64>(tq, tk, p, st);
+    case 128: return launch_qk_dump_t<128>(tq, tk, p, st);
+    case 256: return launch_qk_dump_t<256>(tq, tk, p, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace sage

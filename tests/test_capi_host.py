@@ -1,0 +1,83 @@
+"""The C-ABI library on the host: it loads, exports what include/sage.h declares,
+and rejects bad arguments before touching any GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+FAKE = 0x100000  # never dereferenced: every call below fails its argument checks first
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "sage.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\**\s+\**(sage_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for n in ("sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
+              "sage_status_string", "sage_workspace_bytes", "sage_device_supported"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    raw = ctypes.CDLL(lib.LIB_PATH)
+    for n in _declared():
+        assert hasattr(raw, n), n
+
+
+def test_status_strings(lib):
+    for s in range(7):
+        assert lib.sage_status_string(s)
+    assert "fp16" in lib.sage_status_string(lib.SAGE_ERR_UNSUPPORTED)
+
+
+def _attn(lib, **kw):
+    a = dict(q=FAKE, k=FAKE + 0x100000000, v=FAKE + 0x200000000, out=FAKE + 0x300000000, B=1, Hq=2, Hkv=2, N=256,
+             d=64, dtype=lib.SAGE_FP16, layout=lib.SAGE_HND, causal=0, scale=0.0, pv=0)
+    a.update(kw)
+    return lib.capi.sage_attn(a["q"], a["k"], a["v"], a["out"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                              a["dtype"], a["layout"], a["causal"], a["scale"], a["pv"], None)
+
+
+def test_sage_attn_argument_checks(lib):
+    E, U = lib.SAGE_ERR_INVALID_ARG, lib.SAGE_ERR_UNSUPPORTED
+    assert _attn(lib, dtype=lib.SAGE_FP32) == U              # fp32 inputs are rejected like the reference
+    assert _attn(lib, dtype=7) == E
+    assert _attn(lib, q=None) == E and _attn(lib, out=None) == E
+    assert _attn(lib, Hq=3, Hkv=2) == E                      # GQA needs Hq % Hkv == 0
+    assert _attn(lib, d=257) == E and _attn(lib, d=0) == E
+    assert _attn(lib, N=0) == E and _attn(lib, B=0) == E
+    assert _attn(lib, layout=2) == E and _attn(lib, pv=2) == E
+    assert _attn(lib, out=FAKE + 10) == E                     # out overlaps q
+    assert _attn(lib, B=70000) == E                           # beyond the launch grid
+
+
+def test_other_entry_points_argument_checks(lib):
+    c, E = lib.capi, lib.SAGE_ERR_INVALID_ARG
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, lib.SAGE_FP32, 0, 0, *([FAKE] * 7), None) == \
+        lib.SAGE_ERR_UNSUPPORTED
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, None, *([FAKE] * 6), None) == E
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, FAKE + 1, *([FAKE] * 6), None) == E
+    assert c.sage_attn_quantized(*([FAKE] * 7), 1, 4, 3, 256, 64, 0, 0, 0, 0.0, 0, None) == E
+    assert c.sage_attn_quantized(*([FAKE] * 6), None, 1, 4, 2, 256, 64, 0, 0, 0, 0.0, 0, None) == E
+    assert c.sage_qk_int32(FAKE, FAKE, 1, 2, 2, 256, 64, None, 1, FAKE, None) == E
+    assert c.sage_qk_int32(FAKE, FAKE, 1, 2, 2, 256, 300, FAKE, 1, FAKE, None) == E
+    assert c.sage_qk_int32(FAKE, FAKE, 1, 2, 2, 256, 64, FAKE, 0, FAKE, None) == lib.SAGE_OK  # nothing to do
+
+
+def test_workspace_bytes(lib):
+    assert lib.sage_workspace_bytes(1, 2, 2, 0, 64) == 0
+    # q8 + k8 + v8 codes dominate: (Hq + 2 Hkv) * Np * dp bytes, plus fp32 scales and partial sums
+    ws = lib.sage_workspace_bytes(2, 8, 2, 1000, 96)
+    codes = 2 * (8 + 2 * 2) * 1024 * 128
+    assert codes < ws < codes + 2 * 2 * 8 * 128 * 4 * 2 + 64 * 1024
+
+
+def test_padded_dim(lib):
+    assert [lib.padded_dim(d) for d in (1, 64, 65, 128, 129, 256)] == [64, 64, 128, 128, 256, 256]
+    with pytest.raises(ValueError):
+        lib.padded_dim(300)

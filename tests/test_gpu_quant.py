@@ -1,0 +1,67 @@
+"""GPU quantize/smooth pass vs the oracle's emulation: bit-exact codes and scales."""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from oracle import quant
+from tests._support import cuda, slice_heads
+
+pytestmark = pytest.mark.gpu
+
+SMALL = [
+    W.TINY,
+    W.TINY.with_(name="ragged_d40_gqa_bf16", N=300, d=40, Hq=4, Hkv=2, dtype="bf16"),
+    W.TINY.with_(name="single_token_d96", N=1, d=96),
+    W.TINY.with_(name="nhd_koffset_fp16acc", N=700, d=128, layout="NHD", dist="normal_koffset", pv_mode=1),
+    W.TINY.with_(name="d256_uniform", B=2, N=129, d=256, dist="uniform2"),
+    W.TINY.with_(name="outlier_gqa4", N=640, d=64, Hq=8, Hkv=2, dist="normal_koutlier", dtype="bf16"),
+    W.TINY.with_(name="d33_causal", N=257, d=33, Hq=3, Hkv=1, causal=True),
+]
+
+
+def _gpu_codes(lib, w, q, k, v):
+    z = lib.sage_quantize(cuda(q), cuda(k), cuda(v), w.layout, "fp32" if w.pv_mode == 0 else "fp16+fp32")
+    lib.sage_check_status()
+    out = {k2: z[k2].cpu().numpy() for k2 in ("q8", "qs", "k8", "ks", "km", "vs")}
+    out["v8"] = z["v8t"].cpu().numpy().transpose(0, 1, 3, 2)
+    return out
+
+
+def _assert_same(got, ref, q_sel=slice(None), kv_sel=slice(None)):
+    for key in ("q8", "qs"):
+        assert np.array_equal(got[key][q_sel], ref[key]), key
+    for key in ("k8", "ks", "km", "v8", "vs"):
+        g, r = got[key][kv_sel], ref[key]
+        if g.dtype == np.float32:
+            ok = np.array_equal(g.view(np.uint32), r.view(np.uint32))
+        else:
+            ok = np.array_equal(g, r)
+        if not ok:
+            bad = np.argwhere(g != r)
+            raise AssertionError(f"{key}: {len(bad)} mismatches, first at {bad[:3].tolist()}")
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_quantize_bit_exact_small(lib, w):
+    q, k, v = W.make_inputs(w)
+    got = _gpu_codes(lib, w, q, k, v)
+    ref = quant.quantize(q, k, v, w.layout, w.pv_mode)
+    _assert_same(got, ref)
+
+
+FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"]]
+
+
+@pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
+def test_quantize_bit_exact_full_size_sampled_heads(lib, w):
+    """Full-size launch on the GPU; the oracle recomputes two sampled (batch, kv-head) groups."""
+    q, k, v = W.make_inputs(w)
+    got = _gpu_codes(lib, w, q, k, v)
+    G = w.Hq // w.Hkv
+    for b, hk in {(0, 0), (w.B - 1, w.Hkv - 1)}:
+        hq = list(range(hk * G, (hk + 1) * G))
+        ref = quant.quantize(slice_heads(q, w.layout, b, hq), slice_heads(k, w.layout, b, [hk]),
+                             slice_heads(v, w.layout, b, [hk]), w.layout, w.pv_mode)
+        _assert_same(got, ref, q_sel=(slice(b, b + 1), slice(hk * G, (hk + 1) * G)),
+                     kv_sel=(slice(b, b + 1), slice(hk, hk + 1)))
