@@ -36,15 +36,28 @@ def cos_sim(a, b) -> float:
     return float(a @ b / np.sqrt((a @ a) * (b @ b)))
 
 
-def check_vs_exact(out, ref, nkeys, vmax, what=""):
-    """out, ref: (..., rows, d) float64; nkeys: (rows,) number of visible keys of each row."""
+def check_vs_exact(out, ref, nkeys, vmax, what="", emul=None):
+    """out, ref: (..., rows, d) float64; nkeys: (rows,) number of visible keys of each row.
+
+    The 0.999 cosine bound is stated for unit-variance inputs.  For inputs
+    with K outlier channels (``emul`` given: the method's own output on the
+    same rows), a x8 channel inflates the shared per-block INT8 scale of K
+    and the method itself can fall below these bounds (both were measured on
+    unit-variance inputs); the GPU must then be at least as accurate as the
+    method: cos >= min(0.999, cos(emul, exact) - 2e-4) and, on rows with
+    >= 128 keys, max abs <= max(0.1, max |emul - exact| + 0.02).
+    """
     err = np.abs(out - ref)
     c = cos_sim(out, ref)
-    assert c >= COS_MIN, f"{what}: cosine {c:.6f} < {COS_MIN}"
+    cmin = COS_MIN if emul is None else min(COS_MIN, cos_sim(emul, ref) - 2e-4)
+    assert c >= cmin, f"{what}: cosine {c:.6f} < {cmin:.6f}"
     big = np.asarray(nkeys) >= 128
     if big.any():
         m = err[..., big, :].max()
-        assert m <= PAGES_MAX_ABS, f"{what}: max abs {m:.4f} on rows with >= 128 keys"
+        bound = PAGES_MAX_ABS
+        if emul is not None:
+            bound = max(bound, float(np.abs(emul - ref)[..., big, :].max()) + 0.02)
+        assert m <= bound, f"{what}: max abs {m:.4f} > {bound:.4f} on rows with >= 128 keys"
     m_all = err.max()
     assert m_all <= 0.125 * vmax, f"{what}: max abs {m_all:.4f} > 2^-3 max|V| = {0.125 * vmax:.4f}"
     return dict(cos=c, max_abs=float(m_all), max_abs_128=float(err[..., big, :].max()) if big.any() else 0.0)
