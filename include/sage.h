@@ -126,6 +126,32 @@ const char* sage_status_string(sage_status s);
 /* 1 if the current CUDA device can run this library (compute capability 10.0). */
 int sage_device_supported(void);
 
+/* Largest workspace sage_attn_noalloc can hold: 64 MiB (for example B=2, H=24,
+ * N=4096, d=64 needs about 38 MiB; sage_workspace_bytes() gives the exact need). */
+#define SAGE_NOALLOC_MAX_BYTES (64u << 20)
+
+/* sage_attn without any device allocation.  The paper has no counterpart: this
+ * entry point exists for callers that cannot call cudaMalloc/cudaMallocAsync at
+ * call time -- for example a host framework or server that reserves all device
+ * memory up front and treats any other allocation as an error, a runtime whose
+ * allocations are forbidden after initialisation, or a GPU/driver setup without
+ * stream-ordered memory pools.  Same arguments, checks and result as sage_attn.
+ *
+ * Its workspace is one static device array of SAGE_NOALLOC_MAX_BYTES inside this
+ * library: every GPU that loads the library holds that memory until the process
+ * exits.  Problems whose workspace (sage_workspace_bytes) exceeds the maximum are
+ * rejected with SAGE_ERR_INVALID_ARG before any GPU work.  The first call on each
+ * device looks up the array's device address (cudaGetSymbolAddress) with that
+ * device current; make that first call before any stream capture.  All calls
+ * share the one array and it keeps the previous call's contents (every byte a call
+ * reads is written by the same call first), so calls that can overlap on the GPU --
+ * on different streams, or from different host threads -- race with each other:
+ * order them on one stream or synchronise between them.  It allocates nothing: no
+ * cudaMalloc, cudaFree or allocating library routine is called. */
+sage_status sage_attn_noalloc(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N,
+                              int d, sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale,
+                              sage_pv_mode pv_mode, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -1,7 +1,7 @@
 """INT8-QK / FP8-PV quantized attention for NVIDIA B200 (sm_100a).
 
 Thin Python binding over the C ABI in ``include/sage.h`` (``libsage_b200.so``,
-built in-tree by ``python -m quantized_attention_int8_b200.build_lib``).  The
+built in-tree by ``python quantized_attention_int8_b200/build_lib.py``).  The
 functions keep the C entry points' names and only marshal arguments: torch
 supplies device memory and the current CUDA stream, and every step of the
 computation runs in the library's CUDA kernels.  There is no CPU fallback: if
@@ -24,6 +24,7 @@ import torch
 __all__ = [
     "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
     "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
+    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
@@ -42,7 +43,7 @@ _PV = {"fp32": SAGE_PV_FP32, "fp16+fp32": SAGE_PV_FP16_FP32}
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python -m quantized_attention_int8_b200.build_lib` "
+            f"{LIB_PATH} is not built; run `python quantized_attention_int8_b200/build_lib.py` "
             "(this package has no CPU fallback)")
     lib = ctypes.CDLL(LIB_PATH)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
@@ -55,6 +56,7 @@ def _load() -> ctypes.CDLL:
         "sage_check_status": ([P], I),
         "sage_status_string": ([I], ctypes.c_char_p),
         "sage_device_supported": ([], I),
+        "sage_attn_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -82,10 +84,6 @@ def _check(status: int, where: str) -> None:
 
 def _stream() -> int:
     return torch.cuda.current_stream().cuda_stream
-
-
-def _ptr(t: torch.Tensor | None) -> int | None:
-    return None if t is None else t.data_ptr()
 
 
 def padded_dim(d: int) -> int:
@@ -136,6 +134,29 @@ def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_a
                         _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)),
                         float(sm_scale) if sm_scale is not None else 0.0, _PV[pv_accum_dtype], _stream())
     _check(st, "sage_attn")
+    return out
+
+
+SAGE_NOALLOC_MAX_BYTES = 64 << 20
+
+
+def sage_attn_noalloc(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None):
+    """sage_attn with no device allocation inside the library (for callers that cannot
+    allocate at call time); the caller supplies ``out`` or torch allocates it here.  The
+    library's static workspace holds problems up to SAGE_NOALLOC_MAX_BYTES of workspace;
+    calls that may overlap on the GPU must be ordered by the caller."""
+    B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    need = sage_workspace_bytes(B, Hq, Hkv, N, d)
+    if need > SAGE_NOALLOC_MAX_BYTES:
+        raise ValueError(f"workspace of {need} bytes exceeds the static {SAGE_NOALLOC_MAX_BYTES} bytes; use sage_attn")
+    if out is None:
+        out = torch.empty_like(q)
+    st = capi.sage_attn_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
+                                _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)),
+                                float(sm_scale) if sm_scale is not None else 0.0, _PV[pv_accum_dtype], _stream())
+    _check(st, "sage_attn_noalloc")
     return out
 
 

@@ -1,6 +1,9 @@
 """Builds the CUDA library (libsage_b200.so) in-tree with nvcc for sm_100a.
 
-Usage: python -m quantized_attention_int8_b200.build_lib [--force] [--ptxas-info]
+Usage: python quantized_attention_int8_b200/build_lib.py [--force] [--ptxas-info]
+
+Run it as a script (not as a module of the package): importing the package
+loads the library, which may not exist yet or may be stale.
 """
 from __future__ import annotations
 

@@ -311,3 +311,60 @@ const char* sage_status_string(sage_status s) {
 int sage_device_supported(void) { return check_device() == SAGE_OK ? 1 : 0; }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------------------------------------
+// Allocation-free entry point: the workspace is a static device array in this library.
+// ------------------------------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_noalloc_scratch[SAGE_NOALLOC_MAX_BYTES];
+
+namespace {
+
+// The array's device address, looked up once per device with that device current.
+cudaError_t noalloc_scratch(int dev, unsigned char** out) {
+  constexpr int kMaxDevices = 128;
+  static std::mutex mu;
+  static unsigned char* addr[kMaxDevices] = {};
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = static_cast<unsigned char*>(p);
+  }
+  *out = addr[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+extern "C" sage_status sage_attn_noalloc(const void* q, const void* k, const void* v, void* out, int B, int Hq,
+                                         int Hkv, int N, int d, sage_dtype dtype, sage_layout layout, int is_causal,
+                                         float sm_scale, sage_pv_mode pv_mode, void* stream) {
+  Dims m;
+  sage_status s = check_common(q, k, v, B, Hq, Hkv, N, d, dtype, layout, pv_mode, &m);
+  if (s != SAGE_OK) return s;
+  if (!out) return SAGE_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
+  if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes))
+    return SAGE_ERR_INVALID_ARG;
+  const WsLayout w = ws_layout(m);
+  if (w.total > (size_t)SAGE_NOALLOC_MAX_BYTES) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_device()) != SAGE_OK) return s;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  unsigned char* ws = nullptr;
+  if (noalloc_scratch(dev, &ws) != cudaSuccess) return SAGE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
+  QuantBufs qb{reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
+               reinterpret_cast<int8_t*>(ws + w.k8), reinterpret_cast<float*>(ws + w.ks),
+               reinterpret_cast<float*>(ws + w.km), ws + w.v8t, reinterpret_cast<float*>(ws + w.vs)};
+  qp.q8 = qb.q8, qp.qs = qb.qs, qp.k8 = qb.k8, qp.ks = qb.ks, qp.km = qb.km, qp.v8t = qb.v8t, qp.vs = qb.vs;
+  qp.ksum_part = reinterpret_cast<float*>(ws + w.ksum);
+  qp.vmax_part = reinterpret_cast<float*>(ws + w.vmax);
+  qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
+  s = from_cuda(launch_quantize(qp, st));
+  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode, st);
+  return s;
+}

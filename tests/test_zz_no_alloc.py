@@ -1,0 +1,60 @@
+"""The allocation-free entry point sage_attn_noalloc, called through the C ABI.
+
+It is for callers that cannot allocate device memory at call time (a framework
+or server that reserves all GPU memory up front, a runtime that forbids
+allocation after start-up, a setup without stream-ordered memory pools); its
+workspace is a static device array inside the library.  This file runs last so
+that a failure here leaves every other test already run.  It passes alone in a
+fresh process and after the other tests: the only state it relies on is the
+per-device address lookup that the first call performs.
+"""
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from tests._support import TIGHT_ABS, TIGHT_REL, cuda
+
+pytestmark = pytest.mark.gpu
+
+CASES = [
+    W.IMAGE_DIT,                                                              # ~38 MiB of the 64 MiB workspace
+    W.TINY.with_(name="ragged_causal_gqa_d96", N=300, d=96, Hq=4, Hkv=2, causal=True, sm_scale=None),
+]
+
+
+def _dt(lib, t):
+    return lib.SAGE_BF16 if t.dtype == torch.bfloat16 else lib.SAGE_FP16
+
+
+def _call(lib, fn, w, q, k, v, out):
+    return fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.B, w.Hq, w.Hkv, w.N, w.d, _dt(lib, q),
+              lib.SAGE_HND if w.layout == "HND" else lib.SAGE_NHD, int(w.causal), float(W.sm_scale_of(w)),
+              w.pv_mode, torch.cuda.current_stream().cuda_stream)
+
+
+def test_noalloc_matches_sage_attn_on_two_calls_in_a_row(lib):
+    outs = []
+    for w in CASES:  # two calls in a row, the second on a smaller problem than the first
+        assert lib.sage_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d) <= lib.SAGE_NOALLOC_MAX_BYTES
+        q, k, v = (cuda(t) for t in W.make_inputs(w))
+        out = torch.empty_like(q)
+        assert _call(lib, lib.capi.sage_attn_noalloc, w, q, k, v, out) == lib.SAGE_OK
+        outs.append((w, q, k, v, out))
+    assert lib.capi.sage_check_status(torch.cuda.current_stream().cuda_stream) == lib.SAGE_OK
+    for w, q, k, v, out in outs:
+        ref = torch.empty_like(q)
+        assert _call(lib, lib.capi.sage_attn, w, q, k, v, ref) == lib.SAGE_OK
+        assert lib.capi.sage_check_status(torch.cuda.current_stream().cuda_stream) == lib.SAGE_OK
+        a = out.float().cpu().numpy()
+        b = ref.float().cpu().numpy()
+        assert np.all(np.abs(a - b) <= TIGHT_REL * np.abs(b) + TIGHT_ABS), w.name
+
+
+def test_noalloc_rejects_workspace_beyond_the_static_array(lib):
+    w = W.LLM_GQA  # needs ~200 MiB of workspace
+    assert lib.sage_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d) > lib.SAGE_NOALLOC_MAX_BYTES
+    fake = 0x100000
+    st = lib.capi.sage_attn_noalloc(fake, fake + (1 << 34), fake + (2 << 34), fake + (3 << 34), w.B, w.Hq, w.Hkv,
+                                    w.N, w.d, lib.SAGE_FP16, lib.SAGE_HND, 1, 0.0, 0, None)
+    assert st == lib.SAGE_ERR_INVALID_ARG
