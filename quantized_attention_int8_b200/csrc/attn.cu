@@ -41,19 +41,24 @@ struct FwdCfg {
   static constexpr int K_BYTES = 128 * DQK;
   static constexpr int V_BYTES = DV * 128;
   static constexpr int P_BYTES = 128 * 128;
-  static constexpr int ST = DQK == 64 ? 4 : 3;
+  static constexpr int ST = DQK == 64 ? 5 : 2;                 // K/V ring depth
+  static constexpr int CTAS_PER_SM = DQK <= 128 ? 2 : 1;       // two CTAs share an SM when they fit
   static constexpr int BAR_BYTES = 256;
-  static constexpr int SMEM = 1024 + Q_BYTES + ST * (K_BYTES + V_BYTES) + 2 * P_BYTES + BAR_BYTES;
-  static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t S_COL0 = 0, S_COL1 = 128, O_COL = 256, T_COL = 256 + DV;
-  static_assert(T_COL + DV <= TMEM_COLS, "TMEM plan");
+  static constexpr int SMEM = 1024 + Q_BYTES + ST * (K_BYTES + V_BYTES) + P_BYTES + BAR_BYTES;
+  // TMEM: S (int32 scores, 128 columns) and O (fp32, DV columns).  In fp16+fp32 mode the
+  // per-tile fp16 accumulator T reuses S's columns once the scores are in registers.
+  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t S_COL = 0, O_COL = 128, T_COL = 0;
+  static_assert(O_COL + DV <= TMEM_COLS, "TMEM plan");
+  static_assert(ST <= 8, "barrier array size");
   static_assert(SMEM <= 227 * 1024, "shared memory plan");
+  static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "co-resident CTAs must fit in shared memory");
 };
 
 struct FwdBars {
   uint64_t q_full;
-  uint64_t k_full[4], v_full[4], kv_empty[4];
-  uint64_t s_full[2], s_empty[2], p_full[2], pv_done[2];
+  uint64_t k_full[8], v_full[8], kv_empty[8];
+  uint64_t s_full, s_free, p_full, pv_done;
   uint64_t mma_done;
   uint32_t tmem_base;
   int abort;
@@ -91,8 +96,15 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Two E4M3 codes (RN, saturating) of a and b, a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3) & 0xFFFFu;
+}
+
+constexpr float kLog2_448 = 8.807354922057604f;  // p * 448 = 2^(log2 p + log2 448)
+
 template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     sage_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<DQK, DV>;
@@ -103,7 +115,7 @@ __global__ void __launch_bounds__(192, 1)
   unsigned char* sK = sQ + C::Q_BYTES;
   unsigned char* sV = sK + C::ST * C::K_BYTES;
   unsigned char* sP = sV + C::ST * C::V_BYTES;
-  FwdBars* bars = reinterpret_cast<FwdBars*>(sP + 2 * C::P_BYTES);
+  FwdBars* bars = reinterpret_cast<FwdBars*>(sP + C::P_BYTES);
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -121,12 +133,10 @@ __global__ void __launch_bounds__(192, 1)
       mbar_init(&bars->v_full[s], 1);
       mbar_init(&bars->kv_empty[s], 1);
     }
-    for (int s = 0; s < 2; ++s) {
-      mbar_init(&bars->s_full[s], 1);
-      mbar_init(&bars->s_empty[s], 4);
-      mbar_init(&bars->p_full[s], 4);
-      mbar_init(&bars->pv_done[s], 1);
-    }
+    mbar_init(&bars->s_full, 1);
+    mbar_init(&bars->s_free, 4);
+    mbar_init(&bars->p_full, 4);
+    mbar_init(&bars->pv_done, 1);
     mbar_init(&bars->mma_done, 1);
     bars->abort = 0;
     fence_mbar_init();
@@ -171,23 +181,27 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ UMMA issuer
+    // fp32 mode: QK(j) is issued as soon as S is free (the softmax has it in registers),
+    // ahead of PV(j-1).  fp16+fp32 mode: T(j) lives in S's columns, so QK(j+1) waits
+    // until the softmax has merged T(j) into O, and the order is QK(j), PV(j).
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*S8*/, 128, 128);
       constexpr uint32_t idesc_pv = make_idesc(MODE == 0 ? 1 /*F32*/ : 0 /*F16*/, 0 /*E4M3*/, 128, DV);
       const uint32_t pv_dst = tmem + (MODE == 0 ? C::O_COL : C::T_COL);
+      const uint32_t pa = smem_u32(sP);
       auto issue_pv = [&](int i) -> bool {
-        const int st = i % C::ST, pb = i & 1;
+        const int st = i % C::ST;
         if (!mbar_wait(&bars->v_full[st], (i / C::ST) & 1, abort)) return false;
-        if (!mbar_wait(&bars->p_full[pb], (i >> 1) & 1, abort)) return false;
+        if (!mbar_wait(&bars->p_full, i & 1, abort)) return false;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sP + pb * C::P_BYTES), va = smem_u32(sV + st * C::V_BYTES);
+        const uint32_t va = smem_u32(sV + st * C::V_BYTES);
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           const uint32_t acc = MODE == 0 ? (uint32_t)(i > 0 || k > 0) : (uint32_t)(k > 0);
           umma_f8(pv_dst, smem_desc_kmajor(pa + k * 32, 128), smem_desc_kmajor(va + k * 32, 128), idesc_pv, acc);
         }
         umma_commit(&bars->kv_empty[st]);
-        umma_commit(&bars->pv_done[pb]);
+        umma_commit(&bars->pv_done);
         return true;
       };
       bool ok = mbar_wait(&bars->q_full, 0, abort);
@@ -195,22 +209,25 @@ __global__ void __launch_bounds__(192, 1)
         tc_fence_after();
         const uint32_t qa = smem_u32(sQ);
         for (int j = 0; j < n_kv && ok; ++j) {
-          const int st = j % C::ST, sb = j & 1;
+          const int st = j % C::ST;
           if (!mbar_wait(&bars->k_full[st], (j / C::ST) & 1, abort)) { ok = false; break; }
-          if (!mbar_wait(&bars->s_empty[sb], ((j >> 1) & 1) ^ 1, abort)) { ok = false; break; }
+          if (j > 0 && !mbar_wait(&bars->s_free, (j - 1) & 1, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t ka = smem_u32(sK + st * C::K_BYTES);
 #pragma unroll
           for (int k = 0; k < DQK / 32; ++k) {
             const int sub = (k * 32) / C::KSUB, off = (k * 32) % C::KSUB;
-            umma_i8(tmem + (sb ? C::S_COL1 : C::S_COL0),
-                    smem_desc_kmajor(qa + sub * 128 * C::KSUB + off, C::KSUB),
+            umma_i8(tmem + C::S_COL, smem_desc_kmajor(qa + sub * 128 * C::KSUB + off, C::KSUB),
                     smem_desc_kmajor(ka + sub * 128 * C::KSUB + off, C::KSUB), idesc_qk, (uint32_t)(k > 0));
           }
-          umma_commit(&bars->s_full[sb]);
-          if (j > 0) ok = issue_pv(j - 1);
+          umma_commit(&bars->s_full);
+          if (MODE == 0) {
+            if (j > 0) ok = issue_pv(j - 1);
+          } else {
+            ok = issue_pv(j);
+          }
         }
-        if (ok) issue_pv(n_kv - 1);
+        if (ok && MODE == 0) issue_pv(n_kv - 1);
       }
       // every UMMA this thread issued has finished before TMEM is released
       umma_commit(&bars->mma_done);
@@ -221,172 +238,159 @@ __global__ void __launch_bounds__(192, 1)
     const int row = warp * 32 + lane;            // query row inside the tile, TMEM lane
     const int grow = qt * 128 + row;             // query row in the sequence
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t scol = tmem + lane_base + C::S_COL;
+    const uint32_t ocol = tmem + lane_base + C::O_COL;
     const float qsv = p.qs[((size_t)b * p.Hq + hq) * p.nblk + qt];
     const float* ksp = p.ks + ((size_t)b * p.Hkv + hkv) * p.nblk;
-    float m = -INFINITY, l = 0.f, alpha_prev = 1.f;
+    unsigned char* prow = sP + row * 128;
+    float m = -INFINITY, l = 0.f;  // l accumulates p * 448
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
-      const int sb = i & 1, pb = i & 1;
-      if (!warp_wait(&bars->s_full[sb], (i >> 1) & 1, abort)) { ok = false; break; }
+      if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
       uint32_t s[128];
-      const uint32_t scol = tmem + lane_base + (sb ? C::S_COL1 : C::S_COL0);
       tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
       tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
       tmem_ld32(scol + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
       tmem_ld32(scol + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
       tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->s_empty[sb]);
+      if (MODE == 0) {  // S is in registers: the next QK may overwrite it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+      }
 
       // dequantization factor in the log2 domain
       const float f = __fmul_rn(__fmul_rn(qsv, ksp[i]), p.scale_log2);
       const int key0 = i * 128;
-      int lim = min(p.N - key0, 128);
-      if (CAUSAL && i == qt) lim = min(lim, row + 1);
-      int mx = INT_MIN;
+      const bool edge = (key0 + 128 > p.N) || (CAUSAL && i == qt);
+      int lim = 128;
+      if (edge) {
+        lim = min(p.N - key0, 128);
+        if (CAUSAL && i == qt) lim = min(lim, row + 1);
 #pragma unroll
-      for (int c = 0; c < 128; ++c)
-        if (c < lim) mx = max(mx, (int)s[c]);
+        for (int c = 0; c < 128; ++c)
+          if (c >= lim) s[c] = (uint32_t)INT_MIN;
+      }
+      int mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = (int)s[e];
+#pragma unroll
+      for (int c = 8; c < 128; ++c) mx8[c & 7] = max(mx8[c & 7], (int)s[c]);
+      const int mx = max(max(max(mx8[0], mx8[1]), max(mx8[2], mx8[3])), max(max(mx8[4], mx8[5]), max(mx8[6], mx8[7])));
       const float mt = (mx == INT_MIN) ? -INFINITY : __fmul_rn((float)mx, f);
       const float m_new = fmaxf(m, mt);
       const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-      const float neg = (m_new == -INFINITY) ? 0.f : -m_new;
-      float rs = 0.f;
-      uint32_t pk[32];
-#pragma unroll
-      for (int c4 = 0; c4 < 32; ++c4) {
-        float pv[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int c = c4 * 4 + e;
-          pv[e] = (c < lim) ? ex2_approx(fmaf((float)(int)s[c], f, neg)) : 0.f;
-          rs += pv[e];
-        }
-        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(pv[0] * 448.f, pv[1] * 448.f), __NV_SATFINITE,
-                                                     __NV_E4M3);
-        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(pv[2] * 448.f, pv[3] * 448.f), __NV_SATFINITE,
-                                                     __NV_E4M3);
-        pk[c4] = (lo & 0xFFFF) | (hi << 16);
-      }
-      l = l * alpha + rs;
-      m = m_new;
-
-      // P tile buffer pb was last read by the P.V MMA of tile i-2
-      if (i >= 2 && !warp_wait(&bars->pv_done[pb], ((i >> 1) & 1) ^ 1, abort)) { ok = false; break; }
-      unsigned char* prow = sP + pb * C::P_BYTES + row * 128;
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
-            make_uint4(pk[ch * 4 + 0], pk[ch * 4 + 1], pk[ch * 4 + 2], pk[ch * 4 + 3]);
-      fence_proxy_async_smem();
-
-      if (i >= 1) {
-        // the P.V MMA of tile i-1 must be complete before O is touched
-        if (!warp_wait(&bars->pv_done[(i - 1) & 1], ((i - 1) >> 1) & 1, abort)) { ok = false; break; }
+      const float bias = (m_new == -INFINITY) ? 0.f : kLog2_448 - m_new;
+      if (MODE == 0 && i > 0) {
+        // P's buffer and O were last used by the P.V MMA of tile i-1
+        if (!warp_wait(&bars->pv_done, (i - 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
-        const uint32_t ocol = tmem + lane_base + C::O_COL;
-        if (MODE == 0) {
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-            for (int cc = 0; cc < DV / 32; ++cc) {
-              uint32_t o[32];
-              tmem_ld32(ocol + cc * 32, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(ocol + cc * 32, o);
-            }
-            tmem_wait_st();
-          }
-        } else {
-          // O = O * alpha_{i-1} + T_{i-1}   (T is the fp16 partial of tile i-1)
-          const uint32_t tcol = tmem + lane_base + C::T_COL;
-#pragma unroll 1
-          for (int cc = 0; cc < DV / 64; ++cc) {
-            uint32_t t[32], o0[32], o1[32];
-            tmem_ld32_pack16(tcol + cc * 64, t);
-            if (i > 1) {
-              tmem_ld32(ocol + cc * 64, o0);
-              tmem_ld32(ocol + cc * 64 + 32, o1);
-            }
+          for (int cc = 0; cc < DV / 16; ++cc) {
+            uint32_t o[16];
+            tmem_ld16(ocol + cc * 16, o);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float2 a = __half22float2(*reinterpret_cast<__half2*>(&t[e]));
-              const float2 bb = __half22float2(*reinterpret_cast<__half2*>(&t[16 + e]));
-              const float o_a = i > 1 ? __uint_as_float(o0[2 * e]) * alpha_prev : 0.f;
-              const float o_b = i > 1 ? __uint_as_float(o0[2 * e + 1]) * alpha_prev : 0.f;
-              const float o_c = i > 1 ? __uint_as_float(o1[2 * e]) * alpha_prev : 0.f;
-              const float o_d = i > 1 ? __uint_as_float(o1[2 * e + 1]) * alpha_prev : 0.f;
-              o0[2 * e] = __float_as_uint(o_a + a.x);
-              o0[2 * e + 1] = __float_as_uint(o_b + a.y);
-              o1[2 * e] = __float_as_uint(o_c + bb.x);
-              o1[2 * e + 1] = __float_as_uint(o_d + bb.y);
-            }
-            tmem_st32(ocol + cc * 64, o0);
-            tmem_st32(ocol + cc * 64 + 32, o1);
+            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st16(ocol + cc * 16, o);
           }
           tmem_wait_st();
         }
       }
-      if (MODE == 1) alpha_prev = alpha;
+      // p * 448 = 2^(s*f - m' + log2 448) -> E4M3, 16 keys (one 16-byte chunk) at a time
+      float rs[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+      for (int ch = 0; ch < 8; ++ch) {
+        uint32_t w[4];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          float pv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int c = ch * 16 + c4 * 4 + e;
+            pv[e] = ex2_approx(fmaf((float)(int)s[c], f, bias));
+            if (edge) pv[e] = (c < lim) ? pv[e] : 0.f;
+            rs[e] += pv[e];
+          }
+          w[c4] = e4m3x2(pv[0], pv[1]) | (e4m3x2(pv[2], pv[3]) << 16);
+        }
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      fence_proxy_async_smem();
+      l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
+      m = m_new;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars->p_full[pb]);
+      if (lane == 0) mbar_arrive(&bars->p_full);
+
+      if (MODE == 1) {
+        // O = O * alpha + T(i), T being this tile's fresh fp16 accumulator (in S's columns)
+        if (!warp_wait(&bars->pv_done, i & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t tcol = tmem + lane_base + C::T_COL;
+#pragma unroll 1
+        for (int cc = 0; cc < DV / 32; ++cc) {
+          uint32_t t[16], o0[16], o1[16];
+          tmem_ld16_pack16(tcol + cc * 32, t);
+          if (i > 0) {
+            tmem_ld16(ocol + cc * 32, o0);
+            tmem_ld16(ocol + cc * 32 + 16, o1);
+          }
+          tmem_wait_ld();
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float2 tv = __half22float2(*reinterpret_cast<__half2*>(&t[e]));
+            uint32_t* o = e < 8 ? o0 : o1;
+            const int k = (2 * e) & 15;
+            const float a0 = i > 0 ? __uint_as_float(o[k]) * alpha : 0.f;
+            const float a1 = i > 0 ? __uint_as_float(o[k + 1]) * alpha : 0.f;
+            o[k] = __float_as_uint(a0 + tv.x);
+            o[k + 1] = __float_as_uint(a1 + tv.y);
+          }
+          tmem_st16(ocol + cc * 32, o0);
+          tmem_st16(ocol + cc * 32 + 16, o1);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars->s_free);
+      }
     }
 
     // ---------------------------------------------------------------- epilogue
+    if (ok && MODE == 0) {
+      ok = warp_wait(&bars->pv_done, (n_kv - 1) & 1, abort);
+      if (ok) tc_fence_after();
+    }
     if (ok) {
-      const int last = n_kv - 1;
-      ok = warp_wait(&bars->pv_done[last & 1], (last >> 1) & 1, abort);
-      if (ok) {
-        tc_fence_after();
-        const float inv_l = __fdiv_rn(1.f, 448.f * l);
-        const float* vsp = p.vs + ((size_t)b * p.Hkv + hkv) * p.dp + vh * DV;
-        OutT* out = static_cast<OutT*>(p.out);
-        const size_t orow = (p.layout == SAGE_HND) ? (((size_t)b * p.Hq + hq) * p.N + grow) * p.d
-                                                   : (((size_t)b * p.N + grow) * p.Hq + hq) * p.d;
-        const uint32_t ocol = tmem + lane_base + C::O_COL;
-        const uint32_t tcol = tmem + lane_base + C::T_COL;
+      const float inv_l = __fdiv_rn(1.f, l);
+      const float* vsp = p.vs + ((size_t)b * p.Hkv + hkv) * p.dp + vh * DV;
+      OutT* out = static_cast<OutT*>(p.out);
+      const size_t orow = (p.layout == SAGE_HND) ? (((size_t)b * p.Hq + hq) * p.N + grow) * p.d
+                                                 : (((size_t)b * p.N + grow) * p.Hq + hq) * p.d;
+#pragma unroll 1
+      for (int cc = 0; cc < DV / 32; ++cc) {
+        uint32_t o[32];
+        float of[32];
+        tmem_ld32(ocol + cc * 32, o);
+        tmem_wait_ld();
+        if (grow < p.N) {
+          const int c0 = vh * DV + cc * 32;
 #pragma unroll
-        for (int cc = 0; cc < DV / 32; ++cc) {
-          uint32_t o[32];
-          float of[32];
-          tmem_ld32(ocol + cc * 32, o);
-          if (MODE == 1) {
-            uint32_t t[32];
-            tmem_ld32_pack16(tcol + (cc / 2) * 64, t);
-            tmem_wait_ld();
-            // columns cc*32 .. cc*32+31 are packed pairs 16*(cc&1) .. 16*(cc&1)+15 of this load
+          for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(o[e]) * (vsp[cc * 32 + e] * inv_l);
+          if (c0 + 32 <= p.d && p.vec_out) {
+            uint32_t w[16];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const float2 a = __half22float2(*reinterpret_cast<__half2*>(&t[16 * (cc & 1) + e]));
-              of[2 * e] = (last > 0 ? __uint_as_float(o[2 * e]) * alpha_prev : 0.f) + a.x;
-              of[2 * e + 1] = (last > 0 ? __uint_as_float(o[2 * e + 1]) * alpha_prev : 0.f) + a.y;
-            }
+            for (int e = 0; e < 16; ++e) w[e] = pack2<OutT>(of[2 * e], of[2 * e + 1]);
+            uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
           } else {
-            tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(o[e]);
-          }
-          if (grow < p.N) {
-            const int c0 = vh * DV + cc * 32;
-#pragma unroll
-            for (int e = 0; e < 32; ++e) of[e] = of[e] * (vsp[cc * 32 + e] * inv_l);
-            if (c0 + 32 <= p.d && p.vec_out) {
-              uint32_t w[16];
-#pragma unroll
-              for (int e = 0; e < 16; ++e) w[e] = pack2<OutT>(of[2 * e], of[2 * e + 1]);
-              uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
-#pragma unroll
-              for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
-            } else {
-#pragma unroll
-              for (int e = 0; e < 32; ++e)
-                if (c0 + e < p.d) store_elem(out + orow + c0 + e, of[e]);
-            }
+            for (int e = 0; e < 32; ++e)
+              if (c0 + e < p.d) store_elem(out + orow + c0 + e, of[e]);
           }
         }
       }
