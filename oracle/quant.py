@@ -15,11 +15,13 @@ choice a reader can check here, and the CUDA path implements the same one):
 
 * Smoothing subtracts the per-channel mean of K over all N tokens of a
   (batch, kv-head) (softmax is invariant to it: every score of query row i
-  shifts by q_i . mean(K)).  The mean is summed in float32 in a fixed order:
-  each 128-token block is summed token by token from its lowest token
-  (starting from +0.0, skipping tokens >= N), then the block partial sums are
-  added one by one in block order starting from +0.0, and the total is
-  divided by float(N) with one IEEE division.
+  shifts by q_i . mean(K)).  The pages give no summation order; the mean is
+  summed in float32 in this fixed order: each 128-token block is split into
+  8 groups of 16 consecutive tokens, each group is summed token by token from
+  +0.0 (tokens >= N skipped, so an empty group is +0.0), the block partial is
+  the pairwise tree ((g0 + g1) + (g2 + g3)) + ((g4 + g5) + (g6 + g7)), the
+  block partials are added one by one in block order from +0.0, and the total
+  is divided by float(N) with one IEEE division.
 * Q and K - mean(K) get symmetric INT8 codes per (batch, head, 128-token
   block) over all channels: amax = max |x| over the block's real tokens and
   channels; inv = 127 / amax (one IEEE float32 division; 0 when amax = 0);
@@ -73,6 +75,9 @@ def to_hnd(x, layout: str) -> np.ndarray:
     return np.ascontiguousarray(x)
 
 
+GROUPS, GROUP = 8, 16     # a 128-token block = 8 groups of 16 consecutive tokens
+
+
 def k_token_mean(k: np.ndarray) -> np.ndarray:
     """Per-channel mean of K over tokens, in the fixed float32 order described above.
 
@@ -82,11 +87,15 @@ def k_token_mean(k: np.ndarray) -> np.ndarray:
     nb = n_blocks(N)
     kp = np.zeros((B, H, nb * BLOCK, d), F32)
     kp[:, :, :N] = k
-    kb = kp.reshape(B, H, nb, BLOCK, d)
-    part = np.zeros((B, H, nb, d), F32)
-    for t in range(BLOCK):
-        valid = (np.arange(nb) * BLOCK + t) < N          # skip tokens beyond N
-        part = np.where(valid[None, None, :, None], part + kb[:, :, :, t, :], part)
+    kg = kp.reshape(B, H, nb, GROUPS, GROUP, d)
+    tok = (np.arange(nb)[:, None, None] * BLOCK + np.arange(GROUPS)[None, :, None] * GROUP
+           + np.arange(GROUP)[None, None, :])                # token index of (block, group, t)
+    gs = np.zeros((B, H, nb, GROUPS, d), F32)
+    for t in range(GROUP):
+        valid = tok[:, :, t] < N                          # skip tokens beyond N
+        gs = np.where(valid[None, None, :, :, None], gs + kg[:, :, :, :, t, :], gs)
+    part = ((gs[:, :, :, 0] + gs[:, :, :, 1]) + (gs[:, :, :, 2] + gs[:, :, :, 3])) + \
+           ((gs[:, :, :, 4] + gs[:, :, :, 5]) + (gs[:, :, :, 6] + gs[:, :, :, 7]))
     total = np.zeros((B, H, d), F32)
     for b in range(nb):
         total = total + part[:, :, b, :]

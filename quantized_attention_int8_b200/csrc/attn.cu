@@ -26,6 +26,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 
+#include <atomic>
 #include <climits>
 
 #include "sage_internal.h"
@@ -489,12 +490,26 @@ __global__ void __launch_bounds__(128, 1)
 // ------------------------------------------------------------------------------------------------
 // launchers
 // ------------------------------------------------------------------------------------------------
+// Sets a kernel's dynamic shared-memory limit once per device (the attribute is per device).
+template <typename K>
+static cudaError_t ensure_smem_limit(K kern, int bytes, std::atomic<unsigned long long>& done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = dev < 64 ? (1ull << dev) : 0ull;
+  if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+  return e;
+}
+
 template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, cudaStream_t st) {
   using C = FwdCfg<DQK, DV>;
   auto kern = sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nblk, p.Hq * p.n_vhalves, p.B);
   kern<<<grid, 192, C::SMEM, st>>>(tq, tk, tv, p);
@@ -540,7 +555,8 @@ static cudaError_t launch_qk_dump_t(const CUtensorMap& tq, const CUtensorMap& tk
                                     cudaStream_t st) {
   using C = FwdCfg<DQK, 64>;
   const int smem = 1024 + C::Q_BYTES + C::K_BYTES + C::BAR_BYTES;
-  cudaError_t e = cudaFuncSetAttribute(sage_qk_dump_kernel<DQK>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = ensure_smem_limit(sage_qk_dump_kernel<DQK>, smem, attr_done);
   if (e != cudaSuccess) return e;
   sage_qk_dump_kernel<DQK><<<p.n_tiles, 128, smem, st>>>(tq, tk, p);
   return cudaGetLastError();

@@ -16,6 +16,12 @@
 // this library's readings of what the pages leave open; every float operation
 // below is an explicit IEEE round-to-nearest operation (__fadd_rn, __fmul_rn,
 // __fdiv_rn) so the results are reproducible bit for bit.
+//
+// Thread layout: a CTA of dp threads covers one 128-token block; thread t owns
+// the register tile "group g = t / (dp/8) (tokens 16g .. 16g+15) x channel
+// vector cv = t % (dp/8) (channels 8cv .. 8cv+7)", loaded as sixteen 16-byte
+// vectors.  The K token sum of a block is the pairwise tree over its 8 group
+// sums, each group summed token by token.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -27,41 +33,53 @@ namespace sage {
 __device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
-// Copy rows [n0, n0 + rows) of one head into a zero-padded shared tile
-// tile[128][dp] (16-bit elements, row stride dp).
+// Element e (0..7) of a 16-byte vector of 16-bit values, widened exactly to float.
 template <typename T>
-__device__ void load_tile(T* tile, const T* __restrict__ x, int b, int h, int H, int N, int d, int dp, int n0,
-                          int rows, int layout, bool vec) {
-  const int tid = threadIdx.x, nthr = blockDim.x;
-  // zero the whole tile first (padding rows and channels)
-  uint4* t4 = reinterpret_cast<uint4*>(tile);
-  const int n16 = 128 * dp * (int)sizeof(T) / 16;
-  for (int i = tid; i < n16; i += nthr) t4[i] = make_uint4(0, 0, 0, 0);
-  __syncthreads();
-  auto row_ptr = [&](int n) -> const T* {
-    const size_t off = (layout == SAGE_HND) ? ((size_t)(b * H + h) * N + n) * d : ((size_t)(b * N + n) * H + h) * d;
-    return x + off;
-  };
-  if (vec) {
-    const int vpr = d / 8;  // 16-byte vectors per row
-    for (int i = tid; i < rows * vpr; i += nthr) {
-      const int r = i / vpr, cv = i - r * vpr;
-      const uint4 val = __ldg(reinterpret_cast<const uint4*>(row_ptr(n0 + r)) + cv);
-      *reinterpret_cast<uint4*>(tile + r * dp + cv * 8) = val;
-    }
-  } else {
-    for (int i = tid; i < rows * d; i += nthr) {
-      const int r = i / d, c = i - r * d;
-      tile[r * dp + c] = row_ptr(n0 + r)[c];
+__device__ __forceinline__ float elem(const uint4& v, int e) {
+  const uint32_t w = (&v.x)[e >> 1];
+  const unsigned short h = (e & 1) ? (unsigned short)(w >> 16) : (unsigned short)(w & 0xFFFF);
+  T t;
+  *reinterpret_cast<unsigned short*>(&t) = h;
+  return to_f32(t);
+}
+
+struct TileCoord {
+  int g, cv, c0;  // token group, channel vector, first channel
+};
+
+__device__ __forceinline__ TileCoord tile_coord(int dp) {
+  const int nv = dp / 8;
+  return TileCoord{(int)threadIdx.x / nv, (int)threadIdx.x % nv, ((int)threadIdx.x % nv) * 8};
+}
+
+// Load this thread's 16 x 8 register tile of one head: tokens n0+16g+r (r < 16), channels c0..c0+7.
+// Tokens >= n0+rows and channels >= d read as zero.
+template <typename T>
+__device__ __forceinline__ void load_tile(uint4 (&v)[16], const T* __restrict__ x, int b, int h, int H, int N, int d,
+                                          int n0, int rows, int layout, bool vec, const TileCoord& tc) {
+  const size_t hstride = (layout == SAGE_HND) ? (size_t)d : (size_t)H * d;  // elements between tokens
+  const size_t base = (layout == SAGE_HND) ? ((size_t)(b * H + h) * N + n0) * d : ((size_t)b * N + n0) * H * d + (size_t)h * d;
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int n = tc.g * 16 + r;
+    v[r] = make_uint4(0, 0, 0, 0);
+    if (n < rows && tc.c0 < d) {
+      const T* src = x + base + (size_t)n * hstride + tc.c0;
+      if (vec) {
+        v[r] = __ldg(reinterpret_cast<const uint4*>(src));
+      } else {
+        unsigned short e[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) e[k] = (tc.c0 + k < d) ? *reinterpret_cast<const unsigned short*>(src + k) : 0;
+        v[r] = make_uint4(e[0] | (e[1] << 16), e[2] | (e[3] << 16), e[4] | (e[5] << 16), e[6] | (e[7] << 16));
+      }
     }
   }
-  __syncthreads();
 }
 
 __device__ __forceinline__ float block_max(float v, float* red) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  __syncthreads();
   if ((threadIdx.x & 31) == 0) red[w] = v;
   __syncthreads();
   float r = 0.f;
@@ -69,65 +87,94 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
-// INT8 codes of a 128 x dp tile: x(r, c) is given by `val`, which must return 0
-// for padding.  Writes 128*dp bytes contiguously at `dst`.
+// INT8 codes of this thread's tile, x(r, k) given by `val`; row r of the tile goes to dst_row(r).
 template <typename F>
-__device__ void write_int8_codes(int8_t* __restrict__ dst, int dp, float inv, F val) {
-  const int nchunk = 128 * dp / 16;
-  for (int o = threadIdx.x; o < nchunk; o += blockDim.x) {
-    const int r = (o * 16) / dp, c0 = (o * 16) - r * dp;
-    uint32_t w[4];
+__device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp, const TileCoord& tc, float inv, F val) {
 #pragma unroll
-    for (int g = 0; g < 4; ++g) {
+  for (int r = 0; r < 16; ++r) {
+    uint32_t w[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
       uint32_t packed = 0;
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
-        int code = __float2int_rn(__fmul_rn(val(r, c0 + g * 4 + e), inv));  // rint: ties to even
+        int code = __float2int_rn(__fmul_rn(val(r, half * 4 + e), inv));  // rint: ties to even
         code = max(-127, min(127, code));
         packed |= (uint32_t)(code & 0xFF) << (8 * e);
       }
-      w[g] = packed;
+      w[half] = packed;
     }
-    *reinterpret_cast<uint4*>(dst + (size_t)o * 16) = make_uint4(w[0], w[1], w[2], w[3]);
+    *reinterpret_cast<uint2*>(dst + (size_t)(tc.g * 16 + r) * dp + tc.c0) = make_uint2(w[0], w[1]);
   }
+}
+
+// Column reduction over the 8 groups of a block: part[g][c] in shared memory -> channel c = threadIdx.x.
+__device__ __forceinline__ float tree8_sum(const float* part, int dp, int c) {
+  const float* p = part + c;
+  return __fadd_rn(__fadd_rn(__fadd_rn(p[0], p[dp]), __fadd_rn(p[2 * dp], p[3 * dp])),
+                   __fadd_rn(__fadd_rn(p[4 * dp], p[5 * dp]), __fadd_rn(p[6 * dp], p[7 * dp])));
+}
+__device__ __forceinline__ float tree8_max(const float* part, int dp, int c) {
+  const float* p = part + c;
+  float m = p[0];
+#pragma unroll
+  for (int g = 1; g < 8; ++g) m = fmaxf(m, p[g * dp]);
+  return m;
 }
 
 template <typename T>
 __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* tile = reinterpret_cast<T*>(smem_raw);
   __shared__ float red[8];
+  __shared__ float part[8 * 256];
   const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
   const int n0 = blk * 128, rows = min(128, p.N - n0);
   const int dp = p.dp, d = p.d;
+  const TileCoord tc = tile_coord(dp);
+  uint4 v[16];
   if (y < p.Hq) {  // ---- Q: final INT8 codes and per-block scale
     const int h = y;
-    load_tile<T>(tile, static_cast<const T*>(p.q), b, h, p.Hq, p.N, d, dp, n0, rows, p.layout, p.vec_q);
+    load_tile<T>(v, static_cast<const T*>(p.q), b, h, p.Hq, p.N, d, n0, rows, p.layout, p.vec_q, tc);
     float am = 0.f;
-    for (int i = threadIdx.x; i < rows * dp; i += blockDim.x) am = fmaxf(am, fabsf(to_f32(tile[i])));
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(elem<T>(v[r], e)));
     am = block_max(am, red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
     const size_t bh = (size_t)b * p.Hq + h;
-    write_int8_codes(p.q8 + (bh * p.Np + n0) * dp, dp, inv, [&](int r, int c) { return to_f32(tile[r * dp + c]); });
+    store_int8_tile(p.q8 + (bh * p.Np + n0) * dp, dp, tc, inv, [&](int r, int e) { return elem<T>(v[r], e); });
     if (threadIdx.x == 0) p.qs[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
-  } else if (y < p.Hq + p.Hkv) {  // ---- K: per-block partial column sums, token by token
+  } else if (y < p.Hq + p.Hkv) {  // ---- K: per-block partial column sums
     const int h = y - p.Hq;
-    load_tile<T>(tile, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, dp, n0, rows, p.layout, p.vec_k);
+    load_tile<T>(v, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_k, tc);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      if (tc.g * 16 + r < rows)  // tokens beyond N are skipped, not added as zeros
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], elem<T>(v[r], e));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = acc[e];
+    __syncthreads();
     const size_t base = (((size_t)b * p.Hkv + h) * p.nblk + blk) * dp;
-    for (int c = threadIdx.x; c < dp; c += blockDim.x) {
-      float acc = 0.f;
-      for (int r = 0; r < rows; ++r) acc = __fadd_rn(acc, to_f32(tile[r * dp + c]));
-      p.ksum_part[base + c] = acc;
-    }
+    p.ksum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
   } else {  // ---- V: per-block partial column amax
     const int h = y - p.Hq - p.Hkv;
-    load_tile<T>(tile, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, dp, n0, rows, p.layout, p.vec_v);
+    load_tile<T>(v, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_v, tc);
+    float am[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) am[e] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am[e] = fmaxf(am[e], fabsf(elem<T>(v[r], e)));
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = am[e];
+    __syncthreads();
     const size_t base = (((size_t)b * p.Hkv + h) * p.nblk + blk) * dp;
-    for (int c = threadIdx.x; c < dp; c += blockDim.x) {
-      float am = 0.f;
-      for (int r = 0; r < rows; ++r) am = fmaxf(am, fabsf(to_f32(tile[r * dp + c])));
-      p.vmax_part[base + c] = am;
-    }
+    p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
   }
 }
 
@@ -147,65 +194,67 @@ __global__ void quant_finalize_kernel(QuantParams p) {
   }
 }
 
+// Two E4M3 codes (RN, saturating) of a and b, a in the low byte.
+__device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
+  return __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3) & 0xFFFFu;
+}
+
 template <typename T>
 __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  T* tile = reinterpret_cast<T*>(smem_raw);
   __shared__ float red[8];
-  __shared__ float cvec[256];  // k_mean or v_inv of this head
   const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
   const int n0 = blk * 128, rows = min(128, p.N - n0);
   const int dp = p.dp, d = p.d;
+  const TileCoord tc = tile_coord(dp);
+  uint4 v[16];
   if (y < p.Hkv) {  // ---- K - mean(K): INT8 codes and per-block scale
     const int h = y;
     const size_t bh = (size_t)b * p.Hkv + h;
-    for (int c = threadIdx.x; c < dp; c += blockDim.x) cvec[c] = p.km[bh * dp + c];
-    load_tile<T>(tile, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, dp, n0, rows, p.layout, p.vec_k);
-    auto x = [&](int r, int c) -> float {
-      return (r < rows && c < d) ? __fsub_rn(to_f32(tile[r * dp + c]), cvec[c]) : 0.f;
+    float km[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) km[e] = p.km[bh * dp + tc.c0 + e];
+    load_tile<T>(v, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_k, tc);
+    auto x = [&](int r, int e) -> float {
+      return (tc.g * 16 + r < rows && tc.c0 + e < d) ? __fsub_rn(elem<T>(v[r], e), km[e]) : 0.f;
     };
     float am = 0.f;
-    for (int i = threadIdx.x; i < rows * dp; i += blockDim.x) am = fmaxf(am, fabsf(x(i / dp, i % dp)));
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+#pragma unroll
+      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x(r, e)));
     am = block_max(am, red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
-    write_int8_codes(p.k8 + (bh * p.Np + n0) * dp, dp, inv, x);
+    store_int8_tile(p.k8 + (bh * p.Np + n0) * dp, dp, tc, inv, x);
     if (threadIdx.x == 0) p.ks[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
   } else {  // ---- V: E4M3 codes, transposed to [channel][token]
     const int h = y - p.Hkv;
     const size_t bh = (size_t)b * p.Hkv + h;
-    for (int c = threadIdx.x; c < dp; c += blockDim.x) cvec[c] = p.vinv[bh * dp + c];
-    load_tile<T>(tile, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, dp, n0, rows, p.layout, p.vec_v);
-    const int nchunk = dp * 128 / 16;
-    for (int o = threadIdx.x; o < nchunk; o += blockDim.x) {
-      const int c = o % dp, r0 = (o / dp) * 16;
-      const float inv = cvec[c];
+    float inv[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) inv[e] = p.vinv[bh * dp + tc.c0 + e];
+    load_tile<T>(v, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_v, tc);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
       uint32_t w[4];
 #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float a0 = __fmul_rn(to_f32(tile[(r0 + 4 * g + 0) * dp + c]), inv);
-        const float a1 = __fmul_rn(to_f32(tile[(r0 + 4 * g + 1) * dp + c]), inv);
-        const float a2 = __fmul_rn(to_f32(tile[(r0 + 4 * g + 2) * dp + c]), inv);
-        const float a3 = __fmul_rn(to_f32(tile[(r0 + 4 * g + 3) * dp + c]), inv);
-        const uint32_t lo = __nv_cvt_float2_to_fp8x2(make_float2(a0, a1), __NV_SATFINITE, __NV_E4M3);
-        const uint32_t hi = __nv_cvt_float2_to_fp8x2(make_float2(a2, a3), __NV_SATFINITE, __NV_E4M3);
-        w[g] = (lo & 0xFFFF) | (hi << 16);
+      for (int q = 0; q < 4; ++q) {
+        const float a0 = __fmul_rn(elem<T>(v[4 * q + 0], e), inv[e]);
+        const float a1 = __fmul_rn(elem<T>(v[4 * q + 1], e), inv[e]);
+        const float a2 = __fmul_rn(elem<T>(v[4 * q + 2], e), inv[e]);
+        const float a3 = __fmul_rn(elem<T>(v[4 * q + 3], e), inv[e]);
+        w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
       }
-      *reinterpret_cast<uint4*>(p.v8t + (bh * dp + c) * p.Np + n0 + r0) = make_uint4(w[0], w[1], w[2], w[3]);
+      *reinterpret_cast<uint4*>(p.v8t + (bh * dp + tc.c0 + e) * p.Np + n0 + tc.g * 16) =
+          make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
 }
 
 template <typename T>
 static cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
-  const size_t smem = (size_t)128 * p.dp * sizeof(T);
-  cudaError_t e;
-  if ((e = cudaFuncSetAttribute(quant_pass1_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-    return e;
-  if ((e = cudaFuncSetAttribute(quant_pass2_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)))
-    return e;
-  quant_pass1_kernel<T><<<dim3(p.nblk, p.Hq + 2 * p.Hkv, p.B), 256, smem, st>>>(p);
-  quant_finalize_kernel<<<p.B * p.Hkv, 256, 0, st>>>(p);
-  quant_pass2_kernel<T><<<dim3(p.nblk, 2 * p.Hkv, p.B), 256, smem, st>>>(p);
+  quant_pass1_kernel<T><<<dim3(p.nblk, p.Hq + 2 * p.Hkv, p.B), p.dp, 0, st>>>(p);
+  quant_finalize_kernel<<<p.B * p.Hkv, p.dp, 0, st>>>(p);
+  quant_pass2_kernel<T><<<dim3(p.nblk, 2 * p.Hkv, p.B), p.dp, 0, st>>>(p);
   return cudaGetLastError();
 }
 

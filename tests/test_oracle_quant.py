@@ -40,14 +40,20 @@ def test_k_mean_exact_when_sums_are_exact():
 
 
 def test_k_mean_order_ragged_tail():
-    # Brute-force the stated order with python floats rounded to float32 at every step.
+    # Brute-force the stated order with numpy float32 scalars (each + rounds to float32):
+    # 16-token groups summed in order, a pairwise tree over the 8 groups of a block,
+    # then the blocks in order.
     k = (_rng(2).standard_normal((1, 1, 300, 3)) * 1000).astype(F32)
     for c in range(3):
         total = F32(0)
         for b0 in range(0, 300, 128):
-            part = F32(0)
-            for n in range(b0, min(b0 + 128, 300)):
-                part = F32(part + k[0, 0, n, c])
+            g = []
+            for g0 in range(b0, b0 + 128, 16):
+                acc = F32(0)
+                for n in range(g0, min(g0 + 16, 300)):
+                    acc = F32(acc + k[0, 0, n, c])
+                g.append(acc)
+            part = F32(F32(F32(g[0] + g[1]) + F32(g[2] + g[3])) + F32(F32(g[4] + g[5]) + F32(g[6] + g[7])))
             total = F32(total + part)
         assert quant.k_token_mean(k)[0, 0, c] == F32(total / F32(300))
 
