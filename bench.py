@@ -237,8 +237,14 @@ def run_ours(args, w):
     peak_tops = 2.0 * peaks["bf16"]
     achieved = ops / (k_ms * 1e-3) / 1e12
 
-    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element
-    qtimes = time_steps(lambda: qa.sage_quantize(qd, kd, vd, w.layout, pv), max(3, args.steps // 2), 2, flush)
+    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element;
+    # the C entry point on preallocated outputs, so the Python allocations are not timed
+    qargs = [qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), w.B, w.Hq, w.Hkv, w.N, w.d,
+             qa.SAGE_BF16 if qd.dtype == torch.bfloat16 else qa.SAGE_FP16,
+             qa.SAGE_HND if w.layout == "HND" else qa.SAGE_NHD, w.pv_mode,
+             *(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "km", "v8t", "vs")),
+             torch.cuda.current_stream().cuda_stream]
+    qtimes = time_steps(lambda: qa.capi.sage_quantize(*qargs), max(3, args.steps // 2), 3, flush)
     q_ms = statistics.mean(qtimes)
     q_bytes = 3 * (q.numel() + k.numel() + v.numel())
 

@@ -69,8 +69,11 @@ typedef enum { SAGE_PV_FP32 = 0, SAGE_PV_FP16_FP32 = 1 } sage_pv_mode;
 /* Quantized attention, end to end: quantize/smooth pass, then the fused
  * attention kernel.  q: (B,Hq,N,d), k and v: (B,Hkv,N,d), out: (B,Hq,N,d), all
  * in `layout`, dtype `dtype`.  sm_scale <= 0 or NaN selects 1/sqrt(d) (the
- * original d).  The quantized copies of Q/K/V live in a workspace taken with
- * cudaMallocAsync on `stream` and released stream-ordered before return;
+ * original d).  The quantized copies of Q/K/V live in a workspace taken
+ * stream-ordered on `stream` from a per-device memory pool that the library
+ * creates on first use and that keeps its memory for later calls (it holds as
+ * much device memory as the largest workspace in flight, until the process
+ * exits); the workspace is released stream-ordered before return.
  * SAGE_ERR_OOM if it cannot be allocated.  out must not overlap q, k or v. */
 sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
                       sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
@@ -93,7 +96,7 @@ size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * in order inside a block, then the block sums in order) and divided by N;
  * V: inv = VMAX / amax_channel, code = E4M3_rne_satfinite(v * inv),
  * vs = amax / VMAX with VMAX = 448 (SAGE_PV_FP32) or 1 (SAGE_PV_FP16_FP32).
- * Its own small scratch is taken with cudaMallocAsync on `stream`. */
+ * Its own small scratch comes from the same per-device pool as sage_attn's. */
 sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
                           sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,
                           int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs, void* stream);

@@ -100,6 +100,37 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
+// Workspace memory: a stream-ordered pool per device, owned by the library, that keeps the
+// memory it has handed out (release threshold = unlimited), so that repeated calls reuse
+// it instead of mapping fresh device memory each time.
+cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t st) {
+  constexpr int kMaxDevices = 128;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  cudaMemPool_t pool;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    if (!pools[dev]) {
+      cudaMemPoolProps props;
+      memset(&props, 0, sizeof(props));
+      props.allocType = cudaMemAllocationTypePinned;
+      props.location.type = cudaMemLocationTypeDevice;
+      props.location.id = dev;
+      cudaMemPool_t p = nullptr;
+      if ((e = cudaMemPoolCreate(&p, &props)) != cudaSuccess) return e;
+      uint64_t keep = ~0ull;
+      if ((e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) return e;
+      pools[dev] = p;
+    }
+    pool = pools[dev];
+  }
+  return cudaMallocFromPoolAsync(ptr, bytes, pool, st);
+}
+
 struct QuantBufs {
   int8_t* q8;
   float* qs;
@@ -203,7 +234,7 @@ sage_status sage_attn(const void* q, const void* k, const void* v, void* out, in
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const WsLayout w = ws_layout(m);
   unsigned char* ws = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&ws), w.total, st);
+  cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), w.total, st);
   if (e != cudaSuccess) return from_cuda(e);
   QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
   QuantBufs qb{reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
@@ -233,7 +264,7 @@ sage_status sage_quantize(const void* q, const void* k, const void* v, int B, in
   const size_t part = align_up((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
   const size_t vinv = align_up((size_t)m.B * m.Hkv * m.dp * 4);
   unsigned char* scratch = nullptr;
-  cudaError_t e = cudaMallocAsync(reinterpret_cast<void**>(&scratch), 2 * part + vinv, st);
+  cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&scratch), 2 * part + vinv, st);
   if (e != cudaSuccess) return from_cuda(e);
   QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
   qp.q8 = q8, qp.qs = qs, qp.k8 = k8, qp.ks = ks, qp.km = km, qp.v8t = v8t, qp.vs = vs;
