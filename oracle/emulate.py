@@ -13,14 +13,19 @@ SageAttention README, "Current Features"; qwbw.cn article, pitfalls, for the
 2. Dequantize in the log2 domain: s = S * f with
    f = (qs * ks) * (sm_scale * log2(e)), all float32.  Keys j >= N, and
    j > i under the causal mask, are excluded.
-3. Online softmax: m' = max(m, row max of s); p = 2^(s - m');
-   alpha = 2^(m - m'); l = l * alpha + sum(p).
-4. P is stored as E4M3(p * 448).
+3. Online softmax against a reference max m: the reference moves to
+   m' = max(m, row max of s) only when that exceeds m by more than
+   tau = 2 (log2 units), else it stays (m' = m); p = 2^(s - m') <= 2^tau;
+   alpha = 2^(m - m') (1 when it stays); l = l * alpha + sum(p).  With
+   tau = 0 this is the textbook online softmax; tau = 2 is how the CUDA
+   kernel runs it (it rescales O only when the reference moves), and the
+   result is the same up to rounding because O and l share the reference.
+4. P is stored as E4M3(p * 448 * 2^-tau), so codes stay within +-448.
 5. PV: mode 0 (fp32 accumulation) O = O * alpha + P8 . V8;
    mode 1 (fp16+fp32, "two-level accumulation") the tile's P8 . V8 is first
    rounded to float16 (a fresh fp16 accumulator per tile), then
    O = O * alpha + T.
-6. out = O * vs / (448 * l), rounded to the output dtype by the caller.
+6. out = O * vs / (448 * 2^-tau * l), rounded to the output dtype by the caller.
 """
 from __future__ import annotations
 
@@ -30,9 +35,10 @@ from . import fp8
 from .quant import BLOCK, P_SCALE, F32
 
 LOG2E = 1.4426950408889634
+TAU = 2.0  # reference-max slack of the CUDA kernel's online softmax (log2 units)
 
 
-def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None):
+def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, tau: float = TAU):
     """Emulated output float32 (len(heads), len(q_blocks) * 128, d) in HND row order.
 
     ``qz`` is the dict from ``quant.quantize``.  ``heads`` lists (b, hq) pairs
@@ -46,6 +52,7 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None):
     hs = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
     qbs = list(range(nb)) if q_blocks is None else list(q_blocks)
     c = F32(F32(sm_scale) * F32(LOG2E))
+    pscale = F32(P_SCALE * 2.0 ** -tau)  # exact: 448 * 2^-tau
     out = np.full((len(hs), len(qbs) * BLOCK, d), np.nan, F32)
     for n, (b, h) in enumerate(hs):
         hk = h // G
@@ -68,21 +75,24 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None):
                 smax = np.where(valid, S, np.iinfo(np.int64).min).max(axis=1)
                 has = valid.any(axis=1)
                 tmax = np.where(has, smax.astype(F32) * f, F32(-np.inf)).astype(F32)
-                m_new = np.maximum(m, tmax)
+                mc = np.maximum(m, tmax)
+                upd = mc > (m + F32(tau)).astype(F32)             # the reference max moves
+                m_new = np.where(upd, mc, m).astype(F32)
                 with np.errstate(invalid="ignore"):
                     arg = (S.astype(np.float64) * np.float64(f) - m_new[:, None].astype(np.float64)).astype(F32)
                 p = np.where(valid, np.exp2(arg), F32(0)).astype(F32)
-                alpha = np.where(np.isneginf(m), F32(0), np.exp2((m - m_new).astype(F32))).astype(F32)
-                alpha = np.where(np.isneginf(m_new), F32(1), alpha).astype(F32)
+                with np.errstate(invalid="ignore"):
+                    alpha = np.where(np.isneginf(m), F32(0), np.exp2((m - m_new).astype(F32))).astype(F32)
+                alpha = np.where(upd, alpha, F32(1)).astype(F32)
                 l = (l * alpha + p.sum(axis=1, dtype=F32)).astype(F32)
-                p8 = fp8.decode(fp8.encode((p * F32(P_SCALE)).astype(F32)))
+                p8 = fp8.decode(fp8.encode((p * pscale).astype(F32)))
                 pv = p8 @ v8[j * BLOCK:(j + 1) * BLOCK]                  # exact in float64
                 if mode == 1:
                     pv = pv.astype(np.float16)
                 O = (O * alpha[:, None] + pv.astype(F32)).astype(F32)
                 m = m_new
             vs = qz["vs"][b, hk].astype(F32)
-            o = (O * vs[None, :] / (F32(P_SCALE) * l[:, None])).astype(F32)
+            o = (O * vs[None, :] / (pscale * l[:, None])).astype(F32)
             ok = rows < N
             out[n, r * BLOCK:(r + 1) * BLOCK][ok] = o[ok, :d]
     return out

@@ -103,6 +103,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 }
 
 constexpr float kLog2_448 = 8.807354922057604f;  // p * 448 = 2^(log2 p + log2 448)
+constexpr float kTau = 2.0f;                       // reference-max slack of the online softmax (log2 units)
 
 template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
 __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
@@ -244,7 +245,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     const float qsv = p.qs[((size_t)b * p.Hq + hq) * p.nblk + qt];
     const float* ksp = p.ks + ((size_t)b * p.Hkv + hkv) * p.nblk;
     unsigned char* prow = sP + row * 128;
-    float m = -INFINITY, l = 0.f;  // l accumulates p * 448
+    float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates p * 448 * 2^-kTau
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
       if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
@@ -280,72 +281,70 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
       for (int c = 8; c < 128; ++c) mx8[c & 7] = max(mx8[c & 7], (int)s[c]);
       const int mx = max(max(max(mx8[0], mx8[1]), max(mx8[2], mx8[3])), max(max(mx8[4], mx8[5]), max(mx8[6], mx8[7])));
       const float mt = (mx == INT_MIN) ? -INFINITY : __fmul_rn((float)mx, f);
-      const float m_new = fmaxf(m, mt);
-      const float alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - m_new);
-      const float bias = (m_new == -INFINITY) ? 0.f : kLog2_448 - m_new;
-      if (MODE == 0 && i > 0) {
-        // P's buffer and O were last used by the P.V MMA of tile i-1
-        if (!warp_wait(&bars->pv_done, (i - 1) & 1, abort)) { ok = false; break; }
-        tc_fence_after();
-        if (DV == 64 && __any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll 1
-          for (int cc = 0; cc < DV / 16; ++cc) {
-            uint32_t o[16];
-            tmem_ld16(ocol + cc * 16, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int e = 0; e < 16; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st16(ocol + cc * 16, o);
-          }
-          tmem_wait_st();
-        }
-      }
-      // p * 448 = 2^(s*f - m' + log2 448) -> E4M3, 16 keys (one 16-byte chunk) at a time
+      // The reference max m moves only when the running max exceeds it by more than kTau,
+      // so O is rescaled rarely; p = 2^(s - m) <= 2^kTau is stored as E4M3(p * 448 * 2^-kTau).
+      const float mc = fmaxf(m, mt);
+      const bool upd = mc > __fadd_rn(m, kTau);
+      const float m_new = upd ? mc : m;
+      const float alpha = upd ? ((m == -INFINITY) ? 0.f : ex2_approx(m - m_new)) : 1.f;
+      const float bias = (m_new == -INFINITY) ? 0.f : (kLog2_448 - kTau) - m_new;
+      const bool rescale = MODE == 0 && i > 0 && __any_sync(0xffffffffu, alpha != 1.f);
+      // p * 448 * 2^-kTau = 2^(s*f - m + log2 448 - kTau) -> E4M3, 4 keys per 32-bit word
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
+      uint32_t pw[32];
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch) {
-        uint32_t w[4];
+      for (int c4 = 0; c4 < 32; ++c4) {
+        float pv[4];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          float pv[4];
-#pragma unroll
-          for (int e = 0; e < 4; e += 2) {
-            const int c = ch * 16 + c4 * 4 + e;
-            float x0, x1;
-            if (DQK >= 128 && MODE == 0) {  // packed FMA measured faster only in this configuration
-              const float2 x = __ffma2_rn(make_float2((float)(int)s[c], (float)(int)s[c + 1]), make_float2(f, f),
-                                          make_float2(bias, bias));
-              x0 = x.x;
-              x1 = x.y;
-            } else {
-              x0 = fmaf((float)(int)s[c], f, bias);
-              x1 = fmaf((float)(int)s[c + 1], f, bias);
-            }
-            pv[e] = ex2_approx(x0);
-            pv[e + 1] = ex2_approx(x1);
-            if (edge) {
-              pv[e] = (c < lim) ? pv[e] : 0.f;
-              pv[e + 1] = (c + 1 < lim) ? pv[e + 1] : 0.f;
-            }
-            rs[e] += pv[e];
-            rs[e + 1] += pv[e + 1];
+        for (int e = 0; e < 4; e += 2) {
+          const int c = c4 * 4 + e;
+          float x0, x1;
+          if (DQK >= 128 && MODE == 0) {  // packed FMA measured faster only in this configuration
+            const float2 x = __ffma2_rn(make_float2((float)(int)s[c], (float)(int)s[c + 1]), make_float2(f, f),
+                                        make_float2(bias, bias));
+            x0 = x.x;
+            x1 = x.y;
+          } else {
+            x0 = fmaf((float)(int)s[c], f, bias);
+            x1 = fmaf((float)(int)s[c + 1], f, bias);
           }
-          w[c4] = e4m3x2(pv[0], pv[1]) | (e4m3x2(pv[2], pv[3]) << 16);
+          pv[e] = ex2_approx(x0);
+          pv[e + 1] = ex2_approx(x1);
+          if (edge) {
+            pv[e] = (c < lim) ? pv[e] : 0.f;
+            pv[e + 1] = (c + 1 < lim) ? pv[e + 1] : 0.f;
+          }
+          rs[e] += pv[e];
+          rs[e + 1] += pv[e + 1];
         }
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) = make_uint4(w[0], w[1], w[2], w[3]);
+        pw[c4] = e4m3x2(pv[0], pv[1]) | (e4m3x2(pv[2], pv[3]) << 16);
       }
-      fence_proxy_async_smem();
       l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       m = m_new;
-      if (MODE == 0 && DV == 128 && i > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        uint32_t o[DV];
+      if (MODE == 0 && i > 0) {
+        // P's buffer and O were last used by the P.V MMA of tile i-1 (long done by now)
+        if (!warp_wait(&bars->pv_done, (i - 1) & 1, abort)) { ok = false; break; }
+        tc_fence_after();
+      }
 #pragma unroll
-        for (int cc = 0; cc < DV / 32; ++cc) tmem_ld32(ocol + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[cc * 32]));
-        tmem_wait_ld();
+      for (int ch = 0; ch < 8; ++ch)
+        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+            make_uint4(pw[ch * 4 + 0], pw[ch * 4 + 1], pw[ch * 4 + 2], pw[ch * 4 + 3]);
+      fence_proxy_async_smem();
+      if (rescale) {
+        // O *= alpha (rows whose reference did not move have alpha = 1); 64 columns per batch,
+        // every TMEM load of a batch in flight before one wait
 #pragma unroll
-        for (int e = 0; e < DV; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+        for (int hh = 0; hh < DV / 64; ++hh) {
+          uint32_t o[64];
+          tmem_ld32(ocol + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_ld32(ocol + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+          tmem_wait_ld();
 #pragma unroll
-        for (int cc = 0; cc < DV / 32; ++cc) tmem_st32(ocol + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&o[cc * 32]));
+          for (int e = 0; e < 64; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+          tmem_st32(ocol + hh * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_st32(ocol + hh * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
+        }
         tmem_wait_st();
       }
       tc_fence_before();
@@ -361,10 +360,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
         for (int cc = 0; cc < DV / 32; ++cc) {
           uint32_t t[16], o0[16], o1[16];
           tmem_ld16_pack16(tcol + cc * 32, t);
-          if (i > 0) {
-            tmem_ld16(ocol + cc * 32, o0);
-            tmem_ld16(ocol + cc * 32 + 16, o1);
-          }
+          // O holds nothing yet on tile 0; it is loaded anyway (and discarded below) so that
+          // the load's outputs are defined on every path
+          tmem_ld16(ocol + cc * 32, o0);
+          tmem_ld16(ocol + cc * 32 + 16, o1);
           tmem_wait_ld();
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
