@@ -33,6 +33,8 @@
 #include "sm100.cuh"
 
 namespace sage {
+// CTAs that arrived on each SM so far (only the parity is used; see the stagger below).
+__device__ unsigned int g_sm_arrivals[256];
 
 template <int DQK, int DV>
 struct FwdCfg {
@@ -89,7 +91,7 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
 // Bounded wait used only while winding down (ignores the abort flag).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
   const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) {
     if (clock64() - t0 > kWaitBudgetCycles) {
       atomicOr(&g_device_error, SAGE_DEVERR_TIMEOUT);
       return;
@@ -237,6 +239,20 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
+    {
+      // Two CTAs share an SM and the same MUFU units.  Started together they stay in step,
+      // both in their exponential loops at once (each at half the MUFU rate) and both in their
+      // other work at once (MUFU idle).  Every second CTA to arrive on an SM therefore starts
+      // its softmax about a third of a tile later; measured +2.5% to +6% on the fused kernel.
+      __shared__ unsigned int slot;
+      if (threadIdx.x == 0) {
+        unsigned int smid;
+        asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
+        slot = atomicAdd(&g_sm_arrivals[smid & 255], 1u) & 1u;
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (slot) __nanosleep(300);
+    }
     const int row = warp * 32 + lane;            // query row inside the tile, TMEM lane
     const int grow = qt * 128 + row;             // query row in the sequence
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;

@@ -58,13 +58,29 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   return ok != 0;
 }
 
+// try_wait that may suspend the thread (up to about `hint_ns`) until the phase completes,
+// instead of returning at once: waiting warps then take no issue slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t* bar, uint32_t parity, uint32_t hint_ns) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
+      : "memory");
+  return ok != 0;
+}
+
+constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms per suspension; the budget below still bounds the wait
+
 // Bounded wait for the phase with the given parity.  Returns false (and
 // records a timeout) if the budget runs out or *abort is already set.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitBudgetCycles) {
       atomicOr(&g_device_error, SAGE_DEVERR_TIMEOUT);
