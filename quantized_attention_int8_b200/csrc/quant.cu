@@ -43,6 +43,44 @@ __device__ __forceinline__ float elem(const uint4& v, int e) {
   return to_f32(t);
 }
 
+// Packed pairs of 16-bit floats.
+template <typename T>
+struct Pair2;
+template <>
+struct Pair2<__half> {
+  using type = __half2;
+};
+template <>
+struct Pair2<__nv_bfloat16> {
+  using type = __nv_bfloat162;
+};
+
+// Running max of |x| over packed 16-bit floats, on their bit patterns: with the sign bit
+// cleared, the bit-pattern order of finite 16-bit floats is their magnitude order.
+__device__ __forceinline__ uint32_t absmax_bits(uint32_t acc, uint32_t w) { return __vmaxu2(acc, w & 0x7FFF7FFFu); }
+
+template <typename T>
+__device__ __forceinline__ float bits_to_f32(uint32_t h16) {
+  T t;
+  *reinterpret_cast<unsigned short*>(&t) = (unsigned short)h16;
+  return to_f32(t);
+}
+
+// max |x| of this thread's register tile (padding reads as zero and cannot raise it)
+template <typename T>
+__device__ __forceinline__ float tile_absmax(const uint4 (&v)[16]) {
+  uint32_t a0 = 0, a1 = 0, a2 = 0, a3 = 0;
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    a0 = absmax_bits(a0, v[r].x);
+    a1 = absmax_bits(a1, v[r].y);
+    a2 = absmax_bits(a2, v[r].z);
+    a3 = absmax_bits(a3, v[r].w);
+  }
+  const uint32_t a = __vmaxu2(__vmaxu2(a0, a1), __vmaxu2(a2, a3));
+  return bits_to_f32<T>(max(a & 0xFFFFu, a >> 16));
+}
+
 struct TileCoord {
   int g, cv, c0;  // token group, channel vector, first channel
 };
@@ -87,11 +125,14 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
-// INT8 codes of this thread's tile, x(r, k) given by `val`; row r of the tile goes to dst_row(r).
+// INT8 codes of this thread's tile, x(r, k) given by `val`; rows at or beyond `rows` (tokens
+// past N) get code 0 whatever `val` returns for them.
 template <typename F>
-__device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp, const TileCoord& tc, float inv, F val) {
+__device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp, const TileCoord& tc, float inv, int rows,
+                                                F val) {
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
+    const bool valid = tc.g * 16 + r < rows;
     uint32_t w[2];
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
@@ -102,7 +143,7 @@ __device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp
         code = max(-127, min(127, code));
         packed |= (uint32_t)(code & 0xFF) << (8 * e);
       }
-      w[half] = packed;
+      w[half] = valid ? packed : 0u;
     }
     *reinterpret_cast<uint2*>(dst + (size_t)(tc.g * 16 + r) * dp + tc.c0) = make_uint2(w[0], w[1]);
   }
@@ -134,15 +175,10 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
   if (y < p.Hq) {  // ---- Q: final INT8 codes and per-block scale
     const int h = y;
     load_tile<T>(v, static_cast<const T*>(p.q), b, h, p.Hq, p.N, d, n0, rows, p.layout, p.vec_q, tc);
-    float am = 0.f;
-#pragma unroll
-    for (int r = 0; r < 16; ++r)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(elem<T>(v[r], e)));
-    am = block_max(am, red);
+    const float am = block_max(tile_absmax<T>(v), red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
     const size_t bh = (size_t)b * p.Hq + h;
-    store_int8_tile(p.q8 + (bh * p.Np + n0) * dp, dp, tc, inv, [&](int r, int e) { return elem<T>(v[r], e); });
+    store_int8_tile(p.q8 + (bh * p.Np + n0) * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); });
     if (threadIdx.x == 0) p.qs[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
   } else if (y < p.Hq + p.Hkv) {  // ---- K: per-block partial column sums
     const int h = y - p.Hq;
@@ -163,15 +199,19 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
   } else {  // ---- V: per-block partial column amax
     const int h = y - p.Hq - p.Hkv;
     load_tile<T>(v, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_v, tc);
-    float am[8];
+    uint32_t a[4] = {0, 0, 0, 0};  // channels (2e, 2e+1), |x| as bit patterns
 #pragma unroll
-    for (int e = 0; e < 8; ++e) am[e] = 0.f;
+    for (int r = 0; r < 16; ++r) {
+      a[0] = absmax_bits(a[0], v[r].x);
+      a[1] = absmax_bits(a[1], v[r].y);
+      a[2] = absmax_bits(a[2], v[r].z);
+      a[3] = absmax_bits(a[3], v[r].w);
+    }
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) am[e] = fmaxf(am[e], fabsf(elem<T>(v[r], e)));
-#pragma unroll
-    for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = am[e];
+    for (int e = 0; e < 4; ++e) {
+      part[tc.g * dp + tc.c0 + 2 * e] = bits_to_f32<T>(a[e] & 0xFFFFu);
+      part[tc.g * dp + tc.c0 + 2 * e + 1] = bits_to_f32<T>(a[e] >> 16);
+    }
     __syncthreads();
     const size_t base = (((size_t)b * p.Hkv + h) * p.nblk + blk) * dp;
     p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
@@ -184,7 +224,8 @@ __global__ void quant_finalize_kernel(QuantParams p) {
     const float* ks = p.ksum_part + (size_t)bh * p.nblk * p.dp + c;
     const float* vm = p.vmax_part + (size_t)bh * p.nblk * p.dp + c;
     float acc = 0.f, am = 0.f;
-    for (int i = 0; i < p.nblk; ++i) {
+#pragma unroll 8
+    for (int i = 0; i < p.nblk; ++i) {  // sums stay in block order; the loads overlap
       acc = __fadd_rn(acc, ks[(size_t)i * p.dp]);
       am = fmaxf(am, vm[(size_t)i * p.dp]);
     }
@@ -214,17 +255,43 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) km[e] = p.km[bh * dp + tc.c0 + e];
     load_tile<T>(v, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_k, tc);
-    auto x = [&](int r, int e) -> float {
-      return (tc.g * 16 + r < rows && tc.c0 + e < d) ? __fsub_rn(elem<T>(v[r], e), km[e]) : 0.f;
-    };
+    // padded channels read 0 and have mean 0; padded rows are masked by store_int8_tile
+    auto x = [&](int r, int e) -> float { return __fsub_rn(elem<T>(v[r], e), km[e]); };
+    // max |k - mean| per channel is reached at the channel's largest or smallest k, since
+    // rounding k - mean to float32 is monotonic in k: take per-channel extremes on the packed
+    // values, then subtract the mean from those two only.
+    using P2 = typename Pair2<T>::type;
+    P2 hi[4], lo[4];
+    bool any = false;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      if (tc.g * 16 + r < rows) {
+        const P2* w = reinterpret_cast<const P2*>(&v[r]);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hi[e] = any ? __hmax2(hi[e], w[e]) : w[e];
+          lo[e] = any ? __hmin2(lo[e], w[e]) : w[e];
+        }
+        any = true;
+      }
+    }
     float am = 0.f;
+    if (any) {
 #pragma unroll
-    for (int r = 0; r < 16; ++r)
-#pragma unroll
-      for (int e = 0; e < 8; ++e) am = fmaxf(am, fabsf(x(r, e)));
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi[e]);
+        const uint32_t lb = *reinterpret_cast<const uint32_t*>(&lo[e]);
+        if (tc.c0 + 2 * e < d)
+          am = fmaxf(am, fmaxf(fabsf(__fsub_rn(bits_to_f32<T>(hb & 0xFFFFu), km[2 * e])),
+                               fabsf(__fsub_rn(bits_to_f32<T>(lb & 0xFFFFu), km[2 * e]))));
+        if (tc.c0 + 2 * e + 1 < d)
+          am = fmaxf(am, fmaxf(fabsf(__fsub_rn(bits_to_f32<T>(hb >> 16), km[2 * e + 1])),
+                               fabsf(__fsub_rn(bits_to_f32<T>(lb >> 16), km[2 * e + 1]))));
+      }
+    }
     am = block_max(am, red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
-    store_int8_tile(p.k8 + (bh * p.Np + n0) * dp, dp, tc, inv, x);
+    store_int8_tile(p.k8 + (bh * p.Np + n0) * dp, dp, tc, inv, rows, x);
     if (threadIdx.x == 0) p.ks[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
   } else {  // ---- V: E4M3 codes, transposed to [channel][token]
     const int h = y - p.Hkv;
