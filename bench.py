@@ -158,6 +158,19 @@ def cpu_oracle_sample(w: W.Workload, budget_s: float):
     return ops / dt / 1e12, threads, heads, dt
 
 
+def job_throughput(local_ms: float, ops_per_step: float, steps: int, dist=None, device=None):
+    """Whole-job TOPS for replicas: every rank ran `steps` steps of `ops_per_step` each in
+    `local_ms`; the job's time is the slowest rank's (one MAX all-reduce of a scalar, outside
+    the data path).  Returns (TOPS, max_ms)."""
+    world = 1
+    if dist is not None and dist.is_initialized():
+        world = dist.get_world_size()
+        t = torch.tensor([local_ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        local_ms = float(t.item())
+    return world * ops_per_step * steps / (local_ms * 1e-3) / 1e12, local_ms
+
+
 # ------------------------------------------------------------------------------------ arms
 def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
@@ -220,12 +233,7 @@ def run_ours(args, w):
     with ClockSampler(torch.cuda.current_device()) as clk:
         times = time_steps(step, args.steps, args.warmup, flush)
     qa.sage_check_status()
-    total_ms = sum(times)
-    if dist:
-        t = torch.tensor([total_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
-    value = world * ops * args.steps / (total_ms * 1e-3) / 1e12
+    value, total_ms = job_throughput(sum(times), ops, args.steps, dist, "cuda")
 
     # ---- the fused attention kernel alone (roofline)
     z = qa.sage_quantize(qd, kd, vd, w.layout, pv)
@@ -260,12 +268,7 @@ def run_ours(args, w):
         outh.copy_(o, non_blocking=True)
 
     etimes = time_steps(e2e_step, args.steps, args.warmup, flush)
-    e_ms = sum(etimes)
-    if dist:
-        t = torch.tensor([e_ms], device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e_ms = float(t.item())
-    e2e_value = world * ops * args.steps / (e_ms * 1e-3) / 1e12
+    e2e_value, e_ms = job_throughput(sum(etimes), ops, args.steps, dist, "cuda")
 
     line = None
     if rank == 0:
