@@ -146,9 +146,10 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
   CUtensorMap tq, tk, tv;
   const uint32_t ksub = m.dp >= 128 ? 128 : 64;
   const uint32_t dv = m.dp == 64 ? 64 : 128;
+  const uint32_t bn = 128;  // keys per KV tile of the fused kernel
   if (!make_map(&tq, qb.q8, m.dp, (uint64_t)m.B * m.Hq * m.Np, ksub, 128) ||
-      !make_map(&tk, qb.k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, 128) ||
-      !make_map(&tv, qb.v8t, m.Np, (uint64_t)m.B * m.Hkv * m.dp, 128, dv))
+      !make_map(&tk, qb.k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, bn) ||
+      !make_map(&tv, qb.v8t, m.Np, (uint64_t)m.B * m.Hkv * m.dp, bn, dv))
     return SAGE_ERR_CUDA;
   FwdParams p;
   p.qs = qb.qs, p.ks = qb.ks, p.vs = qb.vs, p.out = out;

@@ -40,22 +40,27 @@ template <int DQK, int DV>
 struct FwdCfg {
   static constexpr int KSUB = DQK >= 128 ? 128 : 64;  // bytes per row of one Q/K sub-tile (= swizzle span)
   static constexpr int NSUB = DQK / KSUB;
+  // Keys per KV tile.  (64-key tiles, which would let three d = 64 CTAs share an SM, measured
+  // no faster and change the online softmax's tile boundaries.)
+  static constexpr int BN = 128;
   static constexpr int Q_BYTES = 128 * DQK;
-  static constexpr int K_BYTES = 128 * DQK;
-  static constexpr int V_BYTES = DV * 128;
-  static constexpr int P_BYTES = 128 * 128;
+  static constexpr int K_BYTES = BN * DQK;
+  static constexpr int V_BYTES = DV * BN;
+  static constexpr int P_BYTES = 128 * BN;
   static constexpr int ST = DQK == 64 ? 5 : 2;                 // K/V ring depth
   static constexpr int CTAS_PER_SM = DQK <= 128 ? 2 : 1;       // two CTAs share an SM when they fit
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + Q_BYTES + ST * (K_BYTES + V_BYTES) + P_BYTES + BAR_BYTES;
-  // TMEM: S (int32 scores, 128 columns) and O (fp32, DV columns).  In fp16+fp32 mode the
+  // TMEM: S (int32 scores, BN columns) and O (fp32, DV columns).  In fp16+fp32 mode the
   // per-tile fp16 accumulator T reuses S's columns once the scores are in registers.
-  static constexpr uint32_t TMEM_COLS = 256;
-  static constexpr uint32_t S_COL = 0, O_COL = 128, T_COL = 0;
+  static constexpr uint32_t TMEM_COLS = BN + DV <= 128 ? 128 : 256;
+  static constexpr uint32_t S_COL = 0, O_COL = BN, T_COL = 0;
   static_assert(O_COL + DV <= TMEM_COLS, "TMEM plan");
+  static_assert(DV <= BN, "the fp16 tile accumulator must fit in S's columns");
   static_assert(ST <= 8, "barrier array size");
   static_assert(SMEM <= 227 * 1024, "shared memory plan");
   static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "co-resident CTAs must fit in shared memory");
+  static_assert(CTAS_PER_SM * TMEM_COLS <= 512, "co-resident CTAs must fit in tensor memory");
 };
 
 struct FwdBars {
@@ -128,7 +133,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
   const int hq = blockIdx.y / p.n_vhalves, vh = blockIdx.y - hq * p.n_vhalves;
   const int b = blockIdx.z;
   const int hkv = hq / p.G;
-  const int n_kv = CAUSAL ? qt + 1 : p.nblk;
+  // KV tiles of C::BN keys: up to the last key below N, and under the causal mask up to the
+  // last key of this query tile's diagonal block
+  const int n_kv_all = (p.N + C::BN - 1) / C::BN;
+  const int n_kv = CAUSAL ? min(n_kv_all, (qt + 1) * (128 / C::BN)) : n_kv_all;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -171,9 +179,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
         if (!mbar_wait(&bars->kv_empty[st], (u & 1) ^ 1, abort)) break;
         mbar_arrive_expect_tx(&bars->k_full[st], C::K_BYTES);
         for (int s = 0; s < C::NSUB; ++s)
-          tma_load_2d(sK + st * C::K_BYTES + s * 128 * C::KSUB, &tmK, &bars->k_full[st], s * C::KSUB, k_row + j * 128);
+          tma_load_2d(sK + st * C::K_BYTES + s * C::BN * C::KSUB, &tmK, &bars->k_full[st], s * C::KSUB,
+                      k_row + j * C::BN);
         mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
-        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], j * 128, v_row);
+        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], j * C::BN, v_row);
         issued = j + 1;
       }
       // make sure no copy is still landing in shared memory when the CTA exits
@@ -189,7 +198,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     // ahead of PV(j-1).  fp16+fp32 mode: T(j) lives in S's columns, so QK(j+1) waits
     // until the softmax has merged T(j) into O, and the order is QK(j), PV(j).
     if (lane == 0) {
-      constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*S8*/, 128, 128);
+      constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*S8*/, 128, C::BN);
       constexpr uint32_t idesc_pv = make_idesc(MODE == 0 ? 1 /*F32*/ : 0 /*F16*/, 0 /*E4M3*/, 128, DV);
       const uint32_t pv_dst = tmem + (MODE == 0 ? C::O_COL : C::T_COL);
       const uint32_t pa = smem_u32(sP);
@@ -200,9 +209,9 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
         tc_fence_after();
         const uint32_t va = smem_u32(sV + st * C::V_BYTES);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
+        for (int k = 0; k < C::BN / 32; ++k) {
           const uint32_t acc = MODE == 0 ? (uint32_t)(i > 0 || k > 0) : (uint32_t)(k > 0);
-          umma_f8(pv_dst, smem_desc_kmajor(pa + k * 32, 128), smem_desc_kmajor(va + k * 32, 128), idesc_pv, acc);
+          umma_f8(pv_dst, smem_desc_kmajor(pa + k * 32, C::BN), smem_desc_kmajor(va + k * 32, C::BN), idesc_pv, acc);
         }
         umma_commit(&bars->kv_empty[st]);
         umma_commit(&bars->pv_done);
@@ -222,7 +231,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
           for (int k = 0; k < DQK / 32; ++k) {
             const int sub = (k * 32) / C::KSUB, off = (k * 32) % C::KSUB;
             umma_i8(tmem + C::S_COL, smem_desc_kmajor(qa + sub * 128 * C::KSUB + off, C::KSUB),
-                    smem_desc_kmajor(ka + sub * 128 * C::KSUB + off, C::KSUB), idesc_qk, (uint32_t)(k > 0));
+                    smem_desc_kmajor(ka + sub * C::BN * C::KSUB + off, C::KSUB), idesc_qk, (uint32_t)(k > 0));
           }
           umma_commit(&bars->s_full);
           if (MODE == 0) {
@@ -240,18 +249,18 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
     {
-      // Two CTAs share an SM and the same MUFU units.  Started together they stay in step,
-      // both in their exponential loops at once (each at half the MUFU rate) and both in their
-      // other work at once (MUFU idle).  Every second CTA to arrive on an SM therefore starts
-      // its softmax about a third of a tile later; measured +2.5% to +6% on the fused kernel.
+      // Co-resident CTAs share an SM and its MUFU units.  Started together they stay in step,
+      // all in their exponential loops at once (each at a fraction of the MUFU rate) and all in
+      // their other work at once (MUFU idle).  The CTAs arriving on an SM are therefore started
+      // a fraction of a tile apart; measured +2.5% to +6% on the fused kernel.
       __shared__ unsigned int slot;
       if (threadIdx.x == 0) {
         unsigned int smid;
         asm volatile("mov.u32 %0, %%smid;" : "=r"(smid));
-        slot = atomicAdd(&g_sm_arrivals[smid & 255], 1u) & 1u;
+        slot = atomicAdd(&g_sm_arrivals[smid & 255], 1u) % C::CTAS_PER_SM;
       }
       asm volatile("bar.sync 1, 128;" ::: "memory");
-      if (slot) __nanosleep(300);
+      if (slot) __nanosleep(slot * (600u / C::CTAS_PER_SM));
     }
     const int row = warp * 32 + lane;            // query row inside the tile, TMEM lane
     const int grow = qt * 128 + row;             // query row in the sequence
@@ -260,17 +269,16 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     const uint32_t ocol = tmem + lane_base + C::O_COL;
     const float qsv = p.qs[((size_t)b * p.Hq + hq) * p.nblk + qt];
     const float* ksp = p.ks + ((size_t)b * p.Hkv + hkv) * p.nblk;
-    unsigned char* prow = sP + row * 128;
+    unsigned char* prow = sP + row * C::BN;
     float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates p * 448 * 2^-kTau
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
       if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
-      uint32_t s[128];
-      tmem_ld32(scol + 0, *reinterpret_cast<uint32_t(*)[32]>(&s[0]));
-      tmem_ld32(scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&s[32]));
-      tmem_ld32(scol + 64, *reinterpret_cast<uint32_t(*)[32]>(&s[64]));
-      tmem_ld32(scol + 96, *reinterpret_cast<uint32_t(*)[32]>(&s[96]));
+      constexpr int BN = C::BN;
+      uint32_t s[BN];
+#pragma unroll
+      for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(scol + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
       tmem_wait_ld();
       if (MODE == 0) {  // S is in registers: the next QK may overwrite it
         tc_fence_before();
@@ -279,22 +287,22 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
       }
 
       // dequantization factor in the log2 domain
-      const float f = __fmul_rn(__fmul_rn(qsv, ksp[i]), p.scale_log2);
-      const int key0 = i * 128;
-      const bool edge = (key0 + 128 > p.N) || (CAUSAL && i == qt);
-      int lim = 128;
+      const float f = __fmul_rn(__fmul_rn(qsv, ksp[i * BN / 128]), p.scale_log2);  // K scale of the 128-key block
+      const int key0 = i * BN;
+      const bool edge = (key0 + BN > p.N) || (CAUSAL && key0 + BN - 1 > qt * 128);
+      int lim = BN;  // this row sees the tile's columns c < lim
       if (edge) {
-        lim = min(p.N - key0, 128);
-        if (CAUSAL && i == qt) lim = min(lim, row + 1);
+        lim = min(p.N - key0, BN);
+        if (CAUSAL) lim = min(lim, grow - key0 + 1);
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
+        for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = (uint32_t)INT_MIN;
       }
       int mx8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) mx8[e] = (int)s[e];
 #pragma unroll
-      for (int c = 8; c < 128; ++c) mx8[c & 7] = max(mx8[c & 7], (int)s[c]);
+      for (int c = 8; c < BN; ++c) mx8[c & 7] = max(mx8[c & 7], (int)s[c]);
       const int mx = max(max(max(mx8[0], mx8[1]), max(mx8[2], mx8[3])), max(max(mx8[4], mx8[5]), max(mx8[6], mx8[7])));
       const float mt = (mx == INT_MIN) ? -INFINITY : __fmul_rn((float)mx, f);
       // The reference max m moves only when the running max exceeds it by more than kTau,
@@ -307,9 +315,9 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
       const bool rescale = MODE == 0 && i > 0 && __any_sync(0xffffffffu, alpha != 1.f);
       // p * 448 * 2^-kTau = 2^(s*f - m + log2 448 - kTau) -> E4M3, 4 keys per 32-bit word
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pw[32];
+      uint32_t pw[BN / 4];
 #pragma unroll
-      for (int c4 = 0; c4 < 32; ++c4) {
+      for (int c4 = 0; c4 < BN / 4; ++c4) {
         float pv[4];
 #pragma unroll
         for (int e = 0; e < 4; e += 2) {
@@ -342,10 +350,14 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
         if (!warp_wait(&bars->pv_done, (i - 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
       }
+      // 16-byte chunk ch of the row goes to chunk ch ^ (row's swizzle phase): the 128-byte
+      // (BN = 128) or 64-byte (BN = 64) swizzle the P.V descriptor expects
 #pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        *reinterpret_cast<uint4*>(prow + ((ch ^ (row & 7)) << 4)) =
+      for (int ch = 0; ch < BN / 16; ++ch) {
+        const int sw = BN == 128 ? (row & 7) : ((row >> 1) & 3);
+        *reinterpret_cast<uint4*>(prow + ((ch ^ sw) << 4)) =
             make_uint4(pw[ch * 4 + 0], pw[ch * 4 + 1], pw[ch * 4 + 2], pw[ch * 4 + 3]);
+      }
       fence_proxy_async_smem();
       if (rescale) {
         // O *= alpha (rows whose reference did not move have alpha = 1); 64 columns per batch,
@@ -452,10 +464,17 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
 // same TMA loads, shared-memory descriptors and kind::i8 UMMA as the fused kernel.
 // ------------------------------------------------------------------------------------------------
 template <int DQK>
+struct QkDumpCfg {
+  static constexpr int KSUB = DQK >= 128 ? 128 : 64;
+  static constexpr int NSUB = DQK / KSUB;
+  static constexpr int Q_BYTES = 128 * DQK, K_BYTES = 128 * DQK, BAR_BYTES = 256;
+};
+
+template <int DQK>
 __global__ void __launch_bounds__(128, 1)
     sage_qk_dump_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                         const QkDumpParams p) {
-  using C = FwdCfg<DQK, 64>;
+  using C = QkDumpCfg<DQK>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sQ = smem_raw + pad;
@@ -594,7 +613,7 @@ cudaError_t read_clear_device_error(int* value) {
 template <int DQK>
 static cudaError_t launch_qk_dump_t(const CUtensorMap& tq, const CUtensorMap& tk, const QkDumpParams& p,
                                     cudaStream_t st) {
-  using C = FwdCfg<DQK, 64>;
+  using C = QkDumpCfg<DQK>;
   const int smem = 1024 + C::Q_BYTES + C::K_BYTES + C::BAR_BYTES;
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = ensure_smem_limit(sage_qk_dump_kernel<DQK>, smem, attr_done);
