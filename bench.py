@@ -46,6 +46,25 @@ DEFAULT_WORKLOAD = W.IMAGE_DIT.name
 L2_FLUSH_BYTES = 256 << 20
 
 
+def _traffic(workload: str):
+    """DRAM bytes per launch of the fused kernel from the committed ncu capture, or None if the
+    kernel source changed since the capture (or the workload was not captured)."""
+    import hashlib
+    try:
+        kv = {}
+        for line in open(os.path.join(ROOT, "profiles", "sage_fwd_traffic.txt")):
+            line = line.strip()
+            if line and not line.startswith("#") and "=" in line:
+                k, v = line.split("=", 1)
+                kv[k.strip()] = v.strip()
+        src = open(os.path.join(ROOT, "quantized_attention_int8_b200", "csrc", "attn.cu"), "rb").read()
+        if hashlib.sha256(src).hexdigest() != kv.get("attn_cu_sha256"):
+            return None
+        return int(kv[workload]) if workload in kv else None
+    except (OSError, ValueError):
+        return None
+
+
 def _peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -283,7 +302,7 @@ def run_ours(args, w):
             "scaling": "weak", "vs_baseline": None, "dtype": "i8+f8e4m3", "data": "synthetic",
             "config": _config(w),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
-                         "frac": achieved / peak_tops, "traffic": None,
+                         "frac": achieved / peak_tops, "traffic": _traffic(w.name),
                          "kernel": "sage_fwd_kernel", "kernel_ms": k_ms,
                          "peak_source": f"2 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s "
                                         "(dense INT8/FP8 = 2x bf16 on B200)"},
