@@ -4,10 +4,13 @@ Test infrastructure only (see the package docstring).  This is a diagnostic:
 it predicts the error the method itself makes against exact attention, so a
 test can tell a kernel bug from the cost of 8-bit arithmetic.
 
-Steps, per (batch, query head, 128-row query block), over the 128-key tiles
-in increasing order (the blockwise online softmax the fused kernels use;
+Steps, per (batch, query head, 128-row query block), over the key tiles in
+increasing order (the blockwise online softmax the fused kernels use;
 SageAttention README, "Current Features"; qwbw.cn article, pitfalls, for the
-``pv_accum_dtype`` options):
+``pv_accum_dtype`` options).  A key tile is 128 keys for FP8 P.V and 64 keys
+for FP16 P.V (the tile width is where the online softmax may move its
+reference and, with fp16+fp32 accumulation, how many keys one fp16 partial
+sums; the pages fix neither):
 
 1. S = Q8 . K8^T exactly in integers (K8 holds codes of K - mean(K)).
 2. Dequantize in the log2 domain: s = S * f with
@@ -20,22 +23,29 @@ SageAttention README, "Current Features"; qwbw.cn article, pitfalls, for the
    tau = 0 this is the textbook online softmax; tau = 2 is how the CUDA
    kernel runs it (it rescales O only when the reference moves), and the
    result is the same up to rounding because O and l share the reference.
-4. P is stored as E4M3(p * 448 * 2^-tau), so codes stay within +-448.
-5. PV: mode 0 (fp32 accumulation) O = O * alpha + P8 . V8;
-   mode 1 (fp16+fp32, "two-level accumulation") the tile's P8 . V8 is first
+4. P is stored as E4M3(p * 448 * 2^-tau), so codes stay within +-448 (FP8
+   P.V modes 0, 1), or as fp16(p) (FP16 P.V modes 2, 3).
+5. PV: modes 0 and 2 (fp32 accumulation) O = O * alpha + P . V;
+   modes 1 and 3 (fp16+fp32, "two-level accumulation") the tile's P . V is first
    rounded to float16 (a fresh fp16 accumulator per tile), then
    O = O * alpha + T.
-6. out = O * vs / (448 * 2^-tau * l), rounded to the output dtype by the caller.
+6. out = O * vs / (P scale * l), P scale being 448 * 2^-tau (FP8) or 1 (FP16),
+   rounded to the output dtype by the caller.
 """
 from __future__ import annotations
 
 import numpy as np
 
 from . import fp8
-from .quant import BLOCK, P_SCALE, F32
+from .quant import BLOCK, P_SCALE, PV_FP16, F32
 
 LOG2E = 1.4426950408889634
 TAU = 2.0  # reference-max slack of the CUDA kernel's online softmax (log2 units)
+
+
+def kv_tile(pv_mode: int) -> int:
+    """Keys per online-softmax tile for a P.V mode: 128 (FP8 P.V) or 64 (FP16 P.V)."""
+    return 64 if pv_mode in PV_FP16 else BLOCK
 
 
 def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, tau: float = TAU):
@@ -52,26 +62,33 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
     hs = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
     qbs = list(range(nb)) if q_blocks is None else list(q_blocks)
     c = F32(F32(sm_scale) * F32(LOG2E))
-    pscale = F32(P_SCALE * 2.0 ** -tau)  # exact: 448 * 2^-tau
+    fp16_pv = mode in PV_FP16
+    T = kv_tile(mode)
+    pscale = F32(1.0) if fp16_pv else F32(P_SCALE * 2.0 ** -tau)  # exact: 448 * 2^-tau
     out = np.full((len(hs), len(qbs) * BLOCK, d), np.nan, F32)
     for n, (b, h) in enumerate(hs):
         hk = h // G
-        v8 = fp8.decode(qz["v8"][b, hk]).astype(np.float64)     # (Np, dp)
+        if fp16_pv:
+            v8 = qz["v8"][b, hk].astype(np.float64)             # fp16 codes (Np, dp)
+        else:
+            v8 = fp8.decode(qz["v8"][b, hk]).astype(np.float64)  # E4M3 codes (Np, dp)
         for r, qb in enumerate(qbs):
             rows = qb * BLOCK + np.arange(BLOCK)
             q8 = qz["q8"][b, h, qb * BLOCK:(qb + 1) * BLOCK].astype(np.int64)
             m = np.full(BLOCK, -np.inf, F32)
             l = np.zeros(BLOCK, F32)
             O = np.zeros((BLOCK, qz["dp"]), F32)
-            last = qb if causal else nb - 1
-            for j in range(last + 1):
-                keys = j * BLOCK + np.arange(BLOCK)
-                k8 = qz["k8"][b, hk, j * BLOCK:(j + 1) * BLOCK].astype(np.int64)
+            n_tiles = (qb + 1) * BLOCK // T if causal else nb * BLOCK // T
+            for j in range(n_tiles):
+                keys = j * T + np.arange(T)
+                if keys[0] >= N:
+                    break
+                k8 = qz["k8"][b, hk, j * T:(j + 1) * T].astype(np.int64)
                 S = q8 @ k8.T
                 valid = (keys[None, :] < N) & np.ones((BLOCK, 1), bool)
                 if causal:
                     valid &= keys[None, :] <= rows[:, None]
-                f = F32(F32(qz["qs"][b, h, qb]) * F32(qz["ks"][b, hk, j])) * c
+                f = F32(F32(qz["qs"][b, h, qb]) * F32(qz["ks"][b, hk, keys[0] // BLOCK])) * c
                 smax = np.where(valid, S, np.iinfo(np.int64).min).max(axis=1)
                 has = valid.any(axis=1)
                 tmax = np.where(has, smax.astype(F32) * f, F32(-np.inf)).astype(F32)
@@ -85,9 +102,12 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
                     alpha = np.where(np.isneginf(m), F32(0), np.exp2((m - m_new).astype(F32))).astype(F32)
                 alpha = np.where(upd, alpha, F32(1)).astype(F32)
                 l = (l * alpha + p.sum(axis=1, dtype=F32)).astype(F32)
-                p8 = fp8.decode(fp8.encode((p * pscale).astype(F32)))
-                pv = p8 @ v8[j * BLOCK:(j + 1) * BLOCK]                  # exact in float64
-                if mode == 1:
+                if fp16_pv:
+                    p8 = p.astype(np.float16).astype(np.float64)
+                else:
+                    p8 = fp8.decode(fp8.encode((p * pscale).astype(F32)))
+                pv = p8 @ v8[j * T:(j + 1) * T]                          # exact in float64
+                if mode in (1, 3):
                     pv = pv.astype(np.float16)
                 O = (O * alpha[:, None] + pv.astype(F32)).astype(F32)
                 m = m_new

@@ -32,6 +32,9 @@ choice a reader can check here, and the CUDA path implements the same one):
   VMAX is 448 for fp32 PV accumulation and 1 for the fp16+fp32 (two-level)
   accumulation, so that one 128-key tile's fp16 partial sum is bounded by
   128 * 448 * 1 = 57344 < 65504 and cannot overflow.
+* For the FP16 P.V variant (README "Available APIs": sageattn_qk_int8_pv_fp16_cuda)
+  V is kept in fp16 with the same per-channel scaling to [-1, 1]: inv = 1 / amax,
+  code = fp16_rne(v * inv), scale = amax.  (Q and K are quantized as above.)
 * All float arithmetic is IEEE float32 with round-to-nearest-even and no
   fused multiply-add; numpy float32 operations satisfy this.
 """
@@ -43,7 +46,10 @@ from . import fp8
 
 BLOCK = 128              # tokens per Q/K scale block and per KV tile
 P_SCALE = 448.0          # p in [0, 1] is stored as E4M3(p * 448)
-VMAX = {0: 448.0, 1: 1.0}  # V code range per PV accumulation mode
+# PV modes: 0 = FP8 P.V, fp32 accumulation; 1 = FP8 P.V, fp16+fp32; 2 = FP16 P.V, fp32;
+# 3 = FP16 P.V, fp16+fp32.  V code range per mode:
+VMAX = {0: 448.0, 1: 1.0, 2: 1.0, 3: 1.0}
+PV_FP16 = (2, 3)
 F32 = np.float32
 
 
@@ -141,14 +147,32 @@ def fp8_per_channel(v: np.ndarray, dp: int, vmax: float):
     return codes, scale
 
 
+def fp16_per_channel(v: np.ndarray, dp: int):
+    """Per-(b, h, channel) fp16 codes of v / amax (float32 (B,H,N,d)) over all tokens.
+
+    Returns codes float16 (B, H, N_pad, dp) and scales float32 (B, H, dp) = amax.
+    """
+    B, H, N, d = v.shape
+    nb = n_blocks(N)
+    amax = np.zeros((B, H, dp), F32)
+    amax[:, :, :d] = np.abs(v).max(axis=2)
+    with np.errstate(divide="ignore"):
+        inv = np.where(amax > 0, F32(1.0) / amax, F32(0.0)).astype(F32)
+    vp = np.zeros((B, H, nb * BLOCK, dp), F32)
+    vp[:, :, :N, :d] = v
+    codes = (vp * inv[:, :, None, :]).astype(F32).astype(np.float16)   # one RNE rounding to fp16
+    return codes, amax.copy()
+
+
 def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
     """The whole quantization step for one attention call.
 
     q: (B, Hq, N, d), k and v: (B, Hkv, N, d) in ``layout`` (fp16/bf16 torch
     tensors or arrays).  Returns a dict of numpy arrays:
       q8 int8 (B,Hq,Np,dp), qs f32 (B,Hq,nb), k8 int8 (B,Hkv,Np,dp),
-      ks f32 (B,Hkv,nb), km f32 (B,Hkv,dp), v8 uint8 (B,Hkv,Np,dp) E4M3 codes,
-      vs f32 (B,Hkv,dp), plus the sizes.
+      ks f32 (B,Hkv,nb), km f32 (B,Hkv,dp), v8 (B,Hkv,Np,dp) V codes (uint8 E4M3
+      for PV modes 0/1, float16 for the FP16 P.V modes 2/3), vs f32 (B,Hkv,dp),
+      plus the sizes.
     """
     qf, kf, vf = (to_hnd(t, layout) for t in (q, k, v))
     B, Hq, N, d = qf.shape
@@ -158,7 +182,10 @@ def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
     ksm = (kf - km[:, :, None, :]).astype(F32)        # one float32 subtraction
     q8, qs = int8_per_block(qf, dp)
     k8, ks = int8_per_block(ksm, dp)
-    v8, vs = fp8_per_channel(vf, dp, VMAX[pv_mode])
+    if pv_mode in PV_FP16:
+        v8, vs = fp16_per_channel(vf, dp)      # "v8" holds the fp16 codes in these modes
+    else:
+        v8, vs = fp8_per_channel(vf, dp, VMAX[pv_mode])
     kmp = np.zeros((B, Hkv, dp), F32)
     kmp[:, :, :d] = km
     return dict(q8=q8, qs=qs, k8=k8, ks=ks, km=kmp, v8=v8, vs=vs,

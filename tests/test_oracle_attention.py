@@ -138,3 +138,42 @@ def test_emulation_tracks_exact_attention():
         ref = attention.attention_f64(q, k, v, "HND", False, 0.125)
         cos = (em * ref).sum() / np.sqrt((em ** 2).sum() * (ref ** 2).sum())
         assert cos >= 0.999 and np.abs(em - ref).max() < 0.1
+
+
+def test_emulation_fp16_pv_modes():
+    # FP16 P.V: Q = 0 gives p = 1 exactly (fp16 1.0), V codes v/amax are exact in fp16 for
+    # these values, so every row is the (prefix) mean of V; causal row 0 is fp16(v0/amax)*amax.
+    rng = np.random.default_rng(4)
+    N = 300
+    q = np.zeros((1, 1, N, 8), np.float32)
+    k = rng.standard_normal((1, 1, N, 8)).astype(np.float32)
+    v = rng.choice([-1.0, -0.5, 0.5, 1.0, 0.25], size=(1, 1, N, 8)).astype(np.float32)
+    v[0, 0, 0] = 1.0
+    for mode in (2, 3):
+        qz = quant.quantize(q, k, v, "HND", mode)
+        assert qz["v8"].dtype == np.float16 and np.allclose(qz["vs"][0, 0, :8], 1.0)
+        em = emulate.emulate(qz, False, 0.35)[0, :N]
+        assert np.allclose(em, v[0, 0].mean(0)[None].repeat(N, 0), rtol=1e-6, atol=1e-7)
+        emc = emulate.emulate(qz, True, 0.35)[0, :N]
+        pref = np.cumsum(v[0, 0].astype(np.float64), 0) / np.arange(1, N + 1)[:, None]
+        assert np.allclose(emc, pref, rtol=1e-6, atol=1e-7)
+    # and the method stays within the spec cosine on the tiny workload
+    w = W.TINY
+    q, k, v = W.make_inputs(w)
+    for mode in (2, 3):
+        qz = quant.quantize(q, k, v, "HND", mode)
+        em = emulate.emulate(qz, False, 0.125).reshape(1, 2, 256, 64).astype(np.float64)
+        ref = attention.attention_f64(q, k, v, "HND", False, 0.125)
+        cos = (em * ref).sum() / np.sqrt((em ** 2).sum() * (ref ** 2).sum())
+        assert cos >= 0.9999 and np.abs(em - ref).max() < 0.02
+
+
+def test_fp16_v_codes_bound():
+    rng = np.random.default_rng(5)
+    v = (rng.standard_normal((1, 2, 200, 20)) * 3).astype(np.float32)
+    codes, scale = quant.fp16_per_channel(v, 64)
+    assert np.allclose(scale[:, :, :20], np.abs(v).max(axis=2)) and np.all(scale[:, :, 20:] == 0)
+    rec = codes[:, :, :200, :20].astype(np.float64) * scale[:, :, None, :20]
+    # fp16 keeps 11 significant bits: relative error <= 2^-11 (subnormals: 2^-25 absolute)
+    assert np.all(np.abs(rec - v) <= np.maximum(np.abs(v) * 2.0 ** -11, 2.0 ** -25 * scale[:, :, None, :20]) * (1 + 1e-6))
+    assert np.all(np.abs(codes[:, :, :200, :20]).max(axis=2) == 1.0)
