@@ -218,7 +218,8 @@ def run_reference(args, w):
 
 def _config(w):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "io_dtype": w.dtype,
-            "layout": w.layout, "causal": w.causal, "pv_accum": "fp32" if w.pv_mode == 0 else "fp16+fp32",
+            "layout": w.layout, "causal": w.causal, "pv_dtype": "fp16" if w.pv_mode & 2 else "fp8",
+            "pv_accum": "fp16+fp32" if w.pv_mode & 1 else "fp32",
             "values": w.dist, "l2": "flushed between steps (256 MiB write outside the events)"}
 
 
@@ -235,7 +236,8 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     if not qa.sage_device_supported():
         raise SystemExit("this device is not a B200 (compute capability 10.0)")
-    pv = "fp32" if w.pv_mode == 0 else "fp16+fp32"
+    pv = "fp16+fp32" if w.pv_mode & 1 else "fp32"
+    pvd = "fp16" if w.pv_mode & 2 else "fp8"
     scale = W.sm_scale_of(w)
     q, k, v = W.make_inputs(w)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
@@ -245,7 +247,7 @@ def run_ours(args, w):
     ops = w.ops()
 
     # ---- whole path (quantize + attention), device-resident inputs
-    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out)
+    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out, pv_dtype=pvd)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -255,16 +257,25 @@ def run_ours(args, w):
     value, total_ms = job_throughput(sum(times), ops, args.steps, dist, "cuda")
 
     # ---- the fused attention kernel alone (roofline)
-    z = qa.sage_quantize(qd, kd, vd, w.layout, pv)
+    z = qa.sage_quantize(qd, kd, vd, w.layout, pv, pvd)
     kern = lambda: qa.sage_attn_quantized(z, qd.dtype, w.layout, w.causal, scale, pv, out=out)
     ktimes = time_steps(kern, args.steps, args.warmup, flush)
     qa.sage_check_status()
     k_ms = statistics.mean(ktimes)
     peaks = _peaks()
-    peak_tops = 2.0 * peaks["bf16"]
+    if w.pv_mode & 2:
+        # half the operations (Q.K^T) at the INT8 rate 2P, half (P.V, fp16) at the fp16 rate P:
+        # the blended peak for all of them is 4P/3
+        peak_tops = 4.0 / 3.0 * peaks["bf16"]
+        peak_src = (f"4/3 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s (half the operations "
+                    "at the INT8 rate 2x bf16, half at the fp16 rate 1x bf16)")
+    else:
+        peak_tops = 2.0 * peaks["bf16"]
+        peak_src = f"2 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s (dense INT8/FP8 = 2x bf16 on B200)"
     achieved = ops / (k_ms * 1e-3) / 1e12
 
-    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element;
+    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element
+    # (V: 2 B written in the FP16 P.V modes);
     # the C entry point on preallocated outputs, so the Python allocations are not timed
     qargs = [qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), w.B, w.Hq, w.Hkv, w.N, w.d,
              qa.SAGE_BF16 if qd.dtype == torch.bfloat16 else qa.SAGE_FP16,
@@ -273,7 +284,7 @@ def run_ours(args, w):
              torch.cuda.current_stream().cuda_stream]
     qtimes = time_steps(lambda: qa.capi.sage_quantize(*qargs), max(3, args.steps // 2), 3, flush)
     q_ms = statistics.mean(qtimes)
-    q_bytes = 3 * (q.numel() + k.numel() + v.numel())
+    q_bytes = 3 * (q.numel() + k.numel()) + (4 if w.pv_mode & 2 else 3) * v.numel()
 
     # ---- end to end through the public API with pinned host buffers
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
@@ -283,7 +294,7 @@ def run_ours(args, w):
         a = qh.to("cuda", non_blocking=True)
         b = kh.to("cuda", non_blocking=True)
         c = vh.to("cuda", non_blocking=True)
-        o = qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv)
+        o = qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv, pv_dtype=pvd)
         outh.copy_(o, non_blocking=True)
 
     etimes = time_steps(e2e_step, args.steps, args.warmup, flush)
@@ -299,13 +310,12 @@ def run_ours(args, w):
         line = {
             "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "i8+f8e4m3", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8+f16" if w.pv_mode & 2 else "i8+f8e4m3", "data": "synthetic",
             "config": _config(w),
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
                          "frac": achieved / peak_tops, "traffic": _traffic(w.name),
                          "kernel": "sage_fwd_kernel", "kernel_ms": k_ms,
-                         "peak_source": f"2 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s "
-                                        "(dense INT8/FP8 = 2x bf16 on B200)"},
+                         "peak_source": peak_src},
             "quantize": {"ms": q_ms, "algorithmic_bytes": q_bytes, "GB_per_s": q_bytes / (q_ms * 1e-3) / 1e9,
                          "hbm_peak_GB_per_s": peaks["hbm"], "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm"]},
             "cpu_baseline": cpu,

@@ -56,15 +56,27 @@ typedef enum {
 typedef enum { SAGE_HND = 0, SAGE_NHD = 1 } sage_layout;
 typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype;
 
-/* P.V accumulation (SageAttention README, "Current Features": FP16 accumulator
- * for FP8 PV and two-level accumulation; qwbw.cn article, pitfalls:
- * pv_accum_dtype = "fp32" | "fp16+fp32").
- *   SAGE_PV_FP32      P8.V8 accumulates in fp32 across all key tiles.
- *   SAGE_PV_FP16_FP32 each 128-key tile's P8.V8 goes to a fresh fp16
- *                     accumulator, which is then added into an fp32 O.
- *                     V codes then span [-1, 1] (instead of [-448, 448]) so
- *                     one tile's fp16 partial (<= 128*448*1) cannot overflow. */
-typedef enum { SAGE_PV_FP32 = 0, SAGE_PV_FP16_FP32 = 1 } sage_pv_mode;
+/* P.V operands and accumulation (SageAttention README, "Current Features": FP8
+ * PV, FP16 accumulator for FP8 PV and two-level accumulation; "Available APIs":
+ * the INT8-QK / FP16-PV CUDA kernel; qwbw.cn article, pitfalls: pv_accum_dtype
+ * = "fp32" | "fp16+fp32").
+ *   SAGE_PV_FP32        FP8 (E4M3) P and V; P8.V8 accumulates in fp32 across
+ *                       all key tiles.
+ *   SAGE_PV_FP16_FP32   FP8 P and V; each 128-key tile's P8.V8 goes to a fresh
+ *                       fp16 accumulator, which is then added into an fp32 O.
+ *                       V codes then span [-1, 1] (instead of [-448, 448]) so
+ *                       one tile's fp16 partial (<= 128*448*1) cannot overflow.
+ *   SAGE_PV16_FP32      FP16 P and V (V codes = fp16(v / amax_channel), in
+ *                       [-1, 1]); fp32 accumulation.  Key tiles of 64.
+ *   SAGE_PV16_FP16_FP32 FP16 P and V; each 64-key tile's P.V in a fresh fp16
+ *                       accumulator (|partial| <= 64 * 4 * 1), added into fp32 O.
+ * Bit 0 of the value selects fp16+fp32 accumulation, bit 1 FP16 operands. */
+typedef enum {
+  SAGE_PV_FP32 = 0,
+  SAGE_PV_FP16_FP32 = 1,
+  SAGE_PV16_FP32 = 2,
+  SAGE_PV16_FP16_FP32 = 3
+} sage_pv_mode;
 
 /* Quantized attention, end to end: quantize/smooth pass, then the fused
  * attention kernel.  q: (B,Hq,N,d), k and v: (B,Hkv,N,d), out: (B,Hq,N,d), all
@@ -79,23 +91,28 @@ sage_status sage_attn(const void* q, const void* k, const void* v, void* out, in
                       sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
                       void* stream);
 
-/* Bytes of workspace sage_attn takes for these sizes (0 on invalid sizes). */
+/* Bytes of workspace sage_attn takes for these sizes, the largest over the P.V
+ * modes (0 on invalid sizes). */
 size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
 /* The quantize/smooth pass alone (K token mean, INT8 Q and K - mean(K) codes with
- * per-128-token-block scales, E4M3 V codes with per-channel scales).  Outputs,
- * with Np = 128 * ceil(N / 128) and dp the padded head dim, all device memory:
+ * per-128-token-block scales, E4M3 or fp16 V codes with per-channel scales).
+ * Outputs, with Np = 128 * ceil(N / 128) and dp the padded head dim, all device
+ * memory:
  *   q8  int8   [B][Hq][Np][dp]     qs  fp32 [B][Hq][Np/128]
  *   k8  int8   [B][Hkv][Np][dp]    ks  fp32 [B][Hkv][Np/128]    km fp32 [B][Hkv][dp]
- *   v8t uint8  [B][Hkv][dp][Np]    E4M3 codes, transposed (keys contiguous)
+ *   v8t        [B][Hkv][dp][Np]    V codes, transposed (keys contiguous): E4M3
+ *                                  bytes (SAGE_PV_FP32, SAGE_PV_FP16_FP32) or
+ *                                  fp16 values, 2 bytes each (SAGE_PV16_*)
  *   vs  fp32   [B][Hkv][dp]
  * Padded tokens and channels hold code 0 (and km 0, vs 0).  Codes and scales
  * follow: amax over the block's real tokens and channels, inv = 127 / amax,
  * code = clamp(rint_even(x * inv), -127, 127), scale = amax / 127 (0 when amax
  * is 0); K is smoothed as x = k - km, km summed in fp32 block by block (tokens
  * in order inside a block, then the block sums in order) and divided by N;
- * V: inv = VMAX / amax_channel, code = E4M3_rne_satfinite(v * inv),
- * vs = amax / VMAX with VMAX = 448 (SAGE_PV_FP32) or 1 (SAGE_PV_FP16_FP32).
+ * V: inv = VMAX / amax_channel, code = E4M3_rne_satfinite(v * inv) (FP8 modes)
+ * or fp16_rne(v * inv) (FP16 modes), vs = amax / VMAX with VMAX = 448
+ * (SAGE_PV_FP32) or 1 (the other modes).
  * Its own small scratch comes from the same per-device pool as sage_attn's. */
 sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
                           sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,

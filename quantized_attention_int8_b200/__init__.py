@@ -12,7 +12,9 @@ the library is missing, importing this package fails.
 
 mirrors the ``sageattn(q, k, v, tensor_layout, is_causal, sm_scale)`` call of
 the SageAttention README ("How to Use"); ``pv_accum_dtype`` selects "fp32" or
-"fp16+fp32" accumulation of the FP8 P.V product (qwbw.cn article, pitfalls).
+"fp16+fp32" accumulation of the P.V product (qwbw.cn article, pitfalls) and
+``pv_dtype`` its operands: "fp8" (E4M3, the INT8-QK / FP8-PV kernel) or "fp16"
+(the INT8-QK / FP16-PV kernel of the README's "Available APIs").
 """
 from __future__ import annotations
 
@@ -24,7 +26,7 @@ import torch
 __all__ = [
     "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
     "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
-    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES",
+    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
@@ -33,11 +35,20 @@ SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_ARCH, SAGE_ERR_CUD
     SAGE_ERR_TIMEOUT = range(7)
 SAGE_HND, SAGE_NHD = 0, 1
 SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
-SAGE_PV_FP32, SAGE_PV_FP16_FP32 = 0, 1
+SAGE_PV_FP32, SAGE_PV_FP16_FP32, SAGE_PV16_FP32, SAGE_PV16_FP16_FP32 = 0, 1, 2, 3
 
 _LAYOUTS = {"HND": SAGE_HND, "NHD": SAGE_NHD}
 _DTYPES = {torch.float16: SAGE_FP16, torch.bfloat16: SAGE_BF16, torch.float32: SAGE_FP32}
-_PV = {"fp32": SAGE_PV_FP32, "fp16+fp32": SAGE_PV_FP16_FP32}
+_PV = {("fp8", "fp32"): SAGE_PV_FP32, ("fp8", "fp16+fp32"): SAGE_PV_FP16_FP32,
+       ("fp16", "fp32"): SAGE_PV16_FP32, ("fp16", "fp16+fp32"): SAGE_PV16_FP16_FP32}
+
+
+def pv_mode(pv_dtype: str = "fp8", pv_accum_dtype: str = "fp32") -> int:
+    """The sage_pv_mode value for P.V operands ``pv_dtype`` and accumulation ``pv_accum_dtype``."""
+    try:
+        return _PV[(pv_dtype, pv_accum_dtype)]
+    except KeyError:
+        raise ValueError(f"unsupported pv_dtype / pv_accum_dtype {pv_dtype!r} / {pv_accum_dtype!r}") from None
 
 
 def _load() -> ctypes.CDLL:
@@ -123,7 +134,8 @@ def _check_inputs(q, k, v, layout):
     return B, Hq, Hkv, N, d
 
 
-def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None):
+def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None,
+              pv_dtype="fp8"):
     """Quantized attention of fp16/bf16 q (B,Hq,N,d), k/v (B,Hkv,N,d) (HND; NHD stores (B,N,H,d))."""
     B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
     if q.dtype not in _DTYPES:
@@ -132,7 +144,8 @@ def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_a
         out = torch.empty_like(q)
     st = capi.sage_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
                         _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)),
-                        float(sm_scale) if sm_scale is not None else 0.0, _PV[pv_accum_dtype], _stream())
+                        float(sm_scale) if sm_scale is not None else 0.0, pv_mode(pv_dtype, pv_accum_dtype),
+                        _stream())
     _check(st, "sage_attn")
     return out
 
@@ -140,22 +153,22 @@ def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_a
 SAGE_NOALLOC_MAX_BYTES = 64 << 20
 
 
-def sage_attn_noalloc(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None):
+def sage_attn_noalloc(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None,
+                      pv_dtype="fp8"):
     """sage_attn with no device allocation inside the library (for callers that cannot
     allocate at call time); the caller supplies ``out`` or torch allocates it here.  The
-    library's static workspace holds problems up to SAGE_NOALLOC_MAX_BYTES of workspace;
-    calls that may overlap on the GPU must be ordered by the caller."""
+    library's static workspace holds problems up to SAGE_NOALLOC_MAX_BYTES of workspace
+    (larger ones raise SageError with SAGE_ERR_INVALID_ARG); calls that may overlap on the
+    GPU must be ordered by the caller."""
     B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
     if q.dtype not in _DTYPES:
         raise ValueError(f"unsupported dtype {q.dtype}")
-    need = sage_workspace_bytes(B, Hq, Hkv, N, d)
-    if need > SAGE_NOALLOC_MAX_BYTES:
-        raise ValueError(f"workspace of {need} bytes exceeds the static {SAGE_NOALLOC_MAX_BYTES} bytes; use sage_attn")
     if out is None:
         out = torch.empty_like(q)
     st = capi.sage_attn_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
                                 _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)),
-                                float(sm_scale) if sm_scale is not None else 0.0, _PV[pv_accum_dtype], _stream())
+                                float(sm_scale) if sm_scale is not None else 0.0, pv_mode(pv_dtype, pv_accum_dtype),
+                        _stream())
     _check(st, "sage_attn_noalloc")
     return out
 
@@ -164,13 +177,15 @@ def sage_workspace_bytes(B, Hq, Hkv, N, d) -> int:
     return int(capi.sage_workspace_bytes(B, Hq, Hkv, N, d))
 
 
-def sage_quantize(q, k, v, tensor_layout="HND", pv_accum_dtype="fp32") -> dict:
+def sage_quantize(q, k, v, tensor_layout="HND", pv_accum_dtype="fp32", pv_dtype="fp8") -> dict:
     """The quantize/smooth pass alone; returns the codes and scales as CUDA tensors.
 
     Layouts (Np = 128*ceil(N/128), dp = padded head dim): q8 int8 (B,Hq,Np,dp),
     qs f32 (B,Hq,Np/128), k8 int8 (B,Hkv,Np,dp), ks f32 (B,Hkv,Np/128),
-    km f32 (B,Hkv,dp), v8t uint8 E4M3 (B,Hkv,dp,Np), vs f32 (B,Hkv,dp).
+    km f32 (B,Hkv,dp), v8t (B,Hkv,dp,Np) uint8 E4M3 codes (pv_dtype "fp8") or
+    float16 codes (pv_dtype "fp16"), vs f32 (B,Hkv,dp).
     """
+    mode = pv_mode(pv_dtype, pv_accum_dtype)
     B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
     dp, nb = padded_dim(d), (N + 127) // 128
     Np = nb * 128
@@ -181,21 +196,22 @@ def sage_quantize(q, k, v, tensor_layout="HND", pv_accum_dtype="fp32") -> dict:
         k8=torch.empty((B, Hkv, Np, dp), dtype=torch.int8, device=dev),
         ks=torch.empty((B, Hkv, nb), dtype=torch.float32, device=dev),
         km=torch.empty((B, Hkv, dp), dtype=torch.float32, device=dev),
-        v8t=torch.empty((B, Hkv, dp, Np), dtype=torch.uint8, device=dev),
+        v8t=torch.empty((B, Hkv, dp, Np), dtype=torch.float16 if pv_dtype == "fp16" else torch.uint8, device=dev),
         vs=torch.empty((B, Hkv, dp), dtype=torch.float32, device=dev),
     )
     st = capi.sage_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d, _DTYPES[q.dtype],
-                            _LAYOUTS[tensor_layout], _PV[pv_accum_dtype], *(z[n].data_ptr() for n in
+                            _LAYOUTS[tensor_layout], mode, *(z[n].data_ptr() for n in
                                                                           ("q8", "qs", "k8", "ks", "km", "v8t", "vs")),
                             _stream())
     _check(st, "sage_quantize")
-    z.update(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d)
+    z.update(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, pv_dtype=pv_dtype)
     return z
 
 
 def sage_attn_quantized(z: dict, out_dtype=torch.float16, tensor_layout="HND", is_causal=False, sm_scale=None,
                         pv_accum_dtype="fp32", out=None):
-    """The fused attention kernel alone on quantized buffers (the dict sage_quantize returns)."""
+    """The fused attention kernel alone on quantized buffers (the dict sage_quantize returns;
+    its ``pv_dtype`` entry selects the P.V operands)."""
     B, Hq, Hkv, N, d = (z[n] for n in ("B", "Hq", "Hkv", "N", "d"))
     if out is None:
         shape = (B, Hq, N, d) if tensor_layout == "HND" else (B, N, Hq, d)
@@ -203,7 +219,7 @@ def sage_attn_quantized(z: dict, out_dtype=torch.float16, tensor_layout="HND", i
     st = capi.sage_attn_quantized(*(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "v8t", "vs")),
                                   out.data_ptr(), B, Hq, Hkv, N, d, _DTYPES[out.dtype], _LAYOUTS[tensor_layout],
                                   int(bool(is_causal)), float(sm_scale) if sm_scale is not None else 0.0,
-                                  _PV[pv_accum_dtype], _stream())
+                                  pv_mode(z.get("pv_dtype", "fp8"), pv_accum_dtype), _stream())
     _check(st, "sage_attn_quantized")
     return out
 

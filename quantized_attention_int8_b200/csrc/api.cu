@@ -100,6 +100,12 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t rows, u
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15) == 0; }
 
+bool pv_mode_valid(int pv_mode) {
+  return pv_mode == SAGE_PV_FP32 || pv_mode == SAGE_PV_FP16_FP32 || pv_mode == SAGE_PV16_FP32 ||
+         pv_mode == SAGE_PV16_FP16_FP32;
+}
+bool pv_mode_fp16_operands(int pv_mode) { return pv_mode == SAGE_PV16_FP32 || pv_mode == SAGE_PV16_FP16_FP32; }
+
 // Workspace memory: a stream-ordered pool per device, owned by the library, that keeps the
 // memory it has handed out (release threshold = unlimited), so that repeated calls reuse
 // it instead of mapping fresh device memory each time.
@@ -146,10 +152,13 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
   CUtensorMap tq, tk, tv;
   const uint32_t ksub = m.dp >= 128 ? 128 : 64;
   const uint32_t dv = m.dp == 64 ? 64 : 128;
-  const uint32_t bn = 128;  // keys per KV tile of the fused kernel
+  const bool pv16 = pv_mode_fp16_operands(pv_mode);
+  const uint32_t bn = pv16 ? 64 : 128;  // keys per KV tile of the fused kernel
+  const uint64_t vrow = (uint64_t)m.Np * (pv16 ? 2 : 1);  // bytes per V^T row (one channel)
+  // V^T tile box: 128 bytes of keys (128 E4M3 or 64 fp16 codes) x dv channels
   if (!make_map(&tq, qb.q8, m.dp, (uint64_t)m.B * m.Hq * m.Np, ksub, 128) ||
       !make_map(&tk, qb.k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, bn) ||
-      !make_map(&tv, qb.v8t, m.Np, (uint64_t)m.B * m.Hkv * m.dp, bn, dv))
+      !make_map(&tv, qb.v8t, vrow, (uint64_t)m.B * m.Hkv * m.dp, 128, dv))
     return SAGE_ERR_CUDA;
   FwdParams p;
   p.qs = qb.qs, p.ks = qb.ks, p.vs = qb.vs, p.out = out;
@@ -165,7 +174,7 @@ struct WsLayout {
   size_t q8, qs, k8, ks, km, v8t, vs, ksum, vmax, vinv, total;
 };
 
-WsLayout ws_layout(const Dims& m) {
+WsLayout ws_layout(const Dims& m, int pv_mode) {
   WsLayout w;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -178,7 +187,7 @@ WsLayout ws_layout(const Dims& m) {
   w.k8 = take((size_t)m.B * m.Hkv * m.Np * m.dp);
   w.ks = take((size_t)m.B * m.Hkv * m.nblk * 4);
   w.km = take((size_t)m.B * m.Hkv * m.dp * 4);
-  w.v8t = take((size_t)m.B * m.Hkv * m.dp * m.Np);
+  w.v8t = take((size_t)m.B * m.Hkv * m.dp * m.Np * (pv_mode_fp16_operands(pv_mode) ? 2 : 1));
   w.vs = take((size_t)m.B * m.Hkv * m.dp * 4);
   w.ksum = take((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
   w.vmax = take((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
@@ -197,7 +206,8 @@ QuantParams quant_params(const Dims& m, const void* q, const void* k, const void
   p.vec_q = (m.d % 8 == 0) && aligned16(q);
   p.vec_k = (m.d % 8 == 0) && aligned16(k);
   p.vec_v = (m.d % 8 == 0) && aligned16(v);
-  p.vmax_code = pv_mode == SAGE_PV_FP16_FP32 ? 1.0f : 448.0f;
+  p.vmax_code = pv_mode == SAGE_PV_FP32 ? 448.0f : 1.0f;
+  p.v_fp16 = pv_mode_fp16_operands(pv_mode) ? 1 : 0;
   return p;
 }
 
@@ -207,7 +217,7 @@ sage_status check_common(const void* q, const void* k, const void* v, int B, int
   sage_status s = check_dtype(dtype);
   if (s != SAGE_OK) return s;
   if (layout != SAGE_HND && layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
-  if (pv_mode != SAGE_PV_FP32 && pv_mode != SAGE_PV_FP16_FP32) return SAGE_ERR_INVALID_ARG;
+  if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
   return check_dims(B, Hq, Hkv, N, d, m);
 }
 
@@ -218,7 +228,7 @@ extern "C" {
 size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   Dims m;
   if (check_dims(B, Hq, Hkv, N, d, &m) != SAGE_OK) return 0;
-  return ws_layout(m).total;
+  return ws_layout(m, SAGE_PV16_FP32).total;  // the largest over the P.V modes
 }
 
 sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
@@ -233,7 +243,7 @@ sage_status sage_attn(const void* q, const void* k, const void* v, void* out, in
     return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const WsLayout w = ws_layout(m);
+  const WsLayout w = ws_layout(m, pv_mode);
   unsigned char* ws = nullptr;
   cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), w.total, st);
   if (e != cudaSuccess) return from_cuda(e);
@@ -286,7 +296,7 @@ sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t*
   sage_status s = check_dtype(out_dtype);
   if (s != SAGE_OK) return s;
   if (out_layout != SAGE_HND && out_layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
-  if (pv_mode != SAGE_PV_FP32 && pv_mode != SAGE_PV_FP16_FP32) return SAGE_ERR_INVALID_ARG;
+  if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
   Dims m;
   if ((s = check_dims(B, Hq, Hkv, N, d, &m)) != SAGE_OK) return s;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
@@ -380,7 +390,7 @@ extern "C" sage_status sage_attn_noalloc(const void* q, const void* k, const voi
   const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
   if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes))
     return SAGE_ERR_INVALID_ARG;
-  const WsLayout w = ws_layout(m);
+  const WsLayout w = ws_layout(m, pv_mode);
   if (w.total > (size_t)SAGE_NOALLOC_MAX_BYTES) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   int dev = 0;

@@ -1,4 +1,4 @@
-// Fused INT8-QK / FP8-PV attention for sm_100a (tcgen05 + TMA + TMEM).
+// Fused INT8-QK / FP8-PV (or FP16-PV) attention for sm_100a (tcgen05 + TMA + TMEM).
 //
 // One CTA computes one 128-row query tile of one (batch, query head) and, when
 // the padded head dim is 256, one 128-column half of the output.  Six warps:
@@ -9,19 +9,24 @@
 //              ST-deep ring of shared-memory stages;
 //   warp 5     TMEM allocator and UMMA issuer (one elected thread).
 //
-// Per 128-key tile j (the blockwise online softmax of the method):
+// Per key tile j of BN keys (the blockwise online softmax of the method):
 //   S_j  = Q8 . K8_j^T                    tcgen05.mma kind::i8 -> int32 in TMEM
 //   s    = S_j * (qs * ks_j * sm_scale * log2 e), causal / length mask
 //   m'   = max(m, rowmax s), p = 2^(s - m'), alpha = 2^(m - m'), l = l alpha + sum p
-//   P8   = E4M3(p * 448)                  written to shared memory (128B swizzle)
-//   mode 0 (fp32 accumulation):  O = O * alpha (in TMEM) ; O += P8 . V8_j   (kind::f8f6f4, f32)
-//   mode 1 (fp16+fp32):          T = P8 . V8_j (fresh f16 accumulator) ; O = O * alpha + T
-//   out  = O * v_scale / (448 * l)
+//   P    = E4M3(p * 448) (FP8 P.V, BN = 128) or fp16(p) (FP16 P.V, BN = 64), written to
+//          shared memory as 128-byte rows with the 128B swizzle
+//   mode 0 (fp32 accumulation):  O = O * alpha (in TMEM) ; O += P . V_j    (f32 accumulator)
+//   mode 1 (fp16+fp32):          T = P . V_j (fresh f16 accumulator) ; O = O * alpha + T
+//   out  = O * v_scale / (P scale * l)
+// FP8 P.V runs as tcgen05.mma kind::f8f6f4 on E4M3 codes, FP16 P.V as kind::f16 on fp16
+// codes (V scaled per channel to [-1, 1]).  The FP16 variant uses 64-key tiles so that its
+// twice-as-large P and V tiles still let two CTAs share an SM.
 //
 // Method: SageAttention README ("Current Features": INT8 QK^T with smoothing,
-// FP8 PV, FP16 accumulator for FP8 PV, two-level accumulation) and the qwbw.cn
-// article (pitfalls: pv_accum_dtype fp32 / fp16+fp32).  The kernel design
-// (tcgen05, TMEM accumulators, TMA ring, warp roles) is this library's own.
+// FP8 PV, FP16 accumulator for FP8 PV, two-level accumulation; "Available APIs":
+// the INT8-QK / FP16-PV kernel) and the qwbw.cn article (pitfalls: pv_accum_dtype
+// fp32 / fp16+fp32).  The kernel design (tcgen05, TMEM accumulators, TMA ring,
+// warp roles) is this library's own.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -36,27 +41,30 @@ namespace sage {
 // CTAs that arrived on each SM so far (only the parity is used; see the stagger below).
 __device__ unsigned int g_sm_arrivals[256];
 
-template <int DQK, int DV>
+template <int DQK, int DV, bool PV16>
 struct FwdCfg {
   static constexpr int KSUB = DQK >= 128 ? 128 : 64;  // bytes per row of one Q/K sub-tile (= swizzle span)
   static constexpr int NSUB = DQK / KSUB;
-  // Keys per KV tile.  (64-key tiles, which would let three d = 64 CTAs share an SM, measured
-  // no faster and change the online softmax's tile boundaries.)
-  static constexpr int BN = 128;
+  static constexpr int PB = PV16 ? 2 : 1;  // bytes per P and V element
+  // Keys per KV tile.  FP8 P.V: 128 (64-key tiles, which would let three d = 64 CTAs share an
+  // SM, measured no faster).  FP16 P.V: 64, so a P row and a V^T row are 128 bytes in both.
+  static constexpr int BN = PV16 ? 64 : 128;
+  static constexpr int ROWB = BN * PB;  // bytes of one P row / V^T row of a tile = the 128B swizzle span
   static constexpr int Q_BYTES = 128 * DQK;
   static constexpr int K_BYTES = BN * DQK;
-  static constexpr int V_BYTES = DV * BN;
-  static constexpr int P_BYTES = 128 * BN;
-  static constexpr int ST = DQK == 64 ? 5 : 2;                 // K/V ring depth
+  static constexpr int V_BYTES = DV * ROWB;
+  static constexpr int P_BYTES = 128 * ROWB;
+  static constexpr int ST = PV16 ? (DQK == 64 ? 4 : DQK == 128 ? 3 : 2) : (DQK == 64 ? 5 : 2);  // ring depth
   static constexpr int CTAS_PER_SM = DQK <= 128 ? 2 : 1;       // two CTAs share an SM when they fit
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + Q_BYTES + ST * (K_BYTES + V_BYTES) + P_BYTES + BAR_BYTES;
   // TMEM: S (int32 scores, BN columns) and O (fp32, DV columns).  In fp16+fp32 mode the
-  // per-tile fp16 accumulator T reuses S's columns once the scores are in registers.
-  static constexpr uint32_t TMEM_COLS = BN + DV <= 128 ? 128 : 256;
-  static constexpr uint32_t S_COL = 0, O_COL = BN, T_COL = 0;
+  // per-tile fp16 accumulator T (DV columns) reuses S's columns (and those up to O) once the
+  // scores are in registers.
+  static constexpr uint32_t S_COL = 0, T_COL = 0, O_COL = BN > DV ? BN : DV;
+  static constexpr uint32_t TMEM_COLS = O_COL + DV <= 128 ? 128 : 256;
+  static_assert(ROWB == 128, "P and V^T rows are one 128-byte swizzle span");
   static_assert(O_COL + DV <= TMEM_COLS, "TMEM plan");
-  static_assert(DV <= BN, "the fp16 tile accumulator must fit in S's columns");
   static_assert(ST <= 8, "barrier array size");
   static_assert(SMEM <= 227 * 1024, "shared memory plan");
   static_assert(CTAS_PER_SM * (SMEM + 1024) <= 228 * 1024, "co-resident CTAs must fit in shared memory");
@@ -112,11 +120,11 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 constexpr float kLog2_448 = 8.807354922057604f;  // p * 448 = 2^(log2 p + log2 448)
 constexpr float kTau = 2.0f;                       // reference-max slack of the online softmax (log2 units)
 
-template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
-__global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
+template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16>
+__global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     sage_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<DQK, DV>;
+  using C = FwdCfg<DQK, DV, PV16>;
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
   unsigned char* sbase = smem_raw + pad;
@@ -182,7 +190,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
           tma_load_2d(sK + st * C::K_BYTES + s * C::BN * C::KSUB, &tmK, &bars->k_full[st], s * C::KSUB,
                       k_row + j * C::BN);
         mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
-        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], j * C::BN, v_row);
+        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], j * C::ROWB, v_row);  // x in bytes
         issued = j + 1;
       }
       // make sure no copy is still landing in shared memory when the CTA exits
@@ -199,7 +207,8 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     // until the softmax has merged T(j) into O, and the order is QK(j), PV(j).
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*S8*/, 128, C::BN);
-      constexpr uint32_t idesc_pv = make_idesc(MODE == 0 ? 1 /*F32*/ : 0 /*F16*/, 0 /*E4M3*/, 128, DV);
+      // A = P, B = V^T, both E4M3 (kind::f8f6f4) or both F16 (kind::f16): format code 0 either way
+      constexpr uint32_t idesc_pv = make_idesc(MODE == 0 ? 1 /*F32*/ : 0 /*F16*/, 0, 128, DV);
       const uint32_t pv_dst = tmem + (MODE == 0 ? C::O_COL : C::T_COL);
       const uint32_t pa = smem_u32(sP);
       auto issue_pv = [&](int i) -> bool {
@@ -208,10 +217,15 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
         if (!mbar_wait(&bars->p_full, i & 1, abort)) return false;
         tc_fence_after();
         const uint32_t va = smem_u32(sV + st * C::V_BYTES);
+        // one MMA per 32 bytes of the 128-byte rows: K = 32 E4M3 or 16 fp16 keys
 #pragma unroll
-        for (int k = 0; k < C::BN / 32; ++k) {
+        for (int k = 0; k < C::ROWB / 32; ++k) {
           const uint32_t acc = MODE == 0 ? (uint32_t)(i > 0 || k > 0) : (uint32_t)(k > 0);
-          umma_f8(pv_dst, smem_desc_kmajor(pa + k * 32, C::BN), smem_desc_kmajor(va + k * 32, C::BN), idesc_pv, acc);
+          const uint64_t ad = smem_desc_kmajor(pa + k * 32, C::ROWB), bd = smem_desc_kmajor(va + k * 32, C::ROWB);
+          if (PV16)
+            umma_f16(pv_dst, ad, bd, idesc_pv, acc);
+          else
+            umma_f8(pv_dst, ad, bd, idesc_pv, acc);
         }
         umma_commit(&bars->kv_empty[st]);
         umma_commit(&bars->pv_done);
@@ -269,8 +283,8 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
     const uint32_t ocol = tmem + lane_base + C::O_COL;
     const float qsv = p.qs[((size_t)b * p.Hq + hq) * p.nblk + qt];
     const float* ksp = p.ks + ((size_t)b * p.Hkv + hkv) * p.nblk;
-    unsigned char* prow = sP + row * C::BN;
-    float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates p * 448 * 2^-kTau
+    unsigned char* prow = sP + row * C::ROWB;
+    float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates the stored P values' scale
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
       if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
@@ -306,16 +320,18 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
       const int mx = max(max(max(mx8[0], mx8[1]), max(mx8[2], mx8[3])), max(max(mx8[4], mx8[5]), max(mx8[6], mx8[7])));
       const float mt = (mx == INT_MIN) ? -INFINITY : __fmul_rn((float)mx, f);
       // The reference max m moves only when the running max exceeds it by more than kTau,
-      // so O is rescaled rarely; p = 2^(s - m) <= 2^kTau is stored as E4M3(p * 448 * 2^-kTau).
+      // so O is rescaled rarely; p = 2^(s - m) <= 2^kTau is stored as E4M3(p * 448 * 2^-kTau)
+      // (FP8 P.V) or as fp16(p) (FP16 P.V).
       const float mc = fmaxf(m, mt);
       const bool upd = mc > __fadd_rn(m, kTau);
       const float m_new = upd ? mc : m;
       const float alpha = upd ? ((m == -INFINITY) ? 0.f : ex2_approx(m - m_new)) : 1.f;
-      const float bias = (m_new == -INFINITY) ? 0.f : (kLog2_448 - kTau) - m_new;
+      const float bias = (m_new == -INFINITY) ? 0.f : (PV16 ? 0.f : kLog2_448 - kTau) - m_new;
       const bool rescale = MODE == 0 && i > 0 && __any_sync(0xffffffffu, alpha != 1.f);
-      // p * 448 * 2^-kTau = 2^(s*f - m + log2 448 - kTau) -> E4M3, 4 keys per 32-bit word
+      // p * 448 * 2^-kTau = 2^(s*f - m + log2 448 - kTau) -> E4M3, 4 keys per 32-bit word;
+      // FP16 P.V: p = 2^(s*f - m) -> fp16, 2 keys per word
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      uint32_t pw[BN / 4];
+      uint32_t pw[C::ROWB / 4];
 #pragma unroll
       for (int c4 = 0; c4 < BN / 4; ++c4) {
         float pv[4];
@@ -341,7 +357,12 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
           rs[e] += pv[e];
           rs[e + 1] += pv[e + 1];
         }
-        pw[c4] = e4m3x2(pv[0], pv[1]) | (e4m3x2(pv[2], pv[3]) << 16);
+        if (PV16) {
+          pw[2 * c4] = pack2<__half>(pv[0], pv[1]);
+          pw[2 * c4 + 1] = pack2<__half>(pv[2], pv[3]);
+        } else {
+          pw[c4] = e4m3x2(pv[0], pv[1]) | (e4m3x2(pv[2], pv[3]) << 16);
+        }
       }
       l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       m = m_new;
@@ -350,11 +371,11 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV>::CTAS_PER_SM)
         if (!warp_wait(&bars->pv_done, (i - 1) & 1, abort)) { ok = false; break; }
         tc_fence_after();
       }
-      // 16-byte chunk ch of the row goes to chunk ch ^ (row's swizzle phase): the 128-byte
-      // (BN = 128) or 64-byte (BN = 64) swizzle the P.V descriptor expects
+      // 16-byte chunk ch of the 128-byte row goes to chunk ch ^ (row & 7): the 128B swizzle the
+      // P.V descriptor expects
 #pragma unroll
-      for (int ch = 0; ch < BN / 16; ++ch) {
-        const int sw = BN == 128 ? (row & 7) : ((row >> 1) & 3);
+      for (int ch = 0; ch < C::ROWB / 16; ++ch) {
+        const int sw = row & 7;
         *reinterpret_cast<uint4*>(prow + ((ch ^ sw) << 4)) =
             make_uint4(pw[ch * 4 + 0], pw[ch * 4 + 1], pw[ch * 4 + 2], pw[ch * 4 + 3]);
       }
@@ -563,11 +584,11 @@ static cudaError_t ensure_smem_limit(K kern, int bytes, std::atomic<unsigned lon
   return e;
 }
 
-template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT>
+template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, cudaStream_t st) {
-  using C = FwdCfg<DQK, DV>;
-  auto kern = sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT>;
+  using C = FwdCfg<DQK, DV, PV16>;
+  auto kern = sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16>;
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done);
   if (e != cudaSuccess) return e;
@@ -576,14 +597,22 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   return cudaGetLastError();
 }
 
+template <int DQK, int DV, typename OutT, bool PV16>
+static cudaError_t launch_fwd_m(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const FwdParams& p, int causal, int accum, cudaStream_t st) {
+  if (accum == 0)
+    return causal ? launch_fwd_t<DQK, DV, 0, true, OutT, PV16>(tq, tk, tv, p, st)
+                  : launch_fwd_t<DQK, DV, 0, false, OutT, PV16>(tq, tk, tv, p, st);
+  return causal ? launch_fwd_t<DQK, DV, 1, true, OutT, PV16>(tq, tk, tv, p, st)
+                : launch_fwd_t<DQK, DV, 1, false, OutT, PV16>(tq, tk, tv, p, st);
+}
+
+// pv_mode: bit 0 = fp16+fp32 accumulation, bit 1 = FP16 P.V operands (sage_pv_mode values)
 template <int DQK, int DV, typename OutT>
 static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                                const FwdParams& p, int causal, int mode, cudaStream_t st) {
-  if (mode == 0)
-    return causal ? launch_fwd_t<DQK, DV, 0, true, OutT>(tq, tk, tv, p, st)
-                  : launch_fwd_t<DQK, DV, 0, false, OutT>(tq, tk, tv, p, st);
-  return causal ? launch_fwd_t<DQK, DV, 1, true, OutT>(tq, tk, tv, p, st)
-                : launch_fwd_t<DQK, DV, 1, false, OutT>(tq, tk, tv, p, st);
+                                const FwdParams& p, int causal, int pv_mode, cudaStream_t st) {
+  return (pv_mode & 2) ? launch_fwd_m<DQK, DV, OutT, true>(tq, tk, tv, p, causal, pv_mode & 1, st)
+                       : launch_fwd_m<DQK, DV, OutT, false>(tq, tk, tv, p, causal, pv_mode & 1, st);
 }
 
 template <typename OutT>

@@ -8,7 +8,8 @@
 //             v_scale = amax / VMAX, v_inv = VMAX / amax.
 //   pass 2  per (batch, kv-head, block):
 //             K - k_mean -> INT8 codes + per-block scale;
-//             V -> E4M3 codes, written transposed (keys contiguous) for the P.V MMA.
+//             V -> E4M3 codes (FP8 P.V) or fp16 codes of v / amax (FP16 P.V), written
+//             transposed (keys contiguous) for the P.V MMA.
 //
 // Method: INT8 quantization with smoothing for Q K^T and FP8 quantization for
 // P V (SageAttention README, "Current Features").  The block size, the
@@ -293,13 +294,31 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
     store_int8_tile(p.k8 + (bh * p.Np + n0) * dp, dp, tc, inv, rows, x);
     if (threadIdx.x == 0) p.ks[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
-  } else {  // ---- V: E4M3 codes, transposed to [channel][token]
+  } else {  // ---- V: E4M3 or fp16 codes, transposed to [channel][token]
     const int h = y - p.Hkv;
     const size_t bh = (size_t)b * p.Hkv + h;
     float inv[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) inv[e] = p.vinv[bh * dp + tc.c0 + e];
     load_tile<T>(v, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_v, tc);
+    if (p.v_fp16) {
+      // fp16_rne(v * inv): 16 tokens of one channel = 32 bytes (padded tokens and channels read 0)
+      uint16_t* vt = reinterpret_cast<uint16_t*>(p.v8t);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        uint32_t w[8];
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          const __half2 h2 = __floats2half2_rn(__fmul_rn(elem<T>(v[2 * q], e), inv[e]),
+                                               __fmul_rn(elem<T>(v[2 * q + 1], e), inv[e]));
+          w[q] = *reinterpret_cast<const uint32_t*>(&h2);
+        }
+        uint4* dst = reinterpret_cast<uint4*>(vt + (bh * dp + tc.c0 + e) * p.Np + n0 + tc.g * 16);
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+      return;
+    }
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       uint32_t w[4];

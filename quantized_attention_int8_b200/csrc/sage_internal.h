@@ -29,7 +29,8 @@ struct QuantParams {
   float* ksum_part;  // [B][Hkv][nblk][dp]
   float* vmax_part;  // [B][Hkv][nblk][dp]
   float* vinv;       // [B][Hkv][dp]
-  float vmax_code;   // 448 (fp32 PV accumulation) or 1 (fp16+fp32)
+  float vmax_code;   // 448 (FP8 P.V, fp32 accumulation) or 1 (the other P.V modes)
+  int v_fp16;        // V codes are fp16 (FP16 P.V) instead of E4M3; v8t then holds 2 bytes per code
 };
 
 struct FwdParams {

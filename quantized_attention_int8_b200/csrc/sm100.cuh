@@ -150,8 +150,9 @@ __device__ __forceinline__ uint64_t smem_desc_kmajor(uint32_t saddr, uint32_t ro
   return d;
 }
 
-// Instruction descriptor (kind::i8 / kind::f8f6f4), both operands K-major, dense.
-// c_format: 0 = F16, 1 = F32, 2 = S32.  a/b format: S8 = 1 (kind::i8), E4M3 = 0 (kind::f8f6f4).
+// Instruction descriptor (kind::i8 / kind::f8f6f4 / kind::f16), both operands K-major, dense.
+// c_format: 0 = F16, 1 = F32, 2 = S32.  a/b format: S8 = 1 (kind::i8), E4M3 = 0 (kind::f8f6f4),
+// F16 = 0 (kind::f16).  A and B always get the same format here.
 __host__ __device__ constexpr uint32_t make_idesc(uint32_t c_format, uint32_t ab_format, int M, int N) {
   return (c_format << 4) | (ab_format << 7) | (ab_format << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
@@ -173,6 +174,16 @@ __device__ __forceinline__ void umma_f8(uint32_t tmem_d, uint64_t adesc, uint64_
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
       "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }

@@ -90,6 +90,7 @@ def oracle_to_device(qz: dict) -> dict:
     z = {k: torch.from_numpy(np.ascontiguousarray(qz[k])).cuda() for k in ("q8", "qs", "k8", "ks", "km", "vs")}
     z["v8t"] = torch.from_numpy(v8t).cuda()
     z.update({k: qz[k] for k in ("B", "Hq", "Hkv", "N", "d")})
+    z["pv_dtype"] = "fp16" if qz["pv_mode"] & 2 else "fp8"
     return z
 
 
@@ -107,4 +108,10 @@ def vmax_of(v) -> float:
 
 
 def pv_name(w: W.Workload) -> str:
-    return "fp32" if w.pv_mode == 0 else "fp16+fp32"
+    """pv_accum_dtype of the workload's P.V mode."""
+    return "fp16+fp32" if w.pv_mode & 1 else "fp32"
+
+
+def pv_dtype(w: W.Workload) -> str:
+    """pv_dtype (P.V operands) of the workload's P.V mode."""
+    return "fp16" if w.pv_mode & 2 else "fp8"

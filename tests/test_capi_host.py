@@ -51,7 +51,7 @@ def test_sage_attn_argument_checks(lib):
     assert _attn(lib, Hq=3, Hkv=2) == E                      # GQA needs Hq % Hkv == 0
     assert _attn(lib, d=257) == E and _attn(lib, d=0) == E
     assert _attn(lib, N=0) == E and _attn(lib, B=0) == E
-    assert _attn(lib, layout=2) == E and _attn(lib, pv=2) == E
+    assert _attn(lib, layout=2) == E and _attn(lib, pv=4) == E and _attn(lib, pv=-1) == E
     assert _attn(lib, out=FAKE + 10) == E                     # out overlaps q
     assert _attn(lib, B=70000) == E                           # beyond the launch grid
 
@@ -71,9 +71,10 @@ def test_other_entry_points_argument_checks(lib):
 
 def test_workspace_bytes(lib):
     assert lib.sage_workspace_bytes(1, 2, 2, 0, 64) == 0
-    # q8 + k8 + v8 codes dominate: (Hq + 2 Hkv) * Np * dp bytes, plus fp32 scales and partial sums
+    # q8 + k8 + V codes dominate: (Hq + Hkv + 2 Hkv) * Np * dp bytes (V codes counted at the
+    # 2 bytes of the FP16 P.V modes, the largest), plus fp32 scales and partial sums
     ws = lib.sage_workspace_bytes(2, 8, 2, 1000, 96)
-    codes = 2 * (8 + 2 * 2) * 1024 * 128
+    codes = 2 * (8 + 2 + 2 * 2) * 1024 * 128
     assert codes < ws < codes + 2 * 2 * 8 * 128 * 4 * 2 + 64 * 1024
 
 

@@ -6,7 +6,7 @@ import torch
 import workloads as W
 from oracle import attention, emulate, quant
 from tests._support import (check_vs_emulation, check_vs_exact, cuda, nkeys, oracle_to_device, out_hnd,
-                            pv_name, slice_heads, vmax_of)
+                            pv_dtype, pv_name, slice_heads, vmax_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -24,6 +24,19 @@ SMALL = [
     W.TINY.with_(name="d96_causal_fp16acc", N=1000, d=96, causal=True, pv_mode=1, dist="uniform2", sm_scale=None),
     W.TINY.with_(name="d256_causal_fp16acc_nhd", N=300, d=256, causal=True, pv_mode=1, layout="NHD",
                  sm_scale=None),
+    # INT8-QK / FP16-PV kernel (64-key tiles): fp32 and fp16+fp32 accumulation
+    W.TINY.with_(name="pv16_tiny", pv_mode=2),
+    W.TINY.with_(name="pv16acc_tiny_causal", causal=True, pv_mode=3),
+    W.TINY.with_(name="pv16_ragged_d40_gqa_bf16", N=300, d=40, Hq=4, Hkv=2, dtype="bf16", pv_mode=2),
+    W.TINY.with_(name="pv16_single_token_d96", N=1, d=96, pv_mode=2),
+    W.TINY.with_(name="pv16acc_nhd_koffset_d128", N=700, d=128, layout="NHD", dist="normal_koffset", pv_mode=3,
+                 sm_scale=None),
+    W.TINY.with_(name="pv16_d256_uniform_causal", B=2, N=329, d=256, dist="uniform2", causal=True, pv_mode=2,
+                 sm_scale=None),
+    W.TINY.with_(name="pv16acc_d256_nhd", N=300, d=256, pv_mode=3, layout="NHD", sm_scale=None),
+    W.TINY.with_(name="pv16_outlier_gqa4_causal_bf16", N=640, d=64, Hq=8, Hkv=2, dist="normal_koutlier",
+                 dtype="bf16", causal=True, pv_mode=2),
+    W.TINY.with_(name="pv16acc_d96_causal", N=1000, d=96, causal=True, pv_mode=3, dist="uniform2", sm_scale=None),
 ]
 
 
@@ -46,7 +59,7 @@ def test_attention_kernel_reproduces_method(lib, w):
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
 def test_sage_attn_vs_exact_attention(lib, w):
     q, k, v = W.make_inputs(w)
-    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w))
+    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w))
     lib.sage_check_status()
     ref = attention.attention_f64(q, k, v, w.layout, w.causal, _scale(w))
     em = None
@@ -56,11 +69,11 @@ def test_sage_attn_vs_exact_attention(lib, w):
     check_vs_exact(out_hnd(out, w.layout), ref, nkeys(w.N, w.causal), vmax_of(v), w.name, emul=em)
 
 
-@pytest.mark.parametrize("w", SMALL[:6], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", SMALL[:6] + SMALL[10:13], ids=lambda w: w.name)
 def test_end_to_end_equals_quantize_then_attend(lib, w):
     q, k, v = (cuda(t) for t in W.make_inputs(w))
-    a = lib.sage_attn(q, k, v, w.layout, w.causal, _scale(w), pv_name(w))
-    z = lib.sage_quantize(q, k, v, w.layout, pv_name(w))
+    a = lib.sage_attn(q, k, v, w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w))
+    z = lib.sage_quantize(q, k, v, w.layout, pv_name(w), pv_dtype(w))
     b = lib.sage_attn_quantized(z, q.dtype, w.layout, w.causal, _scale(w), pv_name(w))
     lib.sage_check_status()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
@@ -92,7 +105,7 @@ def test_rejects_bad_inputs(lib):
 
 
 FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"],
-        W.BY_NAME["pad_sweep_b8_h16_n16384_d64_full"], W.BY_NAME["pad_sweep_b8_h16_n1024_d96_full"]]
+        W.BY_NAME["pad_sweep_b8_h16_n16384_d64_full"], W.BY_NAME["pad_sweep_b8_h16_n1024_d96_full"]] + W.FP16_PV
 
 
 def _rows(out, layout, b, h, rows):
@@ -104,7 +117,7 @@ def _rows(out, layout, b, h, rows):
 def test_full_size_sampled_rows(lib, w):
     """The full-size launch the bench times; the oracle checks sampled heads and 128-row blocks."""
     q, k, v = W.make_inputs(w)
-    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w))
+    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w))
     lib.sage_check_status()
     G = w.Hq // w.Hkv
     nb = (w.N + 127) // 128

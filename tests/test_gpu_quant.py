@@ -5,7 +5,7 @@ import torch
 
 import workloads as W
 from oracle import quant
-from tests._support import cuda, slice_heads
+from tests._support import cuda, pv_dtype, pv_name, slice_heads
 
 pytestmark = pytest.mark.gpu
 
@@ -17,11 +17,14 @@ SMALL = [
     W.TINY.with_(name="d256_uniform", B=2, N=129, d=256, dist="uniform2"),
     W.TINY.with_(name="outlier_gqa4", N=640, d=64, Hq=8, Hkv=2, dist="normal_koutlier", dtype="bf16"),
     W.TINY.with_(name="d33_causal", N=257, d=33, Hq=3, Hkv=1, causal=True),
+    W.TINY.with_(name="pv16_ragged_d40_gqa_bf16", N=300, d=40, Hq=4, Hkv=2, dtype="bf16", pv_mode=2),
+    W.TINY.with_(name="pv16acc_nhd_koffset_d128", N=700, d=128, layout="NHD", dist="normal_koffset", pv_mode=3),
+    W.TINY.with_(name="pv16_d256_outlier", B=2, N=129, d=256, dist="normal_koutlier", pv_mode=2),
 ]
 
 
 def _gpu_codes(lib, w, q, k, v):
-    z = lib.sage_quantize(cuda(q), cuda(k), cuda(v), w.layout, "fp32" if w.pv_mode == 0 else "fp16+fp32")
+    z = lib.sage_quantize(cuda(q), cuda(k), cuda(v), w.layout, pv_name(w), pv_dtype(w))
     lib.sage_check_status()
     out = {k2: z[k2].cpu().numpy() for k2 in ("q8", "qs", "k8", "ks", "km", "vs")}
     out["v8"] = z["v8t"].cpu().numpy().transpose(0, 1, 3, 2)
@@ -35,6 +38,8 @@ def _assert_same(got, ref, q_sel=slice(None), kv_sel=slice(None)):
         g, r = got[key][kv_sel], ref[key]
         if g.dtype == np.float32:
             ok = np.array_equal(g.view(np.uint32), r.view(np.uint32))
+        elif g.dtype == np.float16:  # fp16 V codes, compared bit for bit
+            ok = r.dtype == np.float16 and np.array_equal(g.view(np.uint16), r.view(np.uint16))
         else:
             ok = np.array_equal(g, r)
         if not ok:
@@ -50,7 +55,7 @@ def test_quantize_bit_exact_small(lib, w):
     _assert_same(got, ref)
 
 
-FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"]]
+FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"], W.FP16_PV[1]]
 
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)

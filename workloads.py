@@ -47,7 +47,8 @@ class Workload:
     layout: str = "HND"           # "HND" = (B,H,N,d), "NHD" = (B,N,H,d)
     causal: bool = False
     dist: str = "normal"          # see module docstring
-    pv_mode: int = 0              # 0 = FP8 PV with fp32 accumulation, 1 = fp16+fp32
+    pv_mode: int = 0              # P.V: 0 = FP8, fp32 accumulation; 1 = FP8, fp16+fp32;
+                                  # 2 = FP16 operands, fp32; 3 = FP16 operands, fp16+fp32
     seed: int = 0
     sm_scale: float | None = None  # None -> 1/sqrt(d)
 
@@ -79,7 +80,12 @@ def pad_sweep() -> Iterator[Workload]:
                                8, 16, 16, n, d, "fp16", "HND", causal, "uniform2", 0, 5)
 
 
-ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep())
+# The same inputs through the INT8-QK / FP16-PV kernel (fp32 and fp16+fp32 accumulation).
+FP16_PV = [IMAGE_DIT.with_(name="image_dit_b2_h24_n4096_d64_pv16", pv_mode=2),
+           VIDEO_DIT.with_(name="video_dit_b1_h24_n32768_d128_nhd_pv16", pv_mode=3),
+           LLM_GQA.with_(name="llm_causal_gqa_b4_hq32_hkv8_n8192_d128_pv16", pv_mode=2)]
+
+ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV
 BY_NAME = {w.name: w for w in ALL}
 
 
