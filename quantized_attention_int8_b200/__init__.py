@@ -40,11 +40,20 @@ SAGE_PV_FP32, SAGE_PV_FP16_FP32, SAGE_PV16_FP32, SAGE_PV16_FP16_FP32 = 0, 1, 2, 
 _LAYOUTS = {"HND": SAGE_HND, "NHD": SAGE_NHD}
 _DTYPES = {torch.float16: SAGE_FP16, torch.bfloat16: SAGE_BF16, torch.float32: SAGE_FP32}
 _PV = {("fp8", "fp32"): SAGE_PV_FP32, ("fp8", "fp16+fp32"): SAGE_PV_FP16_FP32,
-       ("fp16", "fp32"): SAGE_PV16_FP32, ("fp16", "fp16+fp32"): SAGE_PV16_FP16_FP32}
+       ("fp8", "fp32+fp16"): SAGE_PV_FP16_FP32,
+       ("fp16", "fp32"): SAGE_PV16_FP32, ("fp16", "fp16+fp32"): SAGE_PV16_FP16_FP32,
+       ("fp16", "fp16"): SAGE_PV16_FP32}
 
 
 def pv_mode(pv_dtype: str = "fp8", pv_accum_dtype: str = "fp32") -> int:
-    """The sage_pv_mode value for P.V operands ``pv_dtype`` and accumulation ``pv_accum_dtype``."""
+    """The sage_pv_mode value for P.V operands ``pv_dtype`` and accumulation ``pv_accum_dtype``.
+
+    "fp32+fp16" is the README's spelling of the two-level (fp16 tile, fp32 total)
+    accumulation of the FP8 kernel.  "fp16" (pure fp16 accumulation, offered for the
+    FP16 kernel as the fastest and least overflow-safe option) runs with the fp32 TMEM
+    accumulator: on sm_100a a tcgen05 MMA issues at the same rate with an F16 or an F32
+    accumulator, so fp16 accumulation would buy no speed and only add error.
+    """
     try:
         return _PV[(pv_dtype, pv_accum_dtype)]
     except KeyError:

@@ -82,3 +82,13 @@ def test_padded_dim(lib):
     assert [lib.padded_dim(d) for d in (1, 64, 65, 128, 129, 256)] == [64, 64, 128, 128, 256, 256]
     with pytest.raises(ValueError):
         lib.padded_dim(300)
+
+
+def test_pv_mode_names(lib):
+    assert lib.pv_mode() == lib.SAGE_PV_FP32 == 0
+    assert lib.pv_mode("fp8", "fp16+fp32") == lib.pv_mode("fp8", "fp32+fp16") == lib.SAGE_PV_FP16_FP32 == 1
+    assert lib.pv_mode("fp16", "fp32") == lib.pv_mode("fp16", "fp16") == lib.SAGE_PV16_FP32 == 2
+    assert lib.pv_mode("fp16", "fp16+fp32") == lib.SAGE_PV16_FP16_FP32 == 3
+    for bad in (("fp8", "fp16"), ("int8", "fp32"), ("fp16", "bf16")):
+        with pytest.raises(ValueError):
+            lib.pv_mode(*bad)
