@@ -14,8 +14,9 @@ sums; the pages fix neither):
 
 1. S = Q8 . K8^T exactly in integers (K8 holds codes of K - mean(K)).
 2. Dequantize in the log2 domain: s = S * f with
-   f = (qs * ks) * (sm_scale * log2(e)), all float32.  Keys j >= N, and
-   j > i under the causal mask, are excluded.
+   f = (qs * ks) * (sm_scale * log2(e)), all float32.  Keys j >= Nk, and
+   j > i + (Nk - Nq) under the (bottom-right aligned) causal mask, are
+   excluded; a row that sees no key at all outputs zeros.
 3. Online softmax against a reference max m: the reference moves to
    m' = max(m, row max of s) only when that exceeds m by more than
    tau = 2 (log2 units), else it stays (m' = m); p = 2^(s - m') <= 2^tau;
@@ -56,8 +57,11 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
     Rows beyond N are returned as NaN.
     """
     B, Hq, Hkv, N, d = qz["B"], qz["Hq"], qz["Hkv"], qz["N"], qz["d"]
+    Nk = qz.get("Nk", N)
+    off = Nk - N                      # causal: query i sees keys j <= i + off
     G = Hq // Hkv
     nb = (N + BLOCK - 1) // BLOCK
+    nbk = (Nk + BLOCK - 1) // BLOCK
     mode = qz["pv_mode"]
     hs = [(b, h) for b in range(B) for h in range(Hq)] if heads is None else list(heads)
     qbs = list(range(nb)) if q_blocks is None else list(q_blocks)
@@ -78,16 +82,18 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
             m = np.full(BLOCK, -np.inf, F32)
             l = np.zeros(BLOCK, F32)
             O = np.zeros((BLOCK, qz["dp"]), F32)
-            n_tiles = (qb + 1) * BLOCK // T if causal else nb * BLOCK // T
+            n_tiles = nbk * BLOCK // T
+            if causal:  # tiles up to the one holding the block's last visible key
+                n_tiles = min(n_tiles, max(0, (qb * BLOCK + BLOCK - 1 + off) // T + 1))
             for j in range(n_tiles):
                 keys = j * T + np.arange(T)
-                if keys[0] >= N:
+                if keys[0] >= Nk:
                     break
                 k8 = qz["k8"][b, hk, j * T:(j + 1) * T].astype(np.int64)
                 S = q8 @ k8.T
-                valid = (keys[None, :] < N) & np.ones((BLOCK, 1), bool)
+                valid = (keys[None, :] < Nk) & np.ones((BLOCK, 1), bool)
                 if causal:
-                    valid &= keys[None, :] <= rows[:, None]
+                    valid &= keys[None, :] <= rows[:, None] + off
                 f = F32(F32(qz["qs"][b, h, qb]) * F32(qz["ks"][b, hk, keys[0] // BLOCK])) * c
                 smax = np.where(valid, S, np.iinfo(np.int64).min).max(axis=1)
                 has = valid.any(axis=1)
@@ -112,7 +118,9 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
                 O = (O * alpha[:, None] + pv.astype(F32)).astype(F32)
                 m = m_new
             vs = qz["vs"][b, hk].astype(F32)
-            o = (O * vs[None, :] / (pscale * l[:, None])).astype(F32)
+            with np.errstate(divide="ignore", invalid="ignore"):
+                o = (O * vs[None, :] / (pscale * l[:, None])).astype(F32)
+            o[l == 0] = 0.0                                   # rows that saw no key
             ok = rows < N
             out[n, r * BLOCK:(r + 1) * BLOCK][ok] = o[ok, :d]
     return out

@@ -167,12 +167,12 @@ def fp16_per_channel(v: np.ndarray, dp: int):
 def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
     """The whole quantization step for one attention call.
 
-    q: (B, Hq, N, d), k and v: (B, Hkv, N, d) in ``layout`` (fp16/bf16 torch
+    q: (B, Hq, Nq, d), k and v: (B, Hkv, Nk, d) in ``layout`` (fp16/bf16 torch
     tensors or arrays).  Returns a dict of numpy arrays:
-      q8 int8 (B,Hq,Np,dp), qs f32 (B,Hq,nb), k8 int8 (B,Hkv,Np,dp),
-      ks f32 (B,Hkv,nb), km f32 (B,Hkv,dp), v8 (B,Hkv,Np,dp) V codes (uint8 E4M3
+      q8 int8 (B,Hq,Nq_pad,dp), qs f32 (B,Hq,nbq), k8 int8 (B,Hkv,Nk_pad,dp),
+      ks f32 (B,Hkv,nbk), km f32 (B,Hkv,dp), v8 (B,Hkv,Nk_pad,dp) V codes (uint8 E4M3
       for PV modes 0/1, float16 for the FP16 P.V modes 2/3), vs f32 (B,Hkv,dp),
-      plus the sizes.
+      plus the sizes (N = Nq, Nk).  Q and K are quantized on their own lengths.
     """
     qf, kf, vf = (to_hnd(t, layout) for t in (q, k, v))
     B, Hq, N, d = qf.shape
@@ -189,7 +189,7 @@ def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
     kmp = np.zeros((B, Hkv, dp), F32)
     kmp[:, :, :d] = km
     return dict(q8=q8, qs=qs, k8=k8, ks=ks, km=kmp, v8=v8, vs=vs,
-                B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, dp=dp, pv_mode=pv_mode)
+                B=B, Hq=Hq, Hkv=Hkv, N=N, Nk=kf.shape[2], d=d, dp=dp, pv_mode=pv_mode)
 
 
 def qk_int32(q8: np.ndarray, k8: np.ndarray) -> np.ndarray:

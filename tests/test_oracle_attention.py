@@ -177,3 +177,109 @@ def test_fp16_v_codes_bound():
     # fp16 keeps 11 significant bits: relative error <= 2^-11 (subnormals: 2^-25 absolute)
     assert np.all(np.abs(rec - v) <= np.maximum(np.abs(v) * 2.0 ** -11, 2.0 ** -25 * scale[:, :, None, :20]) * (1 + 1e-6))
     assert np.all(np.abs(codes[:, :, :200, :20]).max(axis=2) == 1.0)
+
+
+def _brute_rect(q, k, v, causal, scale):
+    # pure-python loops; causal keeps key j for query i iff j <= i + (Nk - Nq); rows that see no key -> 0
+    Nq, Nk, d = len(q), len(k), len(v[0])
+    out = []
+    for i in range(Nq):
+        js = [j for j in range(Nk) if (not causal or j <= i + Nk - Nq)]
+        if not js:
+            out.append([0.0] * d)
+            continue
+        s = [scale * sum(q[i][c] * k[j][c] for c in range(len(q[0]))) for j in js]
+        m = max(s)
+        e = [math.exp(x - m) for x in s]
+        z = sum(e)
+        out.append([sum(e[t] * v[js[t]][c] for t in range(len(js))) / z for c in range(d)])
+    return out
+
+
+@pytest.mark.parametrize("nq,nk", [(5, 9), (9, 5), (1, 7), (7, 1)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_rectangular_brute_force(nq, nk, causal):
+    rng = np.random.default_rng(10 + nq * 10 + nk)
+    q = rng.standard_normal((1, 1, nq, 3)).astype(np.float32)
+    k, v = (rng.standard_normal((1, 1, nk, 3)).astype(np.float32) for _ in range(2))
+    got = attention.attention_f64(q, k, v, "HND", causal, 0.6)[0, 0]
+    ref = _brute_rect(q[0, 0].tolist(), k[0, 0].tolist(), v[0, 0].tolist(), causal, 0.6)
+    assert np.allclose(got, ref, rtol=1e-12, atol=1e-12)
+
+
+def test_rectangular_matches_sdpa_with_bottom_right_mask():
+    rng = np.random.default_rng(11)
+    for nq, nk in ((40, 100), (100, 40), (33, 33)):
+        # float32-representable values (the oracle widens its inputs from float32, like fp16/bf16)
+        q = torch.from_numpy(rng.standard_normal((2, 4, nq, 16)).astype(np.float32)).double()
+        k, v = (torch.from_numpy(rng.standard_normal((2, 2, nk, 16)).astype(np.float32)).double() for _ in range(2))
+        got = attention.attention_f64(q, k, v, "HND", True, 0.25)
+        i = torch.arange(nq)[:, None]
+        j = torch.arange(nk)[None, :]
+        mask = j <= i + (nk - nq)
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q, k.repeat_interleave(2, 1), v.repeat_interleave(2, 1), attn_mask=mask, scale=0.25)
+        seen = mask.any(1)                    # SDPA gives NaN on rows with no key; the reading is 0
+        assert np.allclose(got[:, :, seen.numpy()], ref[:, :, seen].numpy(), rtol=1e-10, atol=1e-12)
+        assert np.all(got[:, :, ~seen.numpy()] == 0)
+    # one query row with the causal mask sees every key (bottom-right alignment)
+    q1 = q[:, :, -1:]
+    assert np.allclose(attention.attention_f64(q1, k, v, "HND", True, 0.25),
+                       attention.attention_f64(q1, k, v, "HND", False, 0.25))
+
+
+def test_varlen_matches_block_diagonal_sdpa():
+    rng = np.random.default_rng(12)
+    lq, lk = [37, 1, 130, 0, 64], [50, 3, 130, 7, 1]
+    cq, ck = np.concatenate([[0], np.cumsum(lq)]), np.concatenate([[0], np.cumsum(lk)])
+    q = torch.from_numpy(rng.standard_normal((cq[-1], 4, 8)).astype(np.float32)).double()
+    k, v = (torch.from_numpy(rng.standard_normal((ck[-1], 2, 8)).astype(np.float32)).double() for _ in range(2))
+    for causal in (False, True):
+        got = attention.attention_varlen_f64(q, k, v, cq, ck, causal, 0.3)
+        mask = torch.zeros((cq[-1], ck[-1]), dtype=torch.bool)
+        for b in range(len(lq)):
+            i = torch.arange(lq[b])[:, None]
+            j = torch.arange(lk[b])[None, :]
+            mask[cq[b]:cq[b + 1], ck[b]:ck[b + 1]] = (j <= i + lk[b] - lq[b]) if causal else True
+        ref = torch.nn.functional.scaled_dot_product_attention(
+            q.permute(1, 0, 2)[None], k.permute(1, 0, 2).repeat_interleave(2, 0)[None],
+            v.permute(1, 0, 2).repeat_interleave(2, 0)[None], attn_mask=mask, scale=0.3)[0].permute(1, 0, 2)
+        seen = mask.any(1).numpy()
+        assert np.allclose(got[seen], ref[seen].numpy(), rtol=1e-10, atol=1e-12)
+        assert np.all(got[~seen] == 0)
+    # equal lengths: the packed batch is the dense NHD batch
+    w = W.TINY.with_(N=70, d=16, Hq=4, Hkv=2, B=3, layout="NHD")
+    qd, kd, vd = W.make_inputs(w)
+    cu = np.arange(4) * 70
+    dense = attention.attention_f64(qd, kd, vd, "NHD", True, 0.3)          # (B, Hq, N, d)
+    packed = attention.attention_varlen_f64(qd.reshape(-1, 4, 16), kd.reshape(-1, 2, 16), vd.reshape(-1, 2, 16),
+                                            cu, cu, True, 0.3)
+    assert np.allclose(packed.reshape(3, 70, 4, 16).transpose(0, 2, 1, 3), dense)
+
+
+@pytest.mark.parametrize("mode", [0, 2])
+def test_emulation_rectangular_closed_forms(mode):
+    # Q = 0 with exactly representable V: row i is the mean of v[0 .. i + Nk - Nq] (causal), or of all V
+    rng = np.random.default_rng(13)
+    for nq, nk in ((200, 300), (300, 140)):
+        q = np.zeros((1, 1, nq, 8), np.float32)
+        k = rng.standard_normal((1, 1, nk, 8)).astype(np.float32)
+        v = rng.choice([-1.0, -0.5, 0.5, 1.0], size=(1, 1, nk, 8)).astype(np.float32)
+        v[0, 0, 0] = 1.0
+        qz = quant.quantize(q, k, v, "HND", mode)
+        assert qz["N"] == nq and qz["Nk"] == nk
+        em = emulate.emulate(qz, False, 0.35)[0, :nq]
+        assert np.allclose(em, v[0, 0].mean(0)[None].repeat(nq, 0), rtol=1e-6, atol=1e-7)
+        emc = emulate.emulate(qz, True, 0.35)[0, :nq]
+        cum = np.cumsum(v[0, 0].astype(np.float64), 0) / np.arange(1, nk + 1)[:, None]
+        last = np.arange(nq) + nk - nq                     # last visible key of each row
+        ref = np.where(last[:, None] >= 0, cum[np.clip(last, 0, None)], 0.0)
+        assert np.allclose(emc, ref, rtol=1e-6, atol=1e-7)
+        # and the method tracks exact attention on random Q
+        qr = rng.standard_normal((1, 2, nq, 64)).astype(np.float32)
+        kr, vr = (rng.standard_normal((1, 2, nk, 64)).astype(np.float32) for _ in range(2))
+        qz = quant.quantize(qr, kr, vr, "HND", mode)
+        for causal in (False, True):
+            em = emulate.emulate(qz, causal, 0.125).reshape(1, 2, -1, 64)[:, :, :nq].astype(np.float64)
+            ex = attention.attention_f64(qr, kr, vr, "HND", causal, 0.125)
+            assert (em * ex).sum() / np.sqrt((em ** 2).sum() * (ex ** 2).sum()) >= 0.999
