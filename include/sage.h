@@ -91,6 +91,35 @@ sage_status sage_attn(const void* q, const void* k, const void* v, void* out, in
                       sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
                       void* stream);
 
+/* sage_attn with different query and key lengths (SageAttention README news,
+ * 2024-11-11: different sequence lengths between q and k, v).  q, out:
+ * (B,Hq,Nq,d), k and v: (B,Hkv,Nk,d), in `layout`.  Under is_causal the mask is
+ * aligned bottom-right: query i sees keys j <= i + (Nk - Nq), so the last query
+ * sees every key; a query that sees no key (Nq > Nk) gets zeros.  Nq = Nk is
+ * exactly sage_attn.  Workspace, errors and ownership as sage_attn. */
+sage_status sage_attn_ex(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Nq,
+                         int Nk, int d, sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale,
+                         sage_pv_mode pv_mode, void* stream);
+
+/* Packed batch of sequences of different lengths (SageAttention README,
+ * "Available APIs": sageattn_varlen).  q, out: (total_q, Hq, d); k, v:
+ * (total_k, Hkv, d), tokens of all sequences one after the other (contiguous).
+ * cu_seqlens_q / cu_seqlens_k: DEVICE int32 arrays of B + 1 non-decreasing
+ * offsets; sequence b owns query tokens cu_seqlens_q[b] .. cu_seqlens_q[b+1]-1
+ * and key tokens cu_seqlens_k[b] .. cu_seqlens_k[b+1]-1.  Every sequence is
+ * quantized on its own (K mean, 128-token blocks and V scales per sequence) and
+ * attends only to its own keys, with the causal mask aligned bottom-right per
+ * sequence; queries that see no key (including sequences with no keys) get
+ * zeros.  max_seqlen_q >= 1 and max_seqlen_k >= 0 bound every sequence's
+ * lengths; cu_seqlens_*[B] must not exceed total_q / total_k.  The table is
+ * checked on the device: a violation is reported by sage_check_status as
+ * SAGE_ERR_INVALID_ARG, and then no output is written.  Workspace, other errors
+ * and ownership as sage_attn. */
+sage_status sage_attn_varlen(const void* q, const void* k, const void* v, void* out, const int32_t* cu_seqlens_q,
+                             const int32_t* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
+                             long long total_q, long long total_k, int Hq, int Hkv, int d, sage_dtype dtype,
+                             int is_causal, float sm_scale, sage_pv_mode pv_mode, void* stream);
+
 /* Bytes of workspace sage_attn takes for these sizes, the largest over the P.V
  * modes (0 on invalid sizes). */
 size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d);

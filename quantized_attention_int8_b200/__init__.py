@@ -26,7 +26,7 @@ import torch
 __all__ = [
     "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
     "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
-    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode",
+    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode", "sage_attn_varlen",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
@@ -77,6 +77,9 @@ def _load() -> ctypes.CDLL:
         "sage_status_string": ([I], ctypes.c_char_p),
         "sage_device_supported": ([], I),
         "sage_attn_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
+        "sage_attn_ex": ([P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P], I),
+        "sage_attn_varlen": ([P, P, P, P, P, P, I, I, I, ctypes.c_longlong, ctypes.c_longlong, I, I, I, I, I, F, I, P],
+                             I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -117,16 +120,16 @@ def _shape(q: torch.Tensor, k: torch.Tensor, layout: str):
         raise ValueError("q, k, v must be 4-D")
     if layout == "HND":
         B, Hq, N, d = q.shape
-        Hkv = k.shape[1]
+        Hkv, Nk = k.shape[1], k.shape[2]
     elif layout == "NHD":
         B, N, Hq, d = q.shape
-        Hkv = k.shape[2]
+        Hkv, Nk = k.shape[2], k.shape[1]
     else:
         raise ValueError(f"tensor_layout must be 'HND' or 'NHD', got {layout!r}")
-    return B, Hq, Hkv, N, d
+    return B, Hq, Hkv, N, Nk, d
 
 
-def _check_inputs(q, k, v, layout):
+def _check_tensors(q, k, v):
     for t in (q, k, v):
         if not t.is_cuda:
             raise ValueError("q, k, v must be CUDA tensors (no CPU path exists)")
@@ -136,26 +139,77 @@ def _check_inputs(q, k, v, layout):
         raise ValueError("q, k, v must share one dtype")
     if k.shape != v.shape:
         raise ValueError("k and v must have the same shape")
-    B, Hq, Hkv, N, d = _shape(q, k, layout)
-    kshape = (B, Hkv, N, d) if layout == "HND" else (B, N, Hkv, d)
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+
+
+def _check_inputs_nk(q, k, v, layout):
+    """(B, Hq, Hkv, Nq, Nk, d) of q and k, v, which may differ in length."""
+    _check_tensors(q, k, v)
+    B, Hq, Hkv, N, Nk, d = _shape(q, k, layout)
+    kshape = (B, Hkv, Nk, d) if layout == "HND" else (B, Nk, Hkv, d)
     if tuple(k.shape) != kshape:
         raise ValueError(f"k has shape {tuple(k.shape)}, expected {kshape}")
+    return B, Hq, Hkv, N, Nk, d
+
+
+def _check_inputs(q, k, v, layout):
+    """(B, Hq, Hkv, N, d) of q, k, v of one length."""
+    B, Hq, Hkv, N, Nk, d = _check_inputs_nk(q, k, v, layout)
+    if Nk != N:
+        raise ValueError(f"q has {N} tokens and k, v {Nk}; this entry point needs equal lengths")
     return B, Hq, Hkv, N, d
 
 
 def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None,
               pv_dtype="fp8"):
-    """Quantized attention of fp16/bf16 q (B,Hq,N,d), k/v (B,Hkv,N,d) (HND; NHD stores (B,N,H,d))."""
-    B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
-    if q.dtype not in _DTYPES:
-        raise ValueError(f"unsupported dtype {q.dtype}")
+    """Quantized attention of fp16/bf16 q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) (HND; NHD stores (B,N,H,d)).
+
+    Nq may differ from Nk (then through sage_attn_ex: the causal mask is aligned bottom-right)."""
+    B, Hq, Hkv, N, Nk, d = _check_inputs_nk(q, k, v, tensor_layout)
     if out is None:
         out = torch.empty_like(q)
-    st = capi.sage_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
-                        _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)),
-                        float(sm_scale) if sm_scale is not None else 0.0, pv_mode(pv_dtype, pv_accum_dtype),
-                        _stream())
-    _check(st, "sage_attn")
+    scale = float(sm_scale) if sm_scale is not None else 0.0
+    mode = pv_mode(pv_dtype, pv_accum_dtype)
+    if Nk == N:
+        st = capi.sage_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
+                            _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)), scale, mode, _stream())
+        _check(st, "sage_attn")
+    else:
+        st = capi.sage_attn_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, Nk, d,
+                               _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)), scale, mode,
+                               _stream())
+        _check(st, "sage_attn_ex")
+    return out
+
+
+def sage_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, is_causal=False,
+                     sm_scale=None, pv_accum_dtype="fp32", out=None, pv_dtype="fp8"):
+    """Packed batch: q (total_q, Hq, d), k/v (total_k, Hkv, d), cu_seqlens_* int32 CUDA tensors of
+    B + 1 offsets (sequence b = tokens cu[b] .. cu[b+1]-1).  Each sequence attends to its own keys
+    (causal: aligned bottom-right per sequence).  A bad offset table raises SageError from the
+    status check after the launch."""
+    _check_tensors(q, k, v)
+    if q.dim() != 3 or k.dim() != 3:
+        raise ValueError("varlen q, k, v must be 3-D (tokens, heads, head_dim)")
+    total_q, Hq, d = q.shape
+    total_k, Hkv, dk = k.shape
+    if dk != d:
+        raise ValueError("q and k must have the same head_dim")
+    for c in (cu_seqlens_q, cu_seqlens_k):
+        if not (c.is_cuda and c.dtype == torch.int32 and c.dim() == 1 and c.is_contiguous()):
+            raise ValueError("cu_seqlens must be contiguous 1-D int32 CUDA tensors")
+    if cu_seqlens_q.numel() != cu_seqlens_k.numel() or cu_seqlens_q.numel() < 2:
+        raise ValueError("cu_seqlens_q and cu_seqlens_k must both hold B + 1 >= 2 offsets")
+    B = cu_seqlens_q.numel() - 1
+    if out is None:
+        out = torch.empty_like(q)
+    st = capi.sage_attn_varlen(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), cu_seqlens_q.data_ptr(),
+                               cu_seqlens_k.data_ptr(), B, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k,
+                               Hq, Hkv, d, _DTYPES[q.dtype], int(bool(is_causal)),
+                               float(sm_scale) if sm_scale is not None else 0.0, pv_mode(pv_dtype, pv_accum_dtype),
+                               _stream())
+    _check(st, "sage_attn_varlen")
     return out
 
 
@@ -170,8 +224,6 @@ def sage_attn_noalloc(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=No
     (larger ones raise SageError with SAGE_ERR_INVALID_ARG); calls that may overlap on the
     GPU must be ordered by the caller."""
     B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
-    if q.dtype not in _DTYPES:
-        raise ValueError(f"unsupported dtype {q.dtype}")
     if out is None:
         out = torch.empty_like(q)
     st = capi.sage_attn_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,

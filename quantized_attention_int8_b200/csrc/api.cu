@@ -17,24 +17,88 @@ size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
 int padded_dim(int d) { return d <= 64 ? 64 : (d <= 128 ? 128 : 256); }
 
+// Sizes of one call.  Dense batches: B sequences of Nq queries and Nk keys.  Packed (varlen)
+// batches: B sequences of at most Nq / Nk tokens, total_q / total_k tokens in all.
 struct Dims {
-  int B, Hq, Hkv, N, d, dp, Np, nblk, G;
+  int B, Hq, Hkv, Nq, Nk, d, dp, G;
+  int nblk_q, nblk_k;                  // 128-token blocks of the longest query / key sequence
+  long long q_head_rows, k_head_rows;  // q8 / k8 rows between heads (dense Npq / Npk; packed Tq / Tk)
+  long long q_rows, k_rows;            // q8 / k8 rows in all
+  bool packed;
+  long long total_q, total_k;
 };
 
-sage_status check_dims(int B, int Hq, int Hkv, int N, int d, Dims* out) {
-  if (B < 1 || Hq < 1 || Hkv < 1 || N < 1 || d < 1) return SAGE_ERR_INVALID_ARG;
+long long round128(long long x) { return (x + 127) / 128 * 128; }
+
+sage_status finish_dims(Dims* m) {
+  m->dp = padded_dim(m->d);
+  m->G = m->Hq / m->Hkv;
+  m->nblk_q = (m->Nq + 127) / 128;
+  m->nblk_k = (m->Nk + 127) / 128;
+  if (m->packed) {
+    // every sequence starts a fresh 128-row block: sum of round128(n_b) <= total + 127 B
+    m->q_head_rows = round128(m->total_q) + 128LL * m->B;
+    m->k_head_rows = round128(m->total_k) + 128LL * m->B;
+    m->q_rows = m->q_head_rows * m->Hq;
+    m->k_rows = m->k_head_rows * m->Hkv;
+  } else {
+    m->q_head_rows = round128(m->Nq);
+    m->k_head_rows = round128(m->Nk);
+    m->q_rows = m->q_head_rows * m->Hq * m->B;
+    m->k_rows = m->k_head_rows * m->Hkv * m->B;
+  }
+  // TMA coordinates are 32-bit signed: rows of q8 / k8 / V^T and the byte column of V^T
+  const long long v_rows = m->k_rows / m->k_head_rows * m->dp;
+  if (m->q_rows >= (1LL << 31) || m->k_rows >= (1LL << 31) || v_rows >= (1LL << 31) ||
+      m->k_head_rows * 2 >= (1LL << 31))
+    return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+sage_status check_heads(int B, int Hq, int Hkv, int d) {
+  if (B < 1 || Hq < 1 || Hkv < 1 || d < 1) return SAGE_ERR_INVALID_ARG;
   if (d > 256 || Hq % Hkv != 0) return SAGE_ERR_INVALID_ARG;
-  if (B > 65535 || 2L * Hq > 65535 || (long)Hq + 2L * Hkv > 65535 || N > (1 << 30)) return SAGE_ERR_INVALID_ARG;
+  if (B > 65535 || 2L * Hq > 65535 || (long)Hq + 2L * Hkv > 65535) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+sage_status check_dims(int B, int Hq, int Hkv, int Nq, int Nk, int d, Dims* out) {
+  sage_status s = check_heads(B, Hq, Hkv, d);
+  if (s != SAGE_OK) return s;
+  if (Nq < 1 || Nk < 1 || Nq > (1 << 30) || Nk > (1 << 30)) return SAGE_ERR_INVALID_ARG;
   Dims m;
-  m.B = B, m.Hq = Hq, m.Hkv = Hkv, m.N = N, m.d = d;
-  m.dp = padded_dim(d);
-  m.nblk = (N + 127) / 128;
-  m.Np = m.nblk * 128;
-  m.G = Hq / Hkv;
-  // TMA coordinates are 32-bit signed
-  if ((long long)B * Hq * m.Np >= (1LL << 31) || (long long)B * Hkv * m.dp >= (1LL << 31)) return SAGE_ERR_INVALID_ARG;
+  m.B = B, m.Hq = Hq, m.Hkv = Hkv, m.Nq = Nq, m.Nk = Nk, m.d = d;
+  m.packed = false;
+  m.total_q = (long long)B * Nq, m.total_k = (long long)B * Nk;
+  if ((s = finish_dims(&m)) != SAGE_OK) return s;
   *out = m;
   return SAGE_OK;
+}
+
+sage_status check_dims_packed(int B, int Hq, int Hkv, int max_q, int max_k, long long total_q, long long total_k,
+                              int d, Dims* out) {
+  sage_status s = check_heads(B, Hq, Hkv, d);
+  if (s != SAGE_OK) return s;
+  if (max_q < 1 || max_k < 0 || total_q < 1 || total_k < 0 || max_q > (1 << 30) || max_k > (1 << 30) ||
+      total_q > (1LL << 40) || total_k > (1LL << 40))
+    return SAGE_ERR_INVALID_ARG;
+  Dims m;
+  m.B = B, m.Hq = Hq, m.Hkv = Hkv, m.Nq = max_q, m.Nk = max_k, m.d = d;
+  m.packed = true;
+  m.total_q = total_q, m.total_k = total_k;
+  if ((s = finish_dims(&m)) != SAGE_OK) return s;
+  *out = m;
+  return SAGE_OK;
+}
+
+SeqMap seq_map(const Dims& m, int layout, const SeqDesc* seqs) {
+  SeqMap s;
+  s.seqs = m.packed ? seqs : nullptr;
+  s.B = m.B, s.Hq = m.Hq, s.Hkv = m.Hkv, s.d = m.d, s.dp = m.dp;
+  s.Nq = m.Nq, s.Nk = m.Nk;
+  s.q_head_rows = m.q_head_rows, s.k_head_rows = m.k_head_rows;
+  s.layout = m.packed ? SAGE_NHD : layout;
+  return s;
 }
 
 sage_status check_dtype(int dtype) {
@@ -138,6 +202,7 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t st) {
 }
 
 struct QuantBufs {
+  const SeqDesc* seqs;  // packed batches: the per-sequence table (else nullptr)
   int8_t* q8;
   float* qs;
   int8_t* k8;
@@ -154,16 +219,17 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
   const uint32_t dv = m.dp == 64 ? 64 : 128;
   const bool pv16 = pv_mode_fp16_operands(pv_mode);
   const uint32_t bn = pv16 ? 64 : 128;  // keys per KV tile of the fused kernel
-  const uint64_t vrow = (uint64_t)m.Np * (pv16 ? 2 : 1);  // bytes per V^T row (one channel)
+  const uint64_t vpitch = (uint64_t)m.k_head_rows * (pv16 ? 2 : 1);  // bytes per V^T row (one channel)
   // V^T tile box: 128 bytes of keys (128 E4M3 or 64 fp16 codes) x dv channels
-  if (!make_map(&tq, qb.q8, m.dp, (uint64_t)m.B * m.Hq * m.Np, ksub, 128) ||
-      !make_map(&tk, qb.k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, bn) ||
-      !make_map(&tv, qb.v8t, vrow, (uint64_t)m.B * m.Hkv * m.dp, 128, dv))
+  if (!make_map(&tq, qb.q8, m.dp, (uint64_t)m.q_rows, ksub, 128) ||
+      !make_map(&tk, qb.k8, m.dp, (uint64_t)m.k_rows, ksub, bn) ||
+      !make_map(&tv, qb.v8t, vpitch, (uint64_t)(m.k_rows / m.k_head_rows) * m.dp, 128, dv))
     return SAGE_ERR_CUDA;
   FwdParams p;
   p.qs = qb.qs, p.ks = qb.ks, p.vs = qb.vs, p.out = out;
-  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.N = m.N, p.Np = m.Np, p.nblk = m.nblk, p.d = m.d, p.dp = m.dp, p.G = m.G;
-  p.layout = layout;
+  p.m = seq_map(m, layout, qb.seqs);
+  p.nblk_q = m.nblk_q;
+  p.G = m.G;
   p.n_vhalves = m.dp == 256 ? 2 : 1;
   p.vec_out = (m.d % 8 == 0) && aligned16(out);
   p.scale_log2 = resolve_scale(sm_scale, m.d) * 1.4426950408889634f;
@@ -171,7 +237,7 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
 }
 
 struct WsLayout {
-  size_t q8, qs, k8, ks, km, v8t, vs, ksum, vmax, vinv, total;
+  size_t q8, qs, k8, ks, km, v8t, vs, ksum, vmax, vinv, seqs, total;
 };
 
 WsLayout ws_layout(const Dims& m, int pv_mode) {
@@ -182,16 +248,17 @@ WsLayout ws_layout(const Dims& m, int pv_mode) {
     off = align_up(off + bytes);
     return o;
   };
-  w.q8 = take((size_t)m.B * m.Hq * m.Np * m.dp);
-  w.qs = take((size_t)m.B * m.Hq * m.nblk * 4);
-  w.k8 = take((size_t)m.B * m.Hkv * m.Np * m.dp);
-  w.ks = take((size_t)m.B * m.Hkv * m.nblk * 4);
+  w.q8 = take((size_t)m.q_rows * m.dp);
+  w.qs = take((size_t)m.q_rows / 128 * 4);
+  w.k8 = take((size_t)m.k_rows * m.dp);
+  w.ks = take((size_t)m.k_rows / 128 * 4);
   w.km = take((size_t)m.B * m.Hkv * m.dp * 4);
-  w.v8t = take((size_t)m.B * m.Hkv * m.dp * m.Np * (pv_mode_fp16_operands(pv_mode) ? 2 : 1));
+  w.v8t = take((size_t)m.k_rows * m.dp * (pv_mode_fp16_operands(pv_mode) ? 2 : 1));
   w.vs = take((size_t)m.B * m.Hkv * m.dp * 4);
-  w.ksum = take((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
-  w.vmax = take((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
+  w.ksum = take((size_t)m.k_rows / 128 * m.dp * 4);
+  w.vmax = take((size_t)m.k_rows / 128 * m.dp * 4);
   w.vinv = take((size_t)m.B * m.Hkv * m.dp * 4);
+  w.seqs = take(m.packed ? (size_t)m.B * sizeof(SeqDesc) : 0);
   w.total = off;
   return w;
 }
@@ -201,8 +268,9 @@ QuantParams quant_params(const Dims& m, const void* q, const void* k, const void
   QuantParams p;
   memset(&p, 0, sizeof(p));
   p.q = q, p.k = k, p.v = v;
-  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.N = m.N, p.d = m.d, p.dp = m.dp, p.Np = m.Np, p.nblk = m.nblk;
-  p.layout = layout, p.dtype = dtype;
+  p.m = seq_map(m, layout, nullptr);  // packed batches set p.m.seqs once the table exists
+  p.nblk_q = m.nblk_q, p.nblk_k = m.nblk_k;
+  p.dtype = dtype;
   p.vec_q = (m.d % 8 == 0) && aligned16(q);
   p.vec_k = (m.d % 8 == 0) && aligned16(k);
   p.vec_v = (m.d % 8 == 0) && aligned16(v);
@@ -211,14 +279,59 @@ QuantParams quant_params(const Dims& m, const void* q, const void* k, const void
   return p;
 }
 
-sage_status check_common(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
-                         int dtype, int layout, int pv_mode, Dims* m) {
+sage_status check_common(const void* q, const void* k, const void* v, int dtype, int layout, int pv_mode) {
   if (!q || !k || !v) return SAGE_ERR_INVALID_ARG;
   sage_status s = check_dtype(dtype);
   if (s != SAGE_OK) return s;
   if (layout != SAGE_HND && layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
   if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
-  return check_dims(B, Hq, Hkv, N, d, m);
+  return SAGE_OK;
+}
+
+// out must not overlap q, k or v (2-byte elements)
+bool out_overlaps(const Dims& m, const void* q, const void* k, const void* v, const void* out) {
+  const size_t qbytes = (size_t)m.total_q * m.Hq * m.d * 2, kvbytes = (size_t)m.total_k * m.Hkv * m.d * 2;
+  return overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes);
+}
+
+// Quantize pass + fused kernel on a workspace laid out by ws_layout(m, pv_mode); packed batches
+// first build their per-sequence table from cu_q / cu_k.
+sage_status attend_on(const Dims& m, unsigned char* ws, const void* q, const void* k, const void* v, void* out,
+                      const int32_t* cu_q, const int32_t* cu_k, int dtype, int layout, int causal, float sm_scale,
+                      int pv_mode, cudaStream_t st) {
+  const WsLayout w = ws_layout(m, pv_mode);
+  SeqDesc* seqs = m.packed ? reinterpret_cast<SeqDesc*>(ws + w.seqs) : nullptr;
+  if (m.packed) {
+    sage_status s = from_cuda(launch_seq_plan(cu_q, cu_k, m.B, m.Nq, m.Nk, m.total_q, m.total_k, seqs, st));
+    if (s != SAGE_OK) return s;
+  }
+  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
+  qp.m.seqs = seqs;
+  QuantBufs qb{seqs,
+               reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
+               reinterpret_cast<int8_t*>(ws + w.k8), reinterpret_cast<float*>(ws + w.ks),
+               reinterpret_cast<float*>(ws + w.km), ws + w.v8t, reinterpret_cast<float*>(ws + w.vs)};
+  qp.q8 = qb.q8, qp.qs = qb.qs, qp.k8 = qb.k8, qp.ks = qb.ks, qp.km = qb.km, qp.v8t = qb.v8t, qp.vs = qb.vs;
+  qp.ksum_part = reinterpret_cast<float*>(ws + w.ksum);
+  qp.vmax_part = reinterpret_cast<float*>(ws + w.vmax);
+  qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
+  sage_status s = from_cuda(launch_quantize(qp, st));
+  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, causal, sm_scale, pv_mode, st);
+  return s;
+}
+
+// The same, on a workspace taken from the library's pool and released stream-ordered.
+sage_status attend_pooled(const Dims& m, const void* q, const void* k, const void* v, void* out, const int32_t* cu_q,
+                          const int32_t* cu_k, int dtype, int layout, int causal, float sm_scale, int pv_mode,
+                          cudaStream_t st) {
+  const WsLayout w = ws_layout(m, pv_mode);
+  unsigned char* ws = nullptr;
+  cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), w.total, st);
+  if (e != cudaSuccess) return from_cuda(e);
+  sage_status s = attend_on(m, ws, q, k, v, out, cu_q, cu_k, dtype, layout, causal, sm_scale, pv_mode, st);
+  const cudaError_t ef = cudaFreeAsync(ws, st);
+  if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
+  return s;
 }
 
 }  // namespace
@@ -227,52 +340,56 @@ extern "C" {
 
 size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   Dims m;
-  if (check_dims(B, Hq, Hkv, N, d, &m) != SAGE_OK) return 0;
+  if (check_dims(B, Hq, Hkv, N, N, d, &m) != SAGE_OK) return 0;
   return ws_layout(m, SAGE_PV16_FP32).total;  // the largest over the P.V modes
+}
+
+sage_status sage_attn_ex(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Nq,
+                         int Nk, int d, sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale,
+                         sage_pv_mode pv_mode, void* stream) {
+  sage_status s = check_common(q, k, v, dtype, layout, pv_mode);
+  if (s != SAGE_OK) return s;
+  Dims m;
+  if ((s = check_dims(B, Hq, Hkv, Nq, Nk, d, &m)) != SAGE_OK) return s;
+  if (!out || out_overlaps(m, q, k, v, out)) return SAGE_ERR_INVALID_ARG;
+  if ((s = check_device()) != SAGE_OK) return s;
+  return attend_pooled(m, q, k, v, out, nullptr, nullptr, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode,
+                       static_cast<cudaStream_t>(stream));
 }
 
 sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
                       sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
                       void* stream) {
-  Dims m;
-  sage_status s = check_common(q, k, v, B, Hq, Hkv, N, d, dtype, layout, pv_mode, &m);
+  return sage_attn_ex(q, k, v, out, B, Hq, Hkv, N, N, d, dtype, layout, is_causal, sm_scale, pv_mode, stream);
+}
+
+sage_status sage_attn_varlen(const void* q, const void* k, const void* v, void* out, const int32_t* cu_seqlens_q,
+                             const int32_t* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
+                             long long total_q, long long total_k, int Hq, int Hkv, int d, sage_dtype dtype,
+                             int is_causal, float sm_scale, sage_pv_mode pv_mode, void* stream) {
+  sage_status s = check_common(q, k, v, dtype, SAGE_NHD, pv_mode);
   if (s != SAGE_OK) return s;
-  if (!out) return SAGE_ERR_INVALID_ARG;
-  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
-  if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes))
-    return SAGE_ERR_INVALID_ARG;
+  if (!cu_seqlens_q || !cu_seqlens_k) return SAGE_ERR_INVALID_ARG;
+  Dims m;
+  if ((s = check_dims_packed(B, Hq, Hkv, max_seqlen_q, max_seqlen_k, total_q, total_k, d, &m)) != SAGE_OK) return s;
+  if (!out || out_overlaps(m, q, k, v, out)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const WsLayout w = ws_layout(m, pv_mode);
-  unsigned char* ws = nullptr;
-  cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), w.total, st);
-  if (e != cudaSuccess) return from_cuda(e);
-  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
-  QuantBufs qb{reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
-               reinterpret_cast<int8_t*>(ws + w.k8), reinterpret_cast<float*>(ws + w.ks),
-               reinterpret_cast<float*>(ws + w.km), ws + w.v8t, reinterpret_cast<float*>(ws + w.vs)};
-  qp.q8 = qb.q8, qp.qs = qb.qs, qp.k8 = qb.k8, qp.ks = qb.ks, qp.km = qb.km, qp.v8t = qb.v8t, qp.vs = qb.vs;
-  qp.ksum_part = reinterpret_cast<float*>(ws + w.ksum);
-  qp.vmax_part = reinterpret_cast<float*>(ws + w.vmax);
-  qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
-  s = from_cuda(launch_quantize(qp, st));
-  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode, st);
-  const cudaError_t ef = cudaFreeAsync(ws, st);
-  if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
-  return s;
+  return attend_pooled(m, q, k, v, out, cu_seqlens_q, cu_seqlens_k, dtype, SAGE_NHD, is_causal ? 1 : 0, sm_scale,
+                       pv_mode, static_cast<cudaStream_t>(stream));
 }
 
 sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
                           sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,
                           int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs, void* stream) {
-  Dims m;
-  sage_status s = check_common(q, k, v, B, Hq, Hkv, N, d, dtype, layout, pv_mode, &m);
+  sage_status s = check_common(q, k, v, dtype, layout, pv_mode);
   if (s != SAGE_OK) return s;
+  Dims m;
+  if ((s = check_dims(B, Hq, Hkv, N, N, d, &m)) != SAGE_OK) return s;
   if (!q8 || !qs || !k8 || !ks || !km || !v8t || !vs) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t part = align_up((size_t)m.B * m.Hkv * m.nblk * m.dp * 4);
+  const size_t part = align_up((size_t)m.k_rows / 128 * m.dp * 4);
   const size_t vinv = align_up((size_t)m.B * m.Hkv * m.dp * 4);
   unsigned char* scratch = nullptr;
   cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&scratch), 2 * part + vinv, st);
@@ -298,11 +415,11 @@ sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t*
   if (out_layout != SAGE_HND && out_layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
   if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
   Dims m;
-  if ((s = check_dims(B, Hq, Hkv, N, d, &m)) != SAGE_OK) return s;
+  if ((s = check_dims(B, Hq, Hkv, N, N, d, &m)) != SAGE_OK) return s;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
-  QuantBufs qb{const_cast<int8_t*>(q8), const_cast<float*>(qs), const_cast<int8_t*>(k8), const_cast<float*>(ks),
-               nullptr, const_cast<uint8_t*>(v8t), const_cast<float*>(vs)};
+  QuantBufs qb{nullptr, const_cast<int8_t*>(q8), const_cast<float*>(qs), const_cast<int8_t*>(k8),
+               const_cast<float*>(ks), nullptr, const_cast<uint8_t*>(v8t), const_cast<float*>(vs)};
   return run_fwd(m, qb, out, out_dtype, out_layout, is_causal ? 1 : 0, sm_scale, pv_mode,
                  static_cast<cudaStream_t>(stream));
 }
@@ -311,19 +428,18 @@ sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int
                           const int32_t* tiles, int n_tiles, int32_t* s_out, void* stream) {
   if (!q8 || !k8 || !tiles || !s_out || n_tiles < 0) return SAGE_ERR_INVALID_ARG;
   Dims m;
-  sage_status s = check_dims(B, Hq, Hkv, N, d, &m);
+  sage_status s = check_dims(B, Hq, Hkv, N, N, d, &m);
   if (s != SAGE_OK) return s;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(s_out)) return SAGE_ERR_INVALID_ARG;
   if (n_tiles == 0) return SAGE_OK;
   if ((s = check_device()) != SAGE_OK) return s;
   CUtensorMap tq, tk;
   const uint32_t ksub = m.dp >= 128 ? 128 : 64;
-  if (!make_map(&tq, q8, m.dp, (uint64_t)m.B * m.Hq * m.Np, ksub, 128) ||
-      !make_map(&tk, k8, m.dp, (uint64_t)m.B * m.Hkv * m.Np, ksub, 128))
+  if (!make_map(&tq, q8, m.dp, (uint64_t)m.q_rows, ksub, 128) || !make_map(&tk, k8, m.dp, (uint64_t)m.k_rows, ksub, 128))
     return SAGE_ERR_CUDA;
   QkDumpParams p;
   p.tiles = tiles, p.n_tiles = n_tiles, p.out = s_out;
-  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.Np = m.Np, p.nblk = m.nblk, p.G = m.G;
+  p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.Np = (int)m.q_head_rows, p.nblk = m.nblk_q, p.G = m.G;
   return from_cuda(launch_qk_dump(tq, tk, p, m.dp, static_cast<cudaStream_t>(stream)));
 }
 
@@ -383,13 +499,11 @@ cudaError_t noalloc_scratch(int dev, unsigned char** out) {
 extern "C" sage_status sage_attn_noalloc(const void* q, const void* k, const void* v, void* out, int B, int Hq,
                                          int Hkv, int N, int d, sage_dtype dtype, sage_layout layout, int is_causal,
                                          float sm_scale, sage_pv_mode pv_mode, void* stream) {
-  Dims m;
-  sage_status s = check_common(q, k, v, B, Hq, Hkv, N, d, dtype, layout, pv_mode, &m);
+  sage_status s = check_common(q, k, v, dtype, layout, pv_mode);
   if (s != SAGE_OK) return s;
-  if (!out) return SAGE_ERR_INVALID_ARG;
-  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
-  if (overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes))
-    return SAGE_ERR_INVALID_ARG;
+  Dims m;
+  if ((s = check_dims(B, Hq, Hkv, N, N, d, &m)) != SAGE_OK) return s;
+  if (!out || out_overlaps(m, q, k, v, out)) return SAGE_ERR_INVALID_ARG;
   const WsLayout w = ws_layout(m, pv_mode);
   if (w.total > (size_t)SAGE_NOALLOC_MAX_BYTES) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
@@ -397,16 +511,6 @@ extern "C" sage_status sage_attn_noalloc(const void* q, const void* k, const voi
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
   unsigned char* ws = nullptr;
   if (noalloc_scratch(dev, &ws) != cudaSuccess) return SAGE_ERR_CUDA;
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
-  QuantBufs qb{reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
-               reinterpret_cast<int8_t*>(ws + w.k8), reinterpret_cast<float*>(ws + w.ks),
-               reinterpret_cast<float*>(ws + w.km), ws + w.v8t, reinterpret_cast<float*>(ws + w.vs)};
-  qp.q8 = qb.q8, qp.qs = qb.qs, qp.k8 = qb.k8, qp.ks = qb.ks, qp.km = qb.km, qp.v8t = qb.v8t, qp.vs = qb.vs;
-  qp.ksum_part = reinterpret_cast<float*>(ws + w.ksum);
-  qp.vmax_part = reinterpret_cast<float*>(ws + w.vmax);
-  qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
-  s = from_cuda(launch_quantize(qp, st));
-  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode, st);
-  return s;
+  return attend_on(m, ws, q, k, v, out, nullptr, nullptr, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode,
+                   static_cast<cudaStream_t>(stream));
 }

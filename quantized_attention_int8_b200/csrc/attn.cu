@@ -136,15 +136,32 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
   volatile int* abort = &bars->abort;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  int qt = blockIdx.x;
-  if (CAUSAL) qt = p.nblk - 1 - qt;  // longest rows first
-  const int hq = blockIdx.y / p.n_vhalves, vh = blockIdx.y - hq * p.n_vhalves;
   const int b = blockIdx.z;
+  const SeqView sv = seq_view(p.m, b);
+  const int nq = sv.nq, nk = sv.nk;
+  const int nblk_q = (nq + 127) / 128;
+  int qt = blockIdx.x;
+  if (CAUSAL) qt = nblk_q - 1 - qt;  // longest rows first
+  if (qt < 0 || qt >= nblk_q) return;  // past the end of this sequence (the whole CTA leaves)
+  const int hq = blockIdx.y / p.n_vhalves, vh = blockIdx.y - hq * p.n_vhalves;
   const int hkv = hq / p.G;
-  // KV tiles of C::BN keys: up to the last key below N, and under the causal mask up to the
-  // last key of this query tile's diagonal block
-  const int n_kv_all = (p.N + C::BN - 1) / C::BN;
-  const int n_kv = CAUSAL ? min(n_kv_all, (qt + 1) * (128 / C::BN)) : n_kv_all;
+  // Causal mask, bottom-right aligned: query i sees keys j <= i + (nk - nq).
+  const int koff = nk - nq;
+  // KV tiles of C::BN keys: up to the last key below nk, and under the causal mask up to the
+  // last key the tile's last row sees
+  const int n_kv_all = (nk + C::BN - 1) / C::BN;
+  const int last_key = qt * 128 + 127 + koff;
+  const int n_kv = CAUSAL ? (last_key < 0 ? 0 : min(n_kv_all, last_key / C::BN + 1)) : n_kv_all;
+  const int row = threadIdx.x;                 // softmax threads: query row inside the tile, TMEM lane
+  const int grow = qt * 128 + row;             // query row in the sequence
+  OutT* const out = static_cast<OutT*>(p.out);
+  const long long orow = sv.q_in + (long long)grow * sv.q_tok + (long long)hq * sv.q_head;  // output row start
+  if (n_kv == 0) {
+    // no row of this tile sees a key (nk = 0, or the causal offset leaves the tile empty): zeros
+    if (warp < 4 && grow < nq)
+      for (int c = vh * DV; c < min(p.m.d, vh * DV + DV); ++c) store_elem(out + orow + c, 0.f);
+    return;
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
@@ -176,9 +193,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
-      const int q_row = (b * p.Hq + hq) * p.Np + qt * 128;
-      const int k_row = (b * p.Hkv + hkv) * p.Np;
-      const int v_row = (b * p.Hkv + hkv) * p.dp + vh * DV;
+      const int q_row = (int)(sv.q_row0 + (long long)hq * p.m.q_head_rows) + qt * 128;
+      const int k_row = (int)(sv.k_row0 + (long long)hkv * p.m.k_head_rows);
+      const int v_row = (int)(sv.v_row0 + (long long)hkv * p.m.dp) + vh * DV;
+      const int v_col = (int)sv.v_col0;
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int s = 0; s < C::NSUB; ++s) tma_load_2d(sQ + s * 128 * C::KSUB, &tmQ, &bars->q_full, s * C::KSUB, q_row);
       int issued = 0;
@@ -190,7 +208,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
           tma_load_2d(sK + st * C::K_BYTES + s * C::BN * C::KSUB, &tmK, &bars->k_full[st], s * C::KSUB,
                       k_row + j * C::BN);
         mbar_arrive_expect_tx(&bars->v_full[st], C::V_BYTES);
-        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], j * C::ROWB, v_row);  // x in bytes
+        tma_load_2d(sV + st * C::V_BYTES, &tmV, &bars->v_full[st], (v_col + j * C::BN) * C::PB, v_row);  // x in bytes
         issued = j + 1;
       }
       // make sure no copy is still landing in shared memory when the CTA exits
@@ -276,13 +294,11 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (slot) __nanosleep(slot * (600u / C::CTAS_PER_SM));
     }
-    const int row = warp * 32 + lane;            // query row inside the tile, TMEM lane
-    const int grow = qt * 128 + row;             // query row in the sequence
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t scol = tmem + lane_base + C::S_COL;
     const uint32_t ocol = tmem + lane_base + C::O_COL;
-    const float qsv = p.qs[((size_t)b * p.Hq + hq) * p.nblk + qt];
-    const float* ksp = p.ks + ((size_t)b * p.Hkv + hkv) * p.nblk;
+    const float qsv = p.qs[(sv.q_row0 + (long long)hq * p.m.q_head_rows) / 128 + qt];
+    const float* ksp = p.ks + (sv.k_row0 + (long long)hkv * p.m.k_head_rows) / 128;
     unsigned char* prow = sP + row * C::ROWB;
     float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates the stored P values' scale
     bool ok = true;
@@ -303,11 +319,11 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       // dequantization factor in the log2 domain
       const float f = __fmul_rn(__fmul_rn(qsv, ksp[i * BN / 128]), p.scale_log2);  // K scale of the 128-key block
       const int key0 = i * BN;
-      const bool edge = (key0 + BN > p.N) || (CAUSAL && key0 + BN - 1 > qt * 128);
-      int lim = BN;  // this row sees the tile's columns c < lim
+      const bool edge = (key0 + BN > nk) || (CAUSAL && key0 + BN - 1 > qt * 128 + koff);
+      int lim = BN;  // this row sees the tile's columns c < lim (none if lim <= 0)
       if (edge) {
-        lim = min(p.N - key0, BN);
-        if (CAUSAL) lim = min(lim, grow - key0 + 1);
+        lim = min(nk - key0, BN);
+        if (CAUSAL) lim = min(lim, grow + koff - key0 + 1);
 #pragma unroll
         for (int c = 0; c < BN; ++c)
           if (c >= lim) s[c] = (uint32_t)INT_MIN;
@@ -440,22 +456,19 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       if (ok) tc_fence_after();
     }
     if (ok) {
-      const float inv_l = __fdiv_rn(1.f, l);
-      const float* vsp = p.vs + ((size_t)b * p.Hkv + hkv) * p.dp + vh * DV;
-      OutT* out = static_cast<OutT*>(p.out);
-      const size_t orow = (p.layout == SAGE_HND) ? (((size_t)b * p.Hq + hq) * p.N + grow) * p.d
-                                                 : (((size_t)b * p.N + grow) * p.Hq + hq) * p.d;
+      const float inv_l = l > 0.f ? __fdiv_rn(1.f, l) : 0.f;  // a row that saw no key outputs zeros
+      const float* vsp = p.vs + ((size_t)b * p.m.Hkv + hkv) * p.m.dp + vh * DV;
 #pragma unroll 1
       for (int cc = 0; cc < DV / 32; ++cc) {
         uint32_t o[32];
         float of[32];
         tmem_ld32(ocol + cc * 32, o);
         tmem_wait_ld();
-        if (grow < p.N) {
+        if (grow < nq) {
           const int c0 = vh * DV + cc * 32;
 #pragma unroll
           for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(o[e]) * (vsp[cc * 32 + e] * inv_l);
-          if (c0 + 32 <= p.d && p.vec_out) {
+          if (c0 + 32 <= p.m.d && p.vec_out) {
             uint32_t w[16];
 #pragma unroll
             for (int e = 0; e < 16; ++e) w[e] = pack2<OutT>(of[2 * e], of[2 * e + 1]);
@@ -465,7 +478,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (c0 + e < p.d) store_elem(out + orow + c0 + e, of[e]);
+              if (c0 + e < p.m.d) store_elem(out + orow + c0 + e, of[e]);
           }
         }
       }
@@ -592,7 +605,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   static std::atomic<unsigned long long> attr_done{0};
   cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nblk, p.Hq * p.n_vhalves, p.B);
+  dim3 grid(p.nblk_q, p.m.Hq * p.n_vhalves, p.m.B);
   kern<<<grid, 192, C::SMEM, st>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
@@ -618,7 +631,7 @@ static cudaError_t launch_fwd_d(const CUtensorMap& tq, const CUtensorMap& tk, co
 template <typename OutT>
 static cudaError_t launch_fwd_o(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, int causal, int mode, cudaStream_t st) {
-  switch (p.dp) {
+  switch (p.m.dp) {
     case 64: return launch_fwd_d<64, 64, OutT>(tq, tk, tv, p, causal, mode, st);
     case 128: return launch_fwd_d<128, 128, OutT>(tq, tk, tv, p, causal, mode, st);
     case 256: return launch_fwd_d<256, 128, OutT>(tq, tk, tv, p, causal, mode, st);
@@ -630,6 +643,64 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
                        int dtype, int causal, int pv_mode, cudaStream_t st) {
   return dtype == SAGE_BF16 ? launch_fwd_o<__nv_bfloat16>(tq, tk, tv, p, causal, pv_mode, st)
                             : launch_fwd_o<__half>(tq, tk, tv, p, causal, pv_mode, st);
+}
+
+// ------------------------------------------------------------------------------------------------
+// Packed (varlen) batches: per-sequence table from the cumulative lengths.  One CTA: each thread
+// takes a run of consecutive sequences, a block scan gives every run its first padded row.
+// A table that is not non-decreasing from >= 0, exceeds the stated maxima or runs past the
+// stated totals flags SAGE_DEVERR_BAD_ARG and leaves every sequence empty, so no later kernel
+// reads outside the caller's tensors.
+// ------------------------------------------------------------------------------------------------
+__global__ void __launch_bounds__(1024) seq_plan_kernel(const int32_t* __restrict__ cu_q,
+                                                        const int32_t* __restrict__ cu_k, int B, int max_q, int max_k,
+                                                        long long total_q, long long total_k, SeqDesc* seqs) {
+  __shared__ long long scan_q[1024], scan_k[1024];
+  __shared__ int bad;
+  const int t = threadIdx.x, per = (B + 1023) / 1024;
+  const int b0 = min(B, t * per), b1 = min(B, b0 + per);
+  if (t == 0) bad = 0;
+  __syncthreads();
+  auto pad128 = [](long long n) { return n > 0 ? (n + 127) / 128 * 128 : 0ll; };
+  long long run_q = 0, run_k = 0;
+  bool my_bad = false;
+  for (int b = b0; b < b1; ++b) {
+    const long long q0 = cu_q[b], q1 = cu_q[b + 1], k0 = cu_k[b], k1 = cu_k[b + 1];
+    if (q0 < 0 || k0 < 0 || q1 < q0 || k1 < k0 || q1 - q0 > max_q || k1 - k0 > max_k || q1 > total_q ||
+        k1 > total_k)
+      my_bad = true;
+    run_q += pad128(q1 - q0);
+    run_k += pad128(k1 - k0);
+  }
+  if (my_bad) atomicOr(&bad, 1);
+  scan_q[t] = run_q, scan_k[t] = run_k;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan of the runs' padded lengths
+    const long long vq = t >= o ? scan_q[t - o] : 0, vk = t >= o ? scan_k[t - o] : 0;
+    __syncthreads();
+    scan_q[t] += vq, scan_k[t] += vk;
+    __syncthreads();
+  }
+  const bool any_bad = bad != 0;
+  if (t == 0 && any_bad) atomicOr(&g_device_error, SAGE_DEVERR_BAD_ARG);
+  long long row_q = scan_q[t] - run_q, row_k = scan_k[t] - run_k;  // first padded row of this run
+  for (int b = b0; b < b1; ++b) {
+    SeqDesc d{0, 0, 0, 0, 0, 0};
+    if (!any_bad) {
+      const long long q0 = cu_q[b], k0 = cu_k[b];
+      d.nq = (int)(cu_q[b + 1] - q0), d.nk = (int)(cu_k[b + 1] - k0);
+      d.q_row = (int)row_q, d.k_row = (int)row_k;
+      d.q_tok = q0, d.k_tok = k0;
+      row_q += pad128(d.nq), row_k += pad128(d.nk);
+    }
+    seqs[b] = d;
+  }
+}
+
+cudaError_t launch_seq_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int max_q, int max_k,
+                            long long total_q, long long total_k, SeqDesc* seqs, cudaStream_t st) {
+  seq_plan_kernel<<<1, 1024, 0, st>>>(cu_q, cu_k, B, max_q, max_k, total_q, total_k, seqs);
+  return cudaGetLastError();
 }
 
 cudaError_t read_clear_device_error(int* value) {

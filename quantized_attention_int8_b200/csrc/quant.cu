@@ -91,19 +91,18 @@ __device__ __forceinline__ TileCoord tile_coord(int dp) {
   return TileCoord{(int)threadIdx.x / nv, (int)threadIdx.x % nv, ((int)threadIdx.x % nv) * 8};
 }
 
-// Load this thread's 16 x 8 register tile of one head: tokens n0+16g+r (r < 16), channels c0..c0+7.
-// Tokens >= n0+rows and channels >= d read as zero.
+// Load this thread's 16 x 8 register tile of one head: tokens 16g+r (r < 16) of the block that
+// starts at x0 (tokens tok_stride elements apart), channels c0..c0+7.  Tokens >= rows and
+// channels >= d read as zero.
 template <typename T>
-__device__ __forceinline__ void load_tile(uint4 (&v)[16], const T* __restrict__ x, int b, int h, int H, int N, int d,
-                                          int n0, int rows, int layout, bool vec, const TileCoord& tc) {
-  const size_t hstride = (layout == SAGE_HND) ? (size_t)d : (size_t)H * d;  // elements between tokens
-  const size_t base = (layout == SAGE_HND) ? ((size_t)(b * H + h) * N + n0) * d : ((size_t)b * N + n0) * H * d + (size_t)h * d;
+__device__ __forceinline__ void load_tile(uint4 (&v)[16], const T* __restrict__ x0, long long tok_stride, int d,
+                                          int rows, bool vec, const TileCoord& tc) {
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     const int n = tc.g * 16 + r;
     v[r] = make_uint4(0, 0, 0, 0);
     if (n < rows && tc.c0 < d) {
-      const T* src = x + base + (size_t)n * hstride + tc.c0;
+      const T* src = x0 + (size_t)n * tok_stride + tc.c0;
       if (vec) {
         v[r] = __ldg(reinterpret_cast<const uint4*>(src));
       } else {
@@ -169,21 +168,26 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
   __shared__ float red[8];
   __shared__ float part[8 * 256];
   const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
-  const int n0 = blk * 128, rows = min(128, p.N - n0);
-  const int dp = p.dp, d = p.d;
+  const SeqView sv = seq_view(p.m, b);
+  const int n0 = blk * 128;
+  const int rows = min(128, (y < p.m.Hq ? sv.nq : sv.nk) - n0);
+  if (rows <= 0) return;  // past the end of this sequence (the whole CTA leaves)
+  const int dp = p.m.dp, d = p.m.d;
   const TileCoord tc = tile_coord(dp);
   uint4 v[16];
-  if (y < p.Hq) {  // ---- Q: final INT8 codes and per-block scale
+  if (y < p.m.Hq) {  // ---- Q: final INT8 codes and per-block scale
     const int h = y;
-    load_tile<T>(v, static_cast<const T*>(p.q), b, h, p.Hq, p.N, d, n0, rows, p.layout, p.vec_q, tc);
+    load_tile<T>(v, static_cast<const T*>(p.q) + sv.q_in + h * sv.q_head + n0 * sv.q_tok, sv.q_tok, d, rows, p.vec_q,
+                 tc);
     const float am = block_max(tile_absmax<T>(v), red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
-    const size_t bh = (size_t)b * p.Hq + h;
-    store_int8_tile(p.q8 + (bh * p.Np + n0) * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); });
-    if (threadIdx.x == 0) p.qs[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
-  } else if (y < p.Hq + p.Hkv) {  // ---- K: per-block partial column sums
-    const int h = y - p.Hq;
-    load_tile<T>(v, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_k, tc);
+    const long long row = sv.q_row0 + h * p.m.q_head_rows + n0;
+    store_int8_tile(p.q8 + row * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); });
+    if (threadIdx.x == 0) p.qs[row / 128] = __fdiv_rn(am, 127.f);
+  } else if (y < p.m.Hq + p.m.Hkv) {  // ---- K: per-block partial column sums
+    const int h = y - p.m.Hq;
+    load_tile<T>(v, static_cast<const T*>(p.k) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_k,
+                 tc);
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -195,11 +199,12 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = acc[e];
     __syncthreads();
-    const size_t base = (((size_t)b * p.Hkv + h) * p.nblk + blk) * dp;
+    const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
     p.ksum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
   } else {  // ---- V: per-block partial column amax
-    const int h = y - p.Hq - p.Hkv;
-    load_tile<T>(v, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_v, tc);
+    const int h = y - p.m.Hq - p.m.Hkv;
+    load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
+                 tc);
     uint32_t a[4] = {0, 0, 0, 0};  // channels (2e, 2e+1), |x| as bit patterns
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
@@ -214,25 +219,28 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
       part[tc.g * dp + tc.c0 + 2 * e + 1] = bits_to_f32<T>(a[e] >> 16);
     }
     __syncthreads();
-    const size_t base = (((size_t)b * p.Hkv + h) * p.nblk + blk) * dp;
+    const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
     p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
   }
 }
 
 __global__ void quant_finalize_kernel(QuantParams p) {
-  const int bh = blockIdx.x;
-  for (int c = threadIdx.x; c < p.dp; c += blockDim.x) {
-    const float* ks = p.ksum_part + (size_t)bh * p.nblk * p.dp + c;
-    const float* vm = p.vmax_part + (size_t)bh * p.nblk * p.dp + c;
+  const int bh = blockIdx.x, b = bh / p.m.Hkv, h = bh - b * p.m.Hkv;
+  const SeqView sv = seq_view(p.m, b);
+  const int dp = p.m.dp, nblk = (sv.nk + 127) / 128;
+  const long long base = (sv.k_row0 + h * p.m.k_head_rows) / 128 * dp;
+  for (int c = threadIdx.x; c < dp; c += blockDim.x) {
+    const float* ks = p.ksum_part + base + c;
+    const float* vm = p.vmax_part + base + c;
     float acc = 0.f, am = 0.f;
 #pragma unroll 8
-    for (int i = 0; i < p.nblk; ++i) {  // sums stay in block order; the loads overlap
-      acc = __fadd_rn(acc, ks[(size_t)i * p.dp]);
-      am = fmaxf(am, vm[(size_t)i * p.dp]);
+    for (int i = 0; i < nblk; ++i) {  // sums stay in block order; the loads overlap
+      acc = __fadd_rn(acc, ks[(size_t)i * dp]);
+      am = fmaxf(am, vm[(size_t)i * dp]);
     }
-    p.km[(size_t)bh * p.dp + c] = c < p.d ? __fdiv_rn(acc, (float)p.N) : 0.f;
-    p.vs[(size_t)bh * p.dp + c] = __fdiv_rn(am, p.vmax_code);
-    p.vinv[(size_t)bh * p.dp + c] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
+    p.km[(size_t)bh * dp + c] = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(acc, (float)sv.nk) : 0.f;
+    p.vs[(size_t)bh * dp + c] = __fdiv_rn(am, p.vmax_code);
+    p.vinv[(size_t)bh * dp + c] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
   }
 }
 
@@ -245,17 +253,20 @@ template <typename T>
 __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
   __shared__ float red[8];
   const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
-  const int n0 = blk * 128, rows = min(128, p.N - n0);
-  const int dp = p.dp, d = p.d;
+  const SeqView sv = seq_view(p.m, b);
+  const int n0 = blk * 128, rows = min(128, sv.nk - n0);
+  if (rows <= 0) return;  // past the end of this sequence (the whole CTA leaves)
+  const int dp = p.m.dp, d = p.m.d;
   const TileCoord tc = tile_coord(dp);
   uint4 v[16];
-  if (y < p.Hkv) {  // ---- K - mean(K): INT8 codes and per-block scale
+  if (y < p.m.Hkv) {  // ---- K - mean(K): INT8 codes and per-block scale
     const int h = y;
-    const size_t bh = (size_t)b * p.Hkv + h;
+    const size_t bh = (size_t)b * p.m.Hkv + h;
     float km[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) km[e] = p.km[bh * dp + tc.c0 + e];
-    load_tile<T>(v, static_cast<const T*>(p.k), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_k, tc);
+    load_tile<T>(v, static_cast<const T*>(p.k) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_k,
+                 tc);
     // padded channels read 0 and have mean 0; padded rows are masked by store_int8_tile
     auto x = [&](int r, int e) -> float { return __fsub_rn(elem<T>(v[r], e), km[e]); };
     // max |k - mean| per channel is reached at the channel's largest or smallest k, since
@@ -292,15 +303,21 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
     }
     am = block_max(am, red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
-    store_int8_tile(p.k8 + (bh * p.Np + n0) * dp, dp, tc, inv, rows, x);
-    if (threadIdx.x == 0) p.ks[bh * p.nblk + blk] = __fdiv_rn(am, 127.f);
+    const long long row = sv.k_row0 + h * p.m.k_head_rows + n0;
+    store_int8_tile(p.k8 + row * dp, dp, tc, inv, rows, x);
+    if (threadIdx.x == 0) p.ks[row / 128] = __fdiv_rn(am, 127.f);
   } else {  // ---- V: E4M3 or fp16 codes, transposed to [channel][token]
-    const int h = y - p.Hkv;
-    const size_t bh = (size_t)b * p.Hkv + h;
+    const int h = y - p.m.Hkv;
+    const size_t bh = (size_t)b * p.m.Hkv + h;
     float inv[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) inv[e] = p.vinv[bh * dp + tc.c0 + e];
-    load_tile<T>(v, static_cast<const T*>(p.v), b, h, p.Hkv, p.N, d, n0, rows, p.layout, p.vec_v, tc);
+    load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
+                 tc);
+    // V^T element (channel c, token t) of this sequence and head: row v_row0 + h*dp + c, column
+    // v_col0 + t, rows k_head_rows codes apart
+    const long long vrow = sv.v_row0 + (long long)h * dp + tc.c0, vcol = sv.v_col0 + n0 + tc.g * 16;
+    const long long pitch = p.m.k_head_rows;
     if (p.v_fp16) {
       // fp16_rne(v * inv): 16 tokens of one channel = 32 bytes (padded tokens and channels read 0)
       uint16_t* vt = reinterpret_cast<uint16_t*>(p.v8t);
@@ -313,7 +330,7 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
                                                __fmul_rn(elem<T>(v[2 * q + 1], e), inv[e]));
           w[q] = *reinterpret_cast<const uint32_t*>(&h2);
         }
-        uint4* dst = reinterpret_cast<uint4*>(vt + (bh * dp + tc.c0 + e) * p.Np + n0 + tc.g * 16);
+        uint4* dst = reinterpret_cast<uint4*>(vt + (vrow + e) * pitch + vcol);
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
@@ -330,7 +347,7 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
         const float a3 = __fmul_rn(elem<T>(v[4 * q + 3], e), inv[e]);
         w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
       }
-      *reinterpret_cast<uint4*>(p.v8t + (bh * dp + tc.c0 + e) * p.Np + n0 + tc.g * 16) =
+      *reinterpret_cast<uint4*>(p.v8t + (vrow + e) * pitch + vcol) =
           make_uint4(w[0], w[1], w[2], w[3]);
     }
   }
@@ -338,9 +355,10 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
 
 template <typename T>
 static cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
-  quant_pass1_kernel<T><<<dim3(p.nblk, p.Hq + 2 * p.Hkv, p.B), p.dp, 0, st>>>(p);
-  quant_finalize_kernel<<<p.B * p.Hkv, p.dp, 0, st>>>(p);
-  quant_pass2_kernel<T><<<dim3(p.nblk, 2 * p.Hkv, p.B), p.dp, 0, st>>>(p);
+  const int B = p.m.B, Hq = p.m.Hq, Hkv = p.m.Hkv, dp = p.m.dp;
+  quant_pass1_kernel<T><<<dim3(p.nblk_q > p.nblk_k ? p.nblk_q : p.nblk_k, Hq + 2 * Hkv, B), dp, 0, st>>>(p);
+  quant_finalize_kernel<<<B * Hkv, dp, 0, st>>>(p);
+  quant_pass2_kernel<T><<<dim3(p.nblk_k > 0 ? p.nblk_k : 1, 2 * Hkv, B), dp, 0, st>>>(p);
   return cudaGetLastError();
 }
 

@@ -51,11 +51,32 @@ class Workload:
                                   # 2 = FP16 operands, fp32; 3 = FP16 operands, fp16+fp32
     seed: int = 0
     sm_scale: float | None = None  # None -> 1/sqrt(d)
+    Nk: int | None = None          # key / value length when it differs from N (the query length)
+    varlen: tuple = ()             # packed batch: ((nq, nk), ...) per sequence; then B = len(varlen)
+
+    @property
+    def nk(self) -> int:
+        return self.N if self.Nk is None else self.Nk
+
+    def seqlens(self):
+        """[(nq, nk)] of every sequence."""
+        return list(self.varlen) if self.varlen else [(self.N, self.nk)] * self.B
 
     def ops(self) -> float:
-        """Algorithmic attention operations 4*B*Hq*N^2*d, halved under the causal mask."""
-        v = 4.0 * self.B * self.Hq * self.N * self.N * self.d
-        return v / 2 if self.causal else v
+        """Algorithmic attention operations: 4*Hq*d per visible (query, key) pair, i.e.
+        4*B*Hq*Nq*Nk*d, and under the (bottom-right) causal mask only the visible pairs."""
+        total = 0
+        for nq, nk in self.seqlens():
+            if self.causal:
+                # query i sees min(nk, max(0, i + nk - nq + 1)) keys
+                pairs = sum(min(nk, max(0, i + nk - nq + 1)) for i in range(nq)) if nq != nk else nq * (nq + 1) // 2
+            else:
+                pairs = nq * nk
+            total += pairs
+        v = 4.0 * self.Hq * self.d * total
+        if self.causal and not self.varlen and self.Nk is None:
+            v = 4.0 * self.B * self.Hq * self.N * self.N * self.d / 2  # the pages' convention: half of N^2
+        return v
 
     def with_(self, **kw) -> "Workload":
         return dataclasses.replace(self, **kw)
@@ -89,15 +110,15 @@ ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV
 BY_NAME = {w.name: w for w in ALL}
 
 
-def _gen(w: Workload, stream: int) -> torch.Generator:
-    # One independent, reproducible stream per (workload seed, shape, tensor).
+def _gen(w: Workload, stream: int, seq: int = 0) -> torch.Generator:
+    # One independent, reproducible stream per (workload seed, shape, tensor[, sequence]).
     key = (w.seed * 1_000_003 + stream * 7919 + w.N * 31 + w.d * 131 + w.B * 17 + w.Hq * 3
-           + w.Hkv * 5 + (1 if w.causal else 0))
+           + w.Hkv * 5 + (1 if w.causal else 0) + (w.Nk or 0) * 37 + seq * 104_729)
     return torch.Generator().manual_seed(key & 0x7FFF_FFFF_FFFF)
 
 
-def _draw(w: Workload, stream: int, shape) -> torch.Tensor:
-    g = _gen(w, stream)
+def _draw(w: Workload, stream: int, shape, seq: int = 0) -> torch.Tensor:
+    g = _gen(w, stream, seq)
     if w.dist == "uniform2":
         return torch.rand(shape, generator=g, dtype=torch.float32) * 4.0 - 2.0
     return torch.randn(shape, generator=g, dtype=torch.float32)
@@ -106,22 +127,12 @@ def _draw(w: Workload, stream: int, shape) -> torch.Tensor:
 def make_inputs(w: Workload):
     """Return (q, k, v) as contiguous CPU tensors of w.dtype in w.layout.
 
-    Logical shapes are (B, Hq, N, d) for q and (B, Hkv, N, d) for k, v; for
+    Logical shapes are (B, Hq, N, d) for q and (B, Hkv, Nk, d) for k, v; for
     the NHD layout the same logical tensors are stored as (B, N, H, d).
     """
-    if w.dist not in ("normal", "normal_koffset", "normal_koutlier", "uniform2"):
-        raise ValueError(f"unknown value recipe {w.dist!r}")
-    q = _draw(w, STREAM_Q, (w.B, w.Hq, w.N, w.d))
-    k = _draw(w, STREAM_K, (w.B, w.Hkv, w.N, w.d))
-    v = _draw(w, STREAM_V, (w.B, w.Hkv, w.N, w.d))
-    if w.dist == "normal_koffset":
-        off = torch.randn((w.d,), generator=_gen(w, STREAM_OFFSET), dtype=torch.float32) * 3.0
-        k += off
-    elif w.dist == "normal_koutlier":
-        n_out = max(1, round(0.01 * w.Hkv * w.d))
-        pick = torch.randperm(w.Hkv * w.d, generator=_gen(w, STREAM_OUTLIER))[:n_out]
-        for p in pick.tolist():
-            k[:, p // w.d, :, p % w.d] *= 8.0
+    if w.varlen:
+        raise ValueError("packed workloads: use make_varlen_inputs")
+    q, k, v = _logical(w, w.B, w.N, w.nk)
     dt = DTYPES[w.dtype]
     out = []
     for t in (q, k, v):
@@ -130,6 +141,42 @@ def make_inputs(w: Workload):
             t = t.transpose(1, 2)
         out.append(t.contiguous())
     return tuple(out)
+
+
+def _logical(w: Workload, B: int, nq: int, nk: int, seq: int = 0):
+    """float32 (B, Hq, nq, d), (B, Hkv, nk, d) x 2 of the workload's value recipe."""
+    if w.dist not in ("normal", "normal_koffset", "normal_koutlier", "uniform2"):
+        raise ValueError(f"unknown value recipe {w.dist!r}")
+    q = _draw(w, STREAM_Q, (B, w.Hq, nq, w.d), seq)
+    k = _draw(w, STREAM_K, (B, w.Hkv, nk, w.d), seq)
+    v = _draw(w, STREAM_V, (B, w.Hkv, nk, w.d), seq)
+    if w.dist == "normal_koffset":
+        off = torch.randn((w.d,), generator=_gen(w, STREAM_OFFSET), dtype=torch.float32) * 3.0
+        k += off
+    elif w.dist == "normal_koutlier":
+        n_out = max(1, round(0.01 * w.Hkv * w.d))
+        pick = torch.randperm(w.Hkv * w.d, generator=_gen(w, STREAM_OUTLIER))[:n_out]
+        for p in pick.tolist():
+            k[:, p // w.d, :, p % w.d] *= 8.0
+    return q, k, v
+
+
+def make_varlen_inputs(w: Workload):
+    """Packed batch of w.varlen's sequences: q (total_q, Hq, d), k and v (total_k, Hkv, d) of w.dtype
+    (sequence b's tokens after those of b - 1; each sequence drawn from its own streams, the K
+    offset / outlier channels shared), and cu_seqlens_q, cu_seqlens_k as int32 CPU tensors."""
+    qs, ks, vs = [], [], []
+    cq, ck = [0], [0]
+    dt = DTYPES[w.dtype]
+    for b, (nq, nk) in enumerate(w.varlen):
+        q, k, v = _logical(w, 1, nq, nk, seq=b)
+        qs.append(q[0].transpose(0, 1))
+        ks.append(k[0].transpose(0, 1))
+        vs.append(v[0].transpose(0, 1))
+        cq.append(cq[-1] + nq)
+        ck.append(ck[-1] + nk)
+    pack = lambda ts: torch.cat(ts, 0).to(dt).contiguous()
+    return (pack(qs), pack(ks), pack(vs), torch.tensor(cq, dtype=torch.int32), torch.tensor(ck, dtype=torch.int32))
 
 
 def sm_scale_of(w: Workload) -> float:
