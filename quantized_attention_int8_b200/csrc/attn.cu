@@ -120,7 +120,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 constexpr float kLog2_448 = 8.807354922057604f;  // p * 448 = 2^(log2 p + log2 448)
 constexpr float kTau = 2.0f;                       // reference-max slack of the online softmax (log2 units)
 
-template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16>
+template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16, bool PACKED>
 __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     sage_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -137,8 +137,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int b = blockIdx.z;
-  const SeqView sv = seq_view(p.m, b);
-  const int nq = sv.nq, nk = sv.nk;
+  // Dense batches are a separate instance: their lengths stay kernel parameters in the loop
+  // below (measured 12% faster at d = 64 than lengths held in registers).
+  const SeqView sv = seq_view<PACKED ? 1 : 0>(p.m, b);
+  const int nq = PACKED ? sv.nq : p.m.Nq, nk = PACKED ? sv.nk : p.m.Nk;
   const int nblk_q = (nq + 127) / 128;
   int qt = blockIdx.x;
   if (CAUSAL) qt = nblk_q - 1 - qt;  // longest rows first
@@ -601,8 +603,10 @@ template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, cudaStream_t st) {
   using C = FwdCfg<DQK, DV, PV16>;
-  auto kern = sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16>;
-  static std::atomic<unsigned long long> attr_done{0};
+  auto kern = p.m.seqs ? sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, true>
+                       : sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, false>;
+  static std::atomic<unsigned long long> attr_done_dense{0}, attr_done_packed{0};
+  std::atomic<unsigned long long>& attr_done = p.m.seqs ? attr_done_packed : attr_done_dense;
   cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nblk_q, p.m.Hq * p.n_vhalves, p.m.B);

@@ -43,9 +43,12 @@ struct SeqView {
   long long k_tok, k_head;   // element strides of k and v
 };
 
+// PACKED: 1 = the table, 0 = the dense formulas (lengths then stay kernel parameters), -1 = decide
+// at run time by m.seqs.
+template <int PACKED = -1>
 __host__ __device__ inline SeqView seq_view(const SeqMap& m, int b) {
   SeqView v;
-  if (m.seqs) {
+  if (PACKED == 1 || (PACKED == -1 && m.seqs)) {
     const SeqDesc s = m.seqs[b];
     v.nq = s.nq, v.nk = s.nk;
     v.q_row0 = s.q_row, v.k_row0 = s.k_row;
