@@ -14,7 +14,8 @@ sums; the pages fix neither):
 
 1. S = Q8 . K8^T exactly in integers (K8 holds codes of K - mean(K)).
 2. Dequantize in the log2 domain: s = S * f with
-   f = (qs * ks) * (sm_scale * log2(e)), all float32.  Keys j >= Nk, and
+   f = (qs * ks) * (sm_scale * log2(e)), all float32 (qs of the query row's
+   Q-scale group: its 128-, 32- or 1-token block).  Keys j >= Nk, and
    j > i + (Nk - Nq) under the (bottom-right aligned) causal mask, are
    excluded; a row that sees no key at all outputs zeros.
 3. Online softmax against a reference max m: the reference moves to
@@ -30,8 +31,9 @@ sums; the pages fix neither):
    modes 1 and 3 (fp16+fp32, "two-level accumulation") the tile's P . V is first
    rounded to float16 (a fresh fp16 accumulator per tile), then
    O = O * alpha + T.
-6. out = O * vs / (P scale * l), P scale being 448 * 2^-tau (FP8) or 1 (FP16),
-   rounded to the output dtype by the caller.
+6. out = O * vs / (P scale * l) (+ vm, V's token mean, when V was smoothed),
+   P scale being 448 * 2^-tau (FP8) or 1 (FP16), rounded to the output dtype
+   by the caller.
 """
 from __future__ import annotations
 
@@ -79,6 +81,8 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
         for r, qb in enumerate(qbs):
             rows = qb * BLOCK + np.arange(BLOCK)
             q8 = qz["q8"][b, h, qb * BLOCK:(qb + 1) * BLOCK].astype(np.int64)
+            qg = qz.get("q_gran", BLOCK)
+            qsr = qz["qs"][b, h, rows // qg].astype(F32)           # Q scale of every row
             m = np.full(BLOCK, -np.inf, F32)
             l = np.zeros(BLOCK, F32)
             O = np.zeros((BLOCK, qz["dp"]), F32)
@@ -94,7 +98,7 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
                 valid = (keys[None, :] < Nk) & np.ones((BLOCK, 1), bool)
                 if causal:
                     valid &= keys[None, :] <= rows[:, None] + off
-                f = F32(F32(qz["qs"][b, h, qb]) * F32(qz["ks"][b, hk, keys[0] // BLOCK])) * c
+                f = ((qsr * F32(qz["ks"][b, hk, keys[0] // BLOCK])).astype(F32) * c).astype(F32)  # (BLOCK,)
                 smax = np.where(valid, S, np.iinfo(np.int64).min).max(axis=1)
                 has = valid.any(axis=1)
                 tmax = np.where(has, smax.astype(F32) * f, F32(-np.inf)).astype(F32)
@@ -102,7 +106,8 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
                 upd = mc > (m + F32(tau)).astype(F32)             # the reference max moves
                 m_new = np.where(upd, mc, m).astype(F32)
                 with np.errstate(invalid="ignore"):
-                    arg = (S.astype(np.float64) * np.float64(f) - m_new[:, None].astype(np.float64)).astype(F32)
+                    arg = (S.astype(np.float64) * f[:, None].astype(np.float64)
+                           - m_new[:, None].astype(np.float64)).astype(F32)
                 p = np.where(valid, np.exp2(arg), F32(0)).astype(F32)
                 with np.errstate(invalid="ignore"):
                     alpha = np.where(np.isneginf(m), F32(0), np.exp2((m - m_new).astype(F32))).astype(F32)
@@ -121,6 +126,8 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
             with np.errstate(divide="ignore", invalid="ignore"):
                 o = (O * vs[None, :] / (pscale * l[:, None])).astype(F32)
             o[l == 0] = 0.0                                   # rows that saw no key
+            if qz.get("smooth_v"):
+                o = np.where((l > 0)[:, None], (o + qz["vm"][b, hk][None, :]).astype(F32), o)
             ok = rows < N
             out[n, r * BLOCK:(r + 1) * BLOCK][ok] = o[ok, :d]
     return out

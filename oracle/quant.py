@@ -35,6 +35,16 @@ choice a reader can check here, and the CUDA path implements the same one):
 * For the FP16 P.V variant (README "Available APIs": sageattn_qk_int8_pv_fp16_cuda)
   V is kept in fp16 with the same per-channel scaling to [-1, 1]: inv = 1 / amax,
   code = fp16_rne(v * inv), scale = amax.  (Q and K are quantized as above.)
+* "Varying granularities" for Q (README "Current Features"; "per-thread
+  quantization", news of 2024-12-20): Q may take one scale per 128 tokens
+  (per block, the default), per 32 tokens (per warp: the rows one warp of the
+  CUDA kernel owns) or per token (per thread: one thread of the kernel owns
+  one query row).  The codes and scales follow the INT8 rule above with the
+  block of that many tokens.  K keeps one scale per 128-token block.
+* Optional V smoothing (the "thorough outlier smoothing" of the SageAttention2
+  title): V - mean_tokens(V) is coded instead of V, the mean summed in the same
+  fixed order as K's, and the mean is added back to the output (each row of
+  softmax weights sums to 1, so the result is unchanged in exact arithmetic).
 * All float arithmetic is IEEE float32 with round-to-nearest-even and no
   fused multiply-add; numpy float32 operations satisfy this.
 """
@@ -108,16 +118,17 @@ def k_token_mean(k: np.ndarray) -> np.ndarray:
     return total / F32(N)
 
 
-def int8_per_block(x: np.ndarray, dp: int):
-    """Symmetric per-(b, h, 128-token block) INT8 codes of x (float32 (B,H,N,d)).
+def int8_per_block(x: np.ndarray, dp: int, rows: int = BLOCK):
+    """Symmetric INT8 codes of x (float32 (B,H,N,d)) with one scale per (b, h, block of
+    ``rows`` tokens) (128: per block; 32: per warp; 1: per token).
 
-    Returns codes int8 (B, H, N_pad, dp) and scales float32 (B, H, nblocks).
+    Returns codes int8 (B, H, N_pad, dp) and scales float32 (B, H, N_pad / rows).
     """
     B, H, N, d = x.shape
     nb = n_blocks(N)
     xp = np.zeros((B, H, nb * BLOCK, dp), F32)
     xp[:, :, :N, :d] = x                               # padding is exact zeros
-    xb = xp.reshape(B, H, nb, BLOCK, dp)
+    xb = xp.reshape(B, H, nb * BLOCK // rows, rows, dp)
     amax = np.abs(xb).max(axis=(3, 4))                 # zeros cannot raise the max
     with np.errstate(divide="ignore"):
         inv = np.where(amax > 0, F32(127.0) / amax, F32(0.0)).astype(F32)
@@ -164,7 +175,10 @@ def fp16_per_channel(v: np.ndarray, dp: int):
     return codes, amax.copy()
 
 
-def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
+Q_GRANS = (128, 32, 1)   # query tokens per Q scale: per block, per warp, per thread
+
+
+def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0, q_gran: int = BLOCK, smooth_v: bool = False) -> dict:
     """The whole quantization step for one attention call.
 
     q: (B, Hq, Nq, d), k and v: (B, Hkv, Nk, d) in ``layout`` (fp16/bf16 torch
@@ -173,23 +187,33 @@ def quantize(q, k, v, layout: str = "HND", pv_mode: int = 0) -> dict:
       ks f32 (B,Hkv,nbk), km f32 (B,Hkv,dp), v8 (B,Hkv,Nk_pad,dp) V codes (uint8 E4M3
       for PV modes 0/1, float16 for the FP16 P.V modes 2/3), vs f32 (B,Hkv,dp),
       plus the sizes (N = Nq, Nk).  Q and K are quantized on their own lengths.
+    q_gran: query tokens per Q scale (qs then has Nq_pad / q_gran entries per head).
+    smooth_v: code V - vm (vm f32 (B,Hkv,dp), the token mean; zeros when off).
     """
+    if q_gran not in Q_GRANS:
+        raise ValueError(f"q_gran must be one of {Q_GRANS}")
     qf, kf, vf = (to_hnd(t, layout) for t in (q, k, v))
     B, Hq, N, d = qf.shape
     Hkv = kf.shape[1]
     dp = padded_dim(d)
     km = k_token_mean(kf)
     ksm = (kf - km[:, :, None, :]).astype(F32)        # one float32 subtraction
-    q8, qs = int8_per_block(qf, dp)
+    q8, qs = int8_per_block(qf, dp, q_gran)
     k8, ks = int8_per_block(ksm, dp)
+    vm = np.zeros((B, Hkv, dp), F32)
+    if smooth_v:
+        vmean = k_token_mean(vf)                      # same fixed summation order as K's mean
+        vm[:, :, :d] = vmean
+        vf = (vf - vmean[:, :, None, :]).astype(F32)  # one float32 subtraction
     if pv_mode in PV_FP16:
         v8, vs = fp16_per_channel(vf, dp)      # "v8" holds the fp16 codes in these modes
     else:
         v8, vs = fp8_per_channel(vf, dp, VMAX[pv_mode])
     kmp = np.zeros((B, Hkv, dp), F32)
     kmp[:, :, :d] = km
-    return dict(q8=q8, qs=qs, k8=k8, ks=ks, km=kmp, v8=v8, vs=vs,
-                B=B, Hq=Hq, Hkv=Hkv, N=N, Nk=kf.shape[2], d=d, dp=dp, pv_mode=pv_mode)
+    return dict(q8=q8, qs=qs, k8=k8, ks=ks, km=kmp, v8=v8, vs=vs, vm=vm,
+                B=B, Hq=Hq, Hkv=Hkv, N=N, Nk=kf.shape[2], d=d, dp=dp, pv_mode=pv_mode, q_gran=q_gran,
+                smooth_v=bool(smooth_v))
 
 
 def qk_int32(q8: np.ndarray, k8: np.ndarray) -> np.ndarray:

@@ -283,3 +283,49 @@ def test_emulation_rectangular_closed_forms(mode):
             em = emulate.emulate(qz, causal, 0.125).reshape(1, 2, -1, 64)[:, :, :nq].astype(np.float64)
             ex = attention.attention_f64(qr, kr, vr, "HND", causal, 0.125)
             assert (em * ex).sum() / np.sqrt((em ** 2).sum() * (ex ** 2).sum()) >= 0.999
+
+
+def test_v_smoothing_identity_in_exact_attention():
+    # softmax rows sum to one: attention(V - mu) + mu = attention(V) for any per-channel mu
+    w = W.TINY.with_(N=90, d=12, Hq=4, Hkv=2)
+    q, k, v = (t.double().numpy() for t in W.make_inputs(w))
+    # the oracle widens its inputs through float32, so v - mu carries one float32 rounding
+    # (<= 2^-24 * 32 for |mu| < 16): the identity holds to that
+    mu = np.round(np.random.default_rng(22).standard_normal((1, 2, 1, 12)) * 5 * 16) / 16
+    for causal in (False, True):
+        a = attention.attention_f64(q, k, v, "HND", causal, 0.3)
+        b = attention.attention_f64(q, k, v - mu, "HND", causal, 0.3) + np.repeat(mu, 2, axis=1)
+        assert np.allclose(a, b, rtol=0, atol=2e-6)
+
+
+def test_emulation_v_smoothing_and_q_granularity():
+    rng = np.random.default_rng(23)
+    # V with large per-channel offsets: smoothing must not change the result beyond rounding, and
+    # must shrink the error of the FP8 codes
+    w = W.TINY.with_(N=384, d=64)
+    q, k, v = W.make_inputs(w)
+    v = (v.float() + torch.from_numpy(rng.standard_normal(64).astype(np.float32) * 20)).half()
+    ref = attention.attention_f64(q, k, v, "HND", False, 0.125)
+    errs = {}
+    for sv in (False, True):
+        for mode in (0, 2):
+            qz = quant.quantize(q, k, v, "HND", mode, smooth_v=sv)
+            em = emulate.emulate(qz, False, 0.125).reshape(1, 2, -1, 64)[:, :, :384].astype(np.float64)
+            errs[(sv, mode)] = np.abs(em - ref).max() / np.abs(ref).max()
+    # FP8 codes gain most (measured 54x smaller error); fp16 codes already carry the offset
+    assert errs[(True, 0)] < 0.25 * errs[(False, 0)] and errs[(True, 2)] < 1.1 * errs[(False, 2)]
+    # V constant over tokens: smoothed codes carry ~nothing, the output is the mean itself
+    vc = torch.from_numpy(np.broadcast_to(rng.standard_normal(64).astype(np.float32), (1, 2, 384, 64)).copy()).half()
+    qz = quant.quantize(q, k, vc, "HND", 0, smooth_v=True)
+    em = emulate.emulate(qz, True, 0.125).reshape(1, 2, -1, 64)[:, :, :384]
+    assert np.allclose(em, vc.float().numpy(), rtol=1e-5, atol=1e-5)
+    # Q rows of very different magnitude: per-token scales track exact attention at least as well
+    qv = (q.float() * torch.from_numpy(np.exp(rng.uniform(-4, 1, (1, 2, 384, 1))).astype(np.float32))).half()
+    ref = attention.attention_f64(qv, k, v, "HND", True, 0.125)
+    cos = {}
+    for g in quant.Q_GRANS:
+        qz = quant.quantize(qv, k, v, "HND", 2, q_gran=g, smooth_v=True)
+        em = emulate.emulate(qz, True, 0.125).reshape(1, 2, -1, 64)[:, :, :384].astype(np.float64)
+        cos[g] = float((em * ref).sum() / np.sqrt((em ** 2).sum() * (ref ** 2).sum()))
+        assert cos[g] >= 0.999
+    assert cos[1] >= cos[32] - 1e-6 and cos[32] >= cos[128] - 1e-6

@@ -156,3 +156,39 @@ def test_quantize_layouts_agree():
                        v.transpose(1, 2).contiguous(), "NHD")
     for key in ("q8", "qs", "k8", "ks", "km", "v8", "vs"):
         assert np.array_equal(a[key], b[key]), key
+
+
+@pytest.mark.parametrize("rows", [32, 1])
+def test_int8_finer_granularity_brute_force(rows):
+    # one scale per `rows` tokens: brute force per group with python max / division
+    rng = np.random.default_rng(21)
+    x = (rng.standard_normal((1, 2, 70, 5)) * np.exp(rng.uniform(-3, 3, (1, 2, 70, 1)))).astype(np.float32)
+    codes, scale = quant.int8_per_block(x, 64, rows)
+    assert codes.shape == (1, 2, 128, 64) and scale.shape == (1, 2, 128 // rows)
+    for h in range(2):
+        for g in range(128 // rows):
+            blk = x[0, h, g * rows:(g + 1) * rows]
+            am = float(np.max(np.abs(blk))) if blk.size else 0.0
+            assert scale[0, h, g] == np.float32(np.float32(am) / np.float32(127.0))
+            if am > 0:
+                inv = np.float32(np.float32(127.0) / np.float32(am))
+                ref = np.clip(np.rint((blk * inv).astype(np.float32)), -127, 127)
+                assert np.array_equal(codes[0, h, g * rows:g * rows + len(blk), :5], ref)
+    # the 128-token default is the same function
+    c128, s128 = quant.int8_per_block(x, 64)
+    c128b, s128b = quant.int8_per_block(x, 64, 128)
+    assert np.array_equal(c128, c128b) and np.array_equal(s128, s128b)
+
+
+def test_quantize_options_validate_and_record():
+    w = W.TINY.with_(N=40, d=16)
+    q, k, v = W.make_inputs(w)
+    qz = quant.quantize(q, k, v, "HND", 0, q_gran=32, smooth_v=True)
+    assert qz["qs"].shape == (1, 2, 4) and qz["q_gran"] == 32 and qz["smooth_v"]
+    # the V mean is the same fixed-order mean as K's, and V - mean is what gets coded
+    vm = quant.k_token_mean(quant.to_hnd(v, "HND"))
+    assert np.array_equal(qz["vm"][:, :, :16], vm) and np.all(qz["vm"][:, :, 16:] == 0)
+    ref = quant.quantize(q, k, (v.float() - torch.from_numpy(vm)[:, :, None, :]).numpy(), "HND", 0)
+    assert np.array_equal(qz["v8"], ref["v8"]) and np.array_equal(qz["vs"], ref["vs"])
+    with pytest.raises(ValueError):
+        quant.quantize(q, k, v, "HND", 0, q_gran=64)
