@@ -26,6 +26,7 @@ rank, no collective on the data path (weak scaling).
 from __future__ import annotations
 
 import argparse
+import ctypes
 import json
 import os
 import statistics
@@ -220,6 +221,7 @@ def _config(w):
     return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d, "io_dtype": w.dtype,
             "layout": w.layout, "causal": w.causal, "pv_dtype": "fp16" if w.pv_mode & 2 else "fp8",
             "pv_accum": "fp16+fp32" if w.pv_mode & 1 else "fp32",
+            "qk_quant_gran": {128: "per_block", 32: "per_warp", 1: "per_thread"}[w.q_gran], "smooth_v": w.smooth_v,
             "values": w.dist, "l2": "flushed between steps (256 MiB write outside the events)"}
 
 
@@ -238,6 +240,7 @@ def run_ours(args, w):
         raise SystemExit("this device is not a B200 (compute capability 10.0)")
     pv = "fp16+fp32" if w.pv_mode & 1 else "fp32"
     pvd = "fp16" if w.pv_mode & 2 else "fp8"
+    okw = dict(qk_quant_gran={128: "per_block", 32: "per_warp", 1: "per_thread"}[w.q_gran], smooth_v=w.smooth_v)
     scale = W.sm_scale_of(w)
     q, k, v = W.make_inputs(w)
     in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
@@ -247,7 +250,7 @@ def run_ours(args, w):
     ops = w.ops()
 
     # ---- whole path (quantize + attention), device-resident inputs
-    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out, pv_dtype=pvd)
+    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out, pv_dtype=pvd, **okw)
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
@@ -257,7 +260,7 @@ def run_ours(args, w):
     value, total_ms = job_throughput(sum(times), ops, args.steps, dist, "cuda")
 
     # ---- the fused attention kernel alone (roofline)
-    z = qa.sage_quantize(qd, kd, vd, w.layout, pv, pvd)
+    z = qa.sage_quantize(qd, kd, vd, w.layout, pv, pvd, **okw)
     kern = lambda: qa.sage_attn_quantized(z, qd.dtype, w.layout, w.causal, scale, pv, out=out)
     ktimes = time_steps(kern, args.steps, args.warmup, flush)
     qa.sage_check_status()
@@ -277,10 +280,11 @@ def run_ours(args, w):
     # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element
     # (V: 2 B written in the FP16 P.V modes);
     # the C entry point on preallocated outputs, so the Python allocations are not timed
+    qopts = qa.opts(**okw)  # kept alive while qargs points at it
     qargs = [qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), w.B, w.Hq, w.Hkv, w.N, w.d,
              qa.SAGE_BF16 if qd.dtype == torch.bfloat16 else qa.SAGE_FP16,
-             qa.SAGE_HND if w.layout == "HND" else qa.SAGE_NHD, w.pv_mode,
-             *(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "km", "v8t", "vs")),
+             qa.SAGE_HND if w.layout == "HND" else qa.SAGE_NHD, w.pv_mode, ctypes.byref(qopts),
+             *(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "km", "v8t", "vs", "vm")),
              torch.cuda.current_stream().cuda_stream]
     qtimes = time_steps(lambda: qa.capi.sage_quantize(*qargs), max(3, args.steps // 2), 3, flush)
     q_ms = statistics.mean(qtimes)
@@ -294,7 +298,7 @@ def run_ours(args, w):
         a = qh.to("cuda", non_blocking=True)
         b = kh.to("cuda", non_blocking=True)
         c = vh.to("cuda", non_blocking=True)
-        o = qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv, pv_dtype=pvd)
+        o = qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv, pv_dtype=pvd, **okw)
         outh.copy_(o, non_blocking=True)
 
     etimes = time_steps(e2e_step, args.steps, args.warmup, flush)

@@ -78,6 +78,22 @@ typedef enum {
   SAGE_PV16_FP16_FP32 = 3
 } sage_pv_mode;
 
+/* Optional quantization settings (SageAttention README, "Current Features":
+ * INT8 quantization for Q K^T with varying granularities; news of 2024-12-20:
+ * per-thread quantization; the SageAttention2 title's outlier smoothing).
+ *   q_gran    query tokens per Q scale: 128 (per block, the default), 32 (per
+ *             warp: the rows one warp of the fused kernel owns) or 1 (per
+ *             thread: one thread of the fused kernel owns one query row);
+ *             0 selects 128.  K keeps one scale per 128-token block.
+ *   smooth_v  1: code V - mean_tokens(V) (the mean summed in the same fixed
+ *             order as K's) and add the mean back to the output (rows that
+ *             see no key stay 0).  0: code V itself.
+ * A NULL sage_opts pointer means {128, 0}. */
+typedef struct {
+  int q_gran;
+  int smooth_v;
+} sage_opts;
+
 /* Quantized attention, end to end: quantize/smooth pass, then the fused
  * attention kernel.  q: (B,Hq,N,d), k and v: (B,Hkv,N,d), out: (B,Hq,N,d), all
  * in `layout`, dtype `dtype`.  sm_scale <= 0 or NaN selects 1/sqrt(d) (the
@@ -96,10 +112,11 @@ sage_status sage_attn(const void* q, const void* k, const void* v, void* out, in
  * (B,Hq,Nq,d), k and v: (B,Hkv,Nk,d), in `layout`.  Under is_causal the mask is
  * aligned bottom-right: query i sees keys j <= i + (Nk - Nq), so the last query
  * sees every key; a query that sees no key (Nq > Nk) gets zeros.  Nq = Nk is
- * exactly sage_attn.  Workspace, errors and ownership as sage_attn. */
+ * exactly sage_attn (with opts NULL).  opts: see sage_opts.  Workspace, errors
+ * and ownership as sage_attn. */
 sage_status sage_attn_ex(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Nq,
                          int Nk, int d, sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale,
-                         sage_pv_mode pv_mode, void* stream);
+                         sage_pv_mode pv_mode, const sage_opts* opts, void* stream);
 
 /* Packed batch of sequences of different lengths (SageAttention README,
  * "Available APIs": sageattn_varlen).  q, out: (total_q, Hq, d); k, v:
@@ -118,7 +135,8 @@ sage_status sage_attn_ex(const void* q, const void* k, const void* v, void* out,
 sage_status sage_attn_varlen(const void* q, const void* k, const void* v, void* out, const int32_t* cu_seqlens_q,
                              const int32_t* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
                              long long total_q, long long total_k, int Hq, int Hkv, int d, sage_dtype dtype,
-                             int is_causal, float sm_scale, sage_pv_mode pv_mode, void* stream);
+                             int is_causal, float sm_scale, sage_pv_mode pv_mode, const sage_opts* opts,
+                             void* stream);
 
 /* Bytes of workspace sage_attn takes for these sizes, the largest over the P.V
  * modes (0 on invalid sizes). */
@@ -134,26 +152,31 @@ size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  *                                  bytes (SAGE_PV_FP32, SAGE_PV_FP16_FP32) or
  *                                  fp16 values, 2 bytes each (SAGE_PV16_*)
  *   vs  fp32   [B][Hkv][dp]
- * Padded tokens and channels hold code 0 (and km 0, vs 0).  Codes and scales
+ *   vm  fp32   [B][Hkv][dp]         V's token mean (zeros unless opts->smooth_v)
+ * qs holds Np / q_gran scales per (b, head) (opts->q_gran, 128 by default).
+ * Padded tokens and channels hold code 0 (and km 0, vs 0, vm 0).  Codes and scales
  * follow: amax over the block's real tokens and channels, inv = 127 / amax,
  * code = clamp(rint_even(x * inv), -127, 127), scale = amax / 127 (0 when amax
  * is 0); K is smoothed as x = k - km, km summed in fp32 block by block (tokens
  * in order inside a block, then the block sums in order) and divided by N;
  * V: inv = VMAX / amax_channel, code = E4M3_rne_satfinite(v * inv) (FP8 modes)
  * or fp16_rne(v * inv) (FP16 modes), vs = amax / VMAX with VMAX = 448
- * (SAGE_PV_FP32) or 1 (the other modes).
+ * (SAGE_PV_FP32) or 1 (the other modes); with smooth_v, v - vm in place of v
+ * (vm summed like km).  vm may be NULL when smooth_v is off.
  * Its own small scratch comes from the same per-device pool as sage_attn's. */
 sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
-                          sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,
-                          int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs, void* stream);
+                          sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, const sage_opts* opts,
+                          int8_t* q8, float* qs, int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs,
+                          float* vm, void* stream);
 
 /* The fused attention kernel alone, on buffers in the layouts sage_quantize
- * writes.  out: (B,Hq,N,d) in `out_layout`, dtype `out_dtype`.  Allocates
- * nothing. */
+ * writes with the same opts.  out: (B,Hq,N,d) in `out_layout`, dtype
+ * `out_dtype`.  vm is added to the output when opts->smooth_v (NULL allowed
+ * otherwise).  Allocates nothing. */
 sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t* k8, const float* ks,
-                                const uint8_t* v8t, const float* vs, void* out, int B, int Hq, int Hkv, int N,
-                                int d, sage_dtype out_dtype, sage_layout out_layout, int is_causal, float sm_scale,
-                                sage_pv_mode pv_mode, void* stream);
+                                const uint8_t* v8t, const float* vs, const float* vm, void* out, int B, int Hq,
+                                int Hkv, int N, int d, sage_dtype out_dtype, sage_layout out_layout, int is_causal,
+                                float sm_scale, sage_pv_mode pv_mode, const sage_opts* opts, void* stream);
 
 /* Diagnostic: the exact int32 scores S = Q8 . K8^T of selected 128x128 tiles,
  * computed by the same TMA + tcgen05 kind::i8 path as the fused kernel.

@@ -14,7 +14,9 @@ mirrors the ``sageattn(q, k, v, tensor_layout, is_causal, sm_scale)`` call of
 the SageAttention README ("How to Use"); ``pv_accum_dtype`` selects "fp32" or
 "fp16+fp32" accumulation of the P.V product (qwbw.cn article, pitfalls) and
 ``pv_dtype`` its operands: "fp8" (E4M3, the INT8-QK / FP8-PV kernel) or "fp16"
-(the INT8-QK / FP16-PV kernel of the README's "Available APIs").
+(the INT8-QK / FP16-PV kernel of the README's "Available APIs"); ``qk_quant_gran``
+the Q scale granularity ("per_block", "per_warp", "per_thread") and ``smooth_v``
+optional V smoothing (see ``sage_opts`` in include/sage.h).
 """
 from __future__ import annotations
 
@@ -26,7 +28,7 @@ import torch
 __all__ = [
     "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
     "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
-    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode", "sage_attn_varlen",
+    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode", "sage_attn_varlen", "SageOpts", "opts",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
@@ -60,6 +62,21 @@ def pv_mode(pv_dtype: str = "fp8", pv_accum_dtype: str = "fp32") -> int:
         raise ValueError(f"unsupported pv_dtype / pv_accum_dtype {pv_dtype!r} / {pv_accum_dtype!r}") from None
 
 
+class SageOpts(ctypes.Structure):
+    """The C ``sage_opts``: query tokens per Q scale (128, 32 or 1) and V smoothing (0 / 1)."""
+    _fields_ = [("q_gran", ctypes.c_int), ("smooth_v", ctypes.c_int)]
+
+
+_GRANS = {"per_block": 128, "per_warp": 32, "per_thread": 1}
+
+
+def opts(qk_quant_gran: str = "per_block", smooth_v: bool = False) -> SageOpts:
+    """SageOpts for a granularity name ("per_block", "per_warp", "per_thread") and V smoothing."""
+    if qk_quant_gran not in _GRANS:
+        raise ValueError(f"qk_quant_gran must be one of {sorted(_GRANS)}, got {qk_quant_gran!r}")
+    return SageOpts(_GRANS[qk_quant_gran], 1 if smooth_v else 0)
+
+
 def _load() -> ctypes.CDLL:
     if not os.path.exists(LIB_PATH):
         raise ImportError(
@@ -70,16 +87,16 @@ def _load() -> ctypes.CDLL:
     sig = {
         "sage_attn": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
         "sage_workspace_bytes": ([I, I, I, I, I], Z),
-        "sage_quantize": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P], I),
-        "sage_attn_quantized": ([P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
+        "sage_quantize": ([P, P, P, I, I, I, I, I, I, I, I, P, P, P, P, P, P, P, P, P, P], I),
+        "sage_attn_quantized": ([P, P, P, P, P, P, P, P, I, I, I, I, I, I, I, I, F, I, P, P], I),
         "sage_qk_int32": ([P, P, I, I, I, I, I, P, I, P, P], I),
         "sage_check_status": ([P], I),
         "sage_status_string": ([I], ctypes.c_char_p),
         "sage_device_supported": ([], I),
         "sage_attn_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
-        "sage_attn_ex": ([P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P], I),
-        "sage_attn_varlen": ([P, P, P, P, P, P, I, I, I, ctypes.c_longlong, ctypes.c_longlong, I, I, I, I, I, F, I, P],
-                             I),
+        "sage_attn_ex": ([P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P, P], I),
+        "sage_attn_varlen": ([P, P, P, P, P, P, I, I, I, ctypes.c_longlong, ctypes.c_longlong, I, I, I, I, I, F, I, P,
+                              P], I),
     }
     for name, (args, res) in sig.items():
         fn = getattr(lib, name)
@@ -162,29 +179,32 @@ def _check_inputs(q, k, v, layout):
 
 
 def sage_attn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, pv_accum_dtype="fp32", out=None,
-              pv_dtype="fp8"):
+              pv_dtype="fp8", qk_quant_gran="per_block", smooth_v=False):
     """Quantized attention of fp16/bf16 q (B,Hq,Nq,d), k/v (B,Hkv,Nk,d) (HND; NHD stores (B,N,H,d)).
 
-    Nq may differ from Nk (then through sage_attn_ex: the causal mask is aligned bottom-right)."""
+    Nq may differ from Nk (then the causal mask is aligned bottom-right); non-default
+    qk_quant_gran / smooth_v, or Nq != Nk, go through sage_attn_ex."""
     B, Hq, Hkv, N, Nk, d = _check_inputs_nk(q, k, v, tensor_layout)
+    o = opts(qk_quant_gran, smooth_v)
     if out is None:
         out = torch.empty_like(q)
     scale = float(sm_scale) if sm_scale is not None else 0.0
     mode = pv_mode(pv_dtype, pv_accum_dtype)
-    if Nk == N:
+    if Nk == N and o.q_gran == 128 and not o.smooth_v:
         st = capi.sage_attn(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, d,
                             _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)), scale, mode, _stream())
         _check(st, "sage_attn")
     else:
         st = capi.sage_attn_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), B, Hq, Hkv, N, Nk, d,
                                _DTYPES[q.dtype], _LAYOUTS[tensor_layout], int(bool(is_causal)), scale, mode,
-                               _stream())
+                               ctypes.byref(o), _stream())
         _check(st, "sage_attn_ex")
     return out
 
 
 def sage_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, is_causal=False,
-                     sm_scale=None, pv_accum_dtype="fp32", out=None, pv_dtype="fp8"):
+                     sm_scale=None, pv_accum_dtype="fp32", out=None, pv_dtype="fp8", qk_quant_gran="per_block",
+                     smooth_v=False):
     """Packed batch: q (total_q, Hq, d), k/v (total_k, Hkv, d), cu_seqlens_* int32 CUDA tensors of
     B + 1 offsets (sequence b = tokens cu[b] .. cu[b+1]-1).  Each sequence attends to its own keys
     (causal: aligned bottom-right per sequence).  A bad offset table raises SageError from the
@@ -208,7 +228,7 @@ def sage_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seql
                                cu_seqlens_k.data_ptr(), B, int(max_seqlen_q), int(max_seqlen_k), total_q, total_k,
                                Hq, Hkv, d, _DTYPES[q.dtype], int(bool(is_causal)),
                                float(sm_scale) if sm_scale is not None else 0.0, pv_mode(pv_dtype, pv_accum_dtype),
-                               _stream())
+                               ctypes.byref(opts(qk_quant_gran, smooth_v)), _stream())
     _check(st, "sage_attn_varlen")
     return out
 
@@ -238,34 +258,37 @@ def sage_workspace_bytes(B, Hq, Hkv, N, d) -> int:
     return int(capi.sage_workspace_bytes(B, Hq, Hkv, N, d))
 
 
-def sage_quantize(q, k, v, tensor_layout="HND", pv_accum_dtype="fp32", pv_dtype="fp8") -> dict:
+def sage_quantize(q, k, v, tensor_layout="HND", pv_accum_dtype="fp32", pv_dtype="fp8", qk_quant_gran="per_block",
+                  smooth_v=False) -> dict:
     """The quantize/smooth pass alone; returns the codes and scales as CUDA tensors.
 
     Layouts (Np = 128*ceil(N/128), dp = padded head dim): q8 int8 (B,Hq,Np,dp),
     qs f32 (B,Hq,Np/128), k8 int8 (B,Hkv,Np,dp), ks f32 (B,Hkv,Np/128),
     km f32 (B,Hkv,dp), v8t (B,Hkv,dp,Np) uint8 E4M3 codes (pv_dtype "fp8") or
-    float16 codes (pv_dtype "fp16"), vs f32 (B,Hkv,dp).
+    float16 codes (pv_dtype "fp16"), vs f32 (B,Hkv,dp), vm f32 (B,Hkv,dp) (V's token mean
+    with smooth_v, else zeros); qs has Np / q_gran entries per head.
     """
     mode = pv_mode(pv_dtype, pv_accum_dtype)
+    o = opts(qk_quant_gran, smooth_v)
     B, Hq, Hkv, N, d = _check_inputs(q, k, v, tensor_layout)
     dp, nb = padded_dim(d), (N + 127) // 128
     Np = nb * 128
     dev = q.device
     z = dict(
         q8=torch.empty((B, Hq, Np, dp), dtype=torch.int8, device=dev),
-        qs=torch.empty((B, Hq, nb), dtype=torch.float32, device=dev),
+        qs=torch.empty((B, Hq, Np // o.q_gran), dtype=torch.float32, device=dev),
         k8=torch.empty((B, Hkv, Np, dp), dtype=torch.int8, device=dev),
         ks=torch.empty((B, Hkv, nb), dtype=torch.float32, device=dev),
         km=torch.empty((B, Hkv, dp), dtype=torch.float32, device=dev),
         v8t=torch.empty((B, Hkv, dp, Np), dtype=torch.float16 if pv_dtype == "fp16" else torch.uint8, device=dev),
         vs=torch.empty((B, Hkv, dp), dtype=torch.float32, device=dev),
+        vm=torch.zeros((B, Hkv, dp), dtype=torch.float32, device=dev),
     )
     st = capi.sage_quantize(q.data_ptr(), k.data_ptr(), v.data_ptr(), B, Hq, Hkv, N, d, _DTYPES[q.dtype],
-                            _LAYOUTS[tensor_layout], mode, *(z[n].data_ptr() for n in
-                                                                          ("q8", "qs", "k8", "ks", "km", "v8t", "vs")),
-                            _stream())
+                            _LAYOUTS[tensor_layout], mode, ctypes.byref(o),
+                            *(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "km", "v8t", "vs", "vm")), _stream())
     _check(st, "sage_quantize")
-    z.update(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, pv_dtype=pv_dtype)
+    z.update(B=B, Hq=Hq, Hkv=Hkv, N=N, d=d, pv_dtype=pv_dtype, qk_quant_gran=qk_quant_gran, smooth_v=bool(smooth_v))
     return z
 
 
@@ -277,10 +300,13 @@ def sage_attn_quantized(z: dict, out_dtype=torch.float16, tensor_layout="HND", i
     if out is None:
         shape = (B, Hq, N, d) if tensor_layout == "HND" else (B, N, Hq, d)
         out = torch.empty(shape, dtype=out_dtype, device=z["q8"].device)
+    o = opts(z.get("qk_quant_gran", "per_block"), z.get("smooth_v", False))
+    vm = z.get("vm")
     st = capi.sage_attn_quantized(*(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "v8t", "vs")),
+                                  vm.data_ptr() if vm is not None else None,
                                   out.data_ptr(), B, Hq, Hkv, N, d, _DTYPES[out.dtype], _LAYOUTS[tensor_layout],
                                   int(bool(is_causal)), float(sm_scale) if sm_scale is not None else 0.0,
-                                  pv_mode(z.get("pv_dtype", "fp8"), pv_accum_dtype), _stream())
+                                  pv_mode(z.get("pv_dtype", "fp8"), pv_accum_dtype), ctypes.byref(o), _stream())
     _check(st, "sage_attn_quantized")
     return out
 

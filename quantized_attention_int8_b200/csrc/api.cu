@@ -170,6 +170,29 @@ bool pv_mode_valid(int pv_mode) {
 }
 bool pv_mode_fp16_operands(int pv_mode) { return pv_mode == SAGE_PV16_FP32 || pv_mode == SAGE_PV16_FP16_FP32; }
 
+// sage_opts, checked: log2 of the query tokens per Q scale, and V smoothing
+struct Opts {
+  int q_gran_log2 = 7;
+  int smooth_v = 0;
+};
+
+sage_status parse_opts(const sage_opts* o, Opts* out) {
+  Opts r;
+  if (o) {
+    switch (o->q_gran) {
+      case 0:
+      case 128: r.q_gran_log2 = 7; break;
+      case 32: r.q_gran_log2 = 5; break;
+      case 1: r.q_gran_log2 = 0; break;
+      default: return SAGE_ERR_INVALID_ARG;
+    }
+    if (o->smooth_v != 0 && o->smooth_v != 1) return SAGE_ERR_INVALID_ARG;
+    r.smooth_v = o->smooth_v;
+  }
+  *out = r;
+  return SAGE_OK;
+}
+
 // Workspace memory: a stream-ordered pool per device, owned by the library, that keeps the
 // memory it has handed out (release threshold = unlimited), so that repeated calls reuse
 // it instead of mapping fresh device memory each time.
@@ -203,6 +226,7 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t st) {
 
 struct QuantBufs {
   const SeqDesc* seqs;  // packed batches: the per-sequence table (else nullptr)
+  float* vm;            // V's token mean (read only when V is smoothed)
   int8_t* q8;
   float* qs;
   int8_t* k8;
@@ -213,7 +237,7 @@ struct QuantBufs {
 };
 
 sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, int layout, int causal, float sm_scale,
-                    int pv_mode, cudaStream_t st) {
+                    int pv_mode, const Opts& o, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   const uint32_t ksub = m.dp >= 128 ? 128 : 64;
   const uint32_t dv = m.dp == 64 ? 64 : 128;
@@ -227,6 +251,8 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
     return SAGE_ERR_CUDA;
   FwdParams p;
   p.qs = qb.qs, p.ks = qb.ks, p.vs = qb.vs, p.out = out;
+  p.vm = o.smooth_v ? qb.vm : nullptr;
+  p.q_gran_log2 = o.q_gran_log2;
   p.m = seq_map(m, layout, qb.seqs);
   p.nblk_q = m.nblk_q;
   p.G = m.G;
@@ -237,10 +263,10 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
 }
 
 struct WsLayout {
-  size_t q8, qs, k8, ks, km, v8t, vs, ksum, vmax, vinv, seqs, total;
+  size_t q8, qs, k8, ks, km, v8t, vs, vm, ksum, vmax, vsum, vmin, vinv, seqs, total;
 };
 
-WsLayout ws_layout(const Dims& m, int pv_mode) {
+WsLayout ws_layout(const Dims& m, int pv_mode, const Opts& o) {
   WsLayout w;
   size_t off = 0;
   auto take = [&](size_t bytes) {
@@ -249,14 +275,17 @@ WsLayout ws_layout(const Dims& m, int pv_mode) {
     return o;
   };
   w.q8 = take((size_t)m.q_rows * m.dp);
-  w.qs = take((size_t)m.q_rows / 128 * 4);
+  w.qs = take(((size_t)m.q_rows >> o.q_gran_log2) * 4);
   w.k8 = take((size_t)m.k_rows * m.dp);
   w.ks = take((size_t)m.k_rows / 128 * 4);
   w.km = take((size_t)m.B * m.Hkv * m.dp * 4);
   w.v8t = take((size_t)m.k_rows * m.dp * (pv_mode_fp16_operands(pv_mode) ? 2 : 1));
   w.vs = take((size_t)m.B * m.Hkv * m.dp * 4);
+  w.vm = take((size_t)m.B * m.Hkv * m.dp * 4);
   w.ksum = take((size_t)m.k_rows / 128 * m.dp * 4);
   w.vmax = take((size_t)m.k_rows / 128 * m.dp * 4);
+  w.vsum = take(o.smooth_v ? (size_t)m.k_rows / 128 * m.dp * 4 : 0);
+  w.vmin = take(o.smooth_v ? (size_t)m.k_rows / 128 * m.dp * 4 : 0);
   w.vinv = take((size_t)m.B * m.Hkv * m.dp * 4);
   w.seqs = take(m.packed ? (size_t)m.B * sizeof(SeqDesc) : 0);
   w.total = off;
@@ -264,7 +293,7 @@ WsLayout ws_layout(const Dims& m, int pv_mode) {
 }
 
 QuantParams quant_params(const Dims& m, const void* q, const void* k, const void* v, int dtype, int layout,
-                         int pv_mode) {
+                         int pv_mode, const Opts& o) {
   QuantParams p;
   memset(&p, 0, sizeof(p));
   p.q = q, p.k = k, p.v = v;
@@ -276,6 +305,8 @@ QuantParams quant_params(const Dims& m, const void* q, const void* k, const void
   p.vec_v = (m.d % 8 == 0) && aligned16(v);
   p.vmax_code = pv_mode == SAGE_PV_FP32 ? 448.0f : 1.0f;
   p.v_fp16 = pv_mode_fp16_operands(pv_mode) ? 1 : 0;
+  p.q_gran_log2 = o.q_gran_log2;
+  p.smooth_v = o.smooth_v;
   return p;
 }
 
@@ -294,41 +325,45 @@ bool out_overlaps(const Dims& m, const void* q, const void* k, const void* v, co
   return overlaps(out, qbytes, q, qbytes) || overlaps(out, qbytes, k, kvbytes) || overlaps(out, qbytes, v, kvbytes);
 }
 
-// Quantize pass + fused kernel on a workspace laid out by ws_layout(m, pv_mode); packed batches
+// Quantize pass + fused kernel on a workspace laid out by ws_layout(m, pv_mode, o); packed batches
 // first build their per-sequence table from cu_q / cu_k.
 sage_status attend_on(const Dims& m, unsigned char* ws, const void* q, const void* k, const void* v, void* out,
                       const int32_t* cu_q, const int32_t* cu_k, int dtype, int layout, int causal, float sm_scale,
-                      int pv_mode, cudaStream_t st) {
-  const WsLayout w = ws_layout(m, pv_mode);
+                      int pv_mode, const Opts& o, cudaStream_t st) {
+  const WsLayout w = ws_layout(m, pv_mode, o);
   SeqDesc* seqs = m.packed ? reinterpret_cast<SeqDesc*>(ws + w.seqs) : nullptr;
   if (m.packed) {
     sage_status s = from_cuda(launch_seq_plan(cu_q, cu_k, m.B, m.Nq, m.Nk, m.total_q, m.total_k, seqs, st));
     if (s != SAGE_OK) return s;
   }
-  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
+  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode, o);
   qp.m.seqs = seqs;
   QuantBufs qb{seqs,
+               reinterpret_cast<float*>(ws + w.vm),
                reinterpret_cast<int8_t*>(ws + w.q8), reinterpret_cast<float*>(ws + w.qs),
                reinterpret_cast<int8_t*>(ws + w.k8), reinterpret_cast<float*>(ws + w.ks),
                reinterpret_cast<float*>(ws + w.km), ws + w.v8t, reinterpret_cast<float*>(ws + w.vs)};
   qp.q8 = qb.q8, qp.qs = qb.qs, qp.k8 = qb.k8, qp.ks = qb.ks, qp.km = qb.km, qp.v8t = qb.v8t, qp.vs = qb.vs;
+  qp.vm = qb.vm;
   qp.ksum_part = reinterpret_cast<float*>(ws + w.ksum);
   qp.vmax_part = reinterpret_cast<float*>(ws + w.vmax);
+  qp.vsum_part = reinterpret_cast<float*>(ws + w.vsum);
+  qp.vmin_part = reinterpret_cast<float*>(ws + w.vmin);
   qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
   sage_status s = from_cuda(launch_quantize(qp, st));
-  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, causal, sm_scale, pv_mode, st);
+  if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, causal, sm_scale, pv_mode, o, st);
   return s;
 }
 
 // The same, on a workspace taken from the library's pool and released stream-ordered.
 sage_status attend_pooled(const Dims& m, const void* q, const void* k, const void* v, void* out, const int32_t* cu_q,
                           const int32_t* cu_k, int dtype, int layout, int causal, float sm_scale, int pv_mode,
-                          cudaStream_t st) {
-  const WsLayout w = ws_layout(m, pv_mode);
+                          const Opts& o, cudaStream_t st) {
+  const WsLayout w = ws_layout(m, pv_mode, o);
   unsigned char* ws = nullptr;
   cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&ws), w.total, st);
   if (e != cudaSuccess) return from_cuda(e);
-  sage_status s = attend_on(m, ws, q, k, v, out, cu_q, cu_k, dtype, layout, causal, sm_scale, pv_mode, st);
+  sage_status s = attend_on(m, ws, q, k, v, out, cu_q, cu_k, dtype, layout, causal, sm_scale, pv_mode, o, st);
   const cudaError_t ef = cudaFreeAsync(ws, st);
   if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
   return s;
@@ -341,64 +376,78 @@ extern "C" {
 size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   Dims m;
   if (check_dims(B, Hq, Hkv, N, N, d, &m) != SAGE_OK) return 0;
-  return ws_layout(m, SAGE_PV16_FP32).total;  // the largest over the P.V modes
+  Opts largest;
+  largest.q_gran_log2 = 0, largest.smooth_v = 1;
+  return ws_layout(m, SAGE_PV16_FP32, largest).total;  // the largest over the P.V modes and options
 }
 
 sage_status sage_attn_ex(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int Nq,
                          int Nk, int d, sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale,
-                         sage_pv_mode pv_mode, void* stream) {
+                         sage_pv_mode pv_mode, const sage_opts* opts, void* stream) {
   sage_status s = check_common(q, k, v, dtype, layout, pv_mode);
   if (s != SAGE_OK) return s;
+  Opts o;
+  if ((s = parse_opts(opts, &o)) != SAGE_OK) return s;
   Dims m;
   if ((s = check_dims(B, Hq, Hkv, Nq, Nk, d, &m)) != SAGE_OK) return s;
   if (!out || out_overlaps(m, q, k, v, out)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
-  return attend_pooled(m, q, k, v, out, nullptr, nullptr, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode,
+  return attend_pooled(m, q, k, v, out, nullptr, nullptr, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode, o,
                        static_cast<cudaStream_t>(stream));
 }
 
 sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
                       sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
                       void* stream) {
-  return sage_attn_ex(q, k, v, out, B, Hq, Hkv, N, N, d, dtype, layout, is_causal, sm_scale, pv_mode, stream);
+  return sage_attn_ex(q, k, v, out, B, Hq, Hkv, N, N, d, dtype, layout, is_causal, sm_scale, pv_mode, nullptr,
+                      stream);
 }
 
 sage_status sage_attn_varlen(const void* q, const void* k, const void* v, void* out, const int32_t* cu_seqlens_q,
                              const int32_t* cu_seqlens_k, int B, int max_seqlen_q, int max_seqlen_k,
                              long long total_q, long long total_k, int Hq, int Hkv, int d, sage_dtype dtype,
-                             int is_causal, float sm_scale, sage_pv_mode pv_mode, void* stream) {
+                             int is_causal, float sm_scale, sage_pv_mode pv_mode, const sage_opts* opts,
+                             void* stream) {
   sage_status s = check_common(q, k, v, dtype, SAGE_NHD, pv_mode);
   if (s != SAGE_OK) return s;
+  Opts o;
+  if ((s = parse_opts(opts, &o)) != SAGE_OK) return s;
   if (!cu_seqlens_q || !cu_seqlens_k) return SAGE_ERR_INVALID_ARG;
   Dims m;
   if ((s = check_dims_packed(B, Hq, Hkv, max_seqlen_q, max_seqlen_k, total_q, total_k, d, &m)) != SAGE_OK) return s;
   if (!out || out_overlaps(m, q, k, v, out)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   return attend_pooled(m, q, k, v, out, cu_seqlens_q, cu_seqlens_k, dtype, SAGE_NHD, is_causal ? 1 : 0, sm_scale,
-                       pv_mode, static_cast<cudaStream_t>(stream));
+                       pv_mode, o, static_cast<cudaStream_t>(stream));
 }
 
 sage_status sage_quantize(const void* q, const void* k, const void* v, int B, int Hq, int Hkv, int N, int d,
-                          sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, int8_t* q8, float* qs,
-                          int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs, void* stream) {
+                          sage_dtype dtype, sage_layout layout, sage_pv_mode pv_mode, const sage_opts* opts,
+                          int8_t* q8, float* qs, int8_t* k8, float* ks, float* km, uint8_t* v8t, float* vs,
+                          float* vm, void* stream) {
   sage_status s = check_common(q, k, v, dtype, layout, pv_mode);
   if (s != SAGE_OK) return s;
+  Opts o;
+  if ((s = parse_opts(opts, &o)) != SAGE_OK) return s;
   Dims m;
   if ((s = check_dims(B, Hq, Hkv, N, N, d, &m)) != SAGE_OK) return s;
-  if (!q8 || !qs || !k8 || !ks || !km || !v8t || !vs) return SAGE_ERR_INVALID_ARG;
+  if (!q8 || !qs || !k8 || !ks || !km || !v8t || !vs || (o.smooth_v && !vm)) return SAGE_ERR_INVALID_ARG;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   const size_t part = align_up((size_t)m.k_rows / 128 * m.dp * 4);
   const size_t vinv = align_up((size_t)m.B * m.Hkv * m.dp * 4);
+  const int nparts = o.smooth_v ? 4 : 2;
   unsigned char* scratch = nullptr;
-  cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&scratch), 2 * part + vinv, st);
+  cudaError_t e = workspace_alloc(reinterpret_cast<void**>(&scratch), nparts * part + vinv, st);
   if (e != cudaSuccess) return from_cuda(e);
-  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode);
-  qp.q8 = q8, qp.qs = qs, qp.k8 = k8, qp.ks = ks, qp.km = km, qp.v8t = v8t, qp.vs = vs;
+  QuantParams qp = quant_params(m, q, k, v, dtype, layout, pv_mode, o);
+  qp.q8 = q8, qp.qs = qs, qp.k8 = k8, qp.ks = ks, qp.km = km, qp.v8t = v8t, qp.vs = vs, qp.vm = vm;
   qp.ksum_part = reinterpret_cast<float*>(scratch);
   qp.vmax_part = reinterpret_cast<float*>(scratch + part);
-  qp.vinv = reinterpret_cast<float*>(scratch + 2 * part);
+  qp.vsum_part = o.smooth_v ? reinterpret_cast<float*>(scratch + 2 * part) : nullptr;
+  qp.vmin_part = o.smooth_v ? reinterpret_cast<float*>(scratch + 3 * part) : nullptr;
+  qp.vinv = reinterpret_cast<float*>(scratch + nparts * part);
   s = from_cuda(launch_quantize(qp, st));
   const cudaError_t ef = cudaFreeAsync(scratch, st);
   if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
@@ -406,21 +455,25 @@ sage_status sage_quantize(const void* q, const void* k, const void* v, int B, in
 }
 
 sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t* k8, const float* ks,
-                                const uint8_t* v8t, const float* vs, void* out, int B, int Hq, int Hkv, int N,
-                                int d, sage_dtype out_dtype, sage_layout out_layout, int is_causal, float sm_scale,
-                                sage_pv_mode pv_mode, void* stream) {
+                                const uint8_t* v8t, const float* vs, const float* vm, void* out, int B, int Hq,
+                                int Hkv, int N, int d, sage_dtype out_dtype, sage_layout out_layout, int is_causal,
+                                float sm_scale, sage_pv_mode pv_mode, const sage_opts* opts, void* stream) {
   if (!q8 || !qs || !k8 || !ks || !v8t || !vs || !out) return SAGE_ERR_INVALID_ARG;
   sage_status s = check_dtype(out_dtype);
   if (s != SAGE_OK) return s;
   if (out_layout != SAGE_HND && out_layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
   if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
+  Opts o;
+  if ((s = parse_opts(opts, &o)) != SAGE_OK) return s;
+  if (o.smooth_v && !vm) return SAGE_ERR_INVALID_ARG;
   Dims m;
   if ((s = check_dims(B, Hq, Hkv, N, N, d, &m)) != SAGE_OK) return s;
   if (!aligned16(q8) || !aligned16(k8) || !aligned16(v8t)) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
-  QuantBufs qb{nullptr, const_cast<int8_t*>(q8), const_cast<float*>(qs), const_cast<int8_t*>(k8),
-               const_cast<float*>(ks), nullptr, const_cast<uint8_t*>(v8t), const_cast<float*>(vs)};
-  return run_fwd(m, qb, out, out_dtype, out_layout, is_causal ? 1 : 0, sm_scale, pv_mode,
+  QuantBufs qb{nullptr, const_cast<float*>(vm), const_cast<int8_t*>(q8), const_cast<float*>(qs),
+               const_cast<int8_t*>(k8), const_cast<float*>(ks), nullptr, const_cast<uint8_t*>(v8t),
+               const_cast<float*>(vs)};
+  return run_fwd(m, qb, out, out_dtype, out_layout, is_causal ? 1 : 0, sm_scale, pv_mode, o,
                  static_cast<cudaStream_t>(stream));
 }
 
@@ -504,13 +557,14 @@ extern "C" sage_status sage_attn_noalloc(const void* q, const void* k, const voi
   Dims m;
   if ((s = check_dims(B, Hq, Hkv, N, N, d, &m)) != SAGE_OK) return s;
   if (!out || out_overlaps(m, q, k, v, out)) return SAGE_ERR_INVALID_ARG;
-  const WsLayout w = ws_layout(m, pv_mode);
+  const Opts o;  // defaults
+  const WsLayout w = ws_layout(m, pv_mode, o);
   if (w.total > (size_t)SAGE_NOALLOC_MAX_BYTES) return SAGE_ERR_INVALID_ARG;
   if ((s = check_device()) != SAGE_OK) return s;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
   unsigned char* ws = nullptr;
   if (noalloc_scratch(dev, &ws) != cudaSuccess) return SAGE_ERR_CUDA;
-  return attend_on(m, ws, q, k, v, out, nullptr, nullptr, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode,
+  return attend_on(m, ws, q, k, v, out, nullptr, nullptr, dtype, layout, is_causal ? 1 : 0, sm_scale, pv_mode, o,
                    static_cast<cudaStream_t>(stream));
 }

@@ -120,7 +120,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 constexpr float kLog2_448 = 8.807354922057604f;  // p * 448 = 2^(log2 p + log2 448)
 constexpr float kTau = 2.0f;                       // reference-max slack of the online softmax (log2 units)
 
-template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16, bool PACKED>
+template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16, bool PACKED, bool OPTS>
 __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     sage_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                     const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -299,7 +299,11 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
     const uint32_t scol = tmem + lane_base + C::S_COL;
     const uint32_t ocol = tmem + lane_base + C::O_COL;
-    const float qsv = p.qs[(sv.q_row0 + (long long)hq * p.m.q_head_rows) / 128 + qt];
+    // the Q scale of this row's group (its 128-token block, or with finer scales (OPTS) its 32-token
+    // warp group or the row itself).  Instances without the options keep the plain block index:
+    // changing it was measured to slow the tile loop's schedule by 2%.
+    const float qsv = OPTS ? p.qs[(sv.q_row0 + (long long)hq * p.m.q_head_rows + qt * 128 + row) >> p.q_gran_log2]
+                           : p.qs[(sv.q_row0 + (long long)hq * p.m.q_head_rows) / 128 + qt];
     const float* ksp = p.ks + (sv.k_row0 + (long long)hkv * p.m.k_head_rows) / 128;
     unsigned char* prow = sP + row * C::ROWB;
     float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates the stored P values' scale
@@ -460,6 +464,9 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     if (ok) {
       const float inv_l = l > 0.f ? __fdiv_rn(1.f, l) : 0.f;  // a row that saw no key outputs zeros
       const float* vsp = p.vs + ((size_t)b * p.m.Hkv + hkv) * p.m.dp + vh * DV;
+      // smoothed V: its token mean goes back on (rows that saw a key)
+      const float* vmp =
+          (OPTS && p.vm && l > 0.f) ? p.vm + ((size_t)b * p.m.Hkv + hkv) * p.m.dp + vh * DV : nullptr;
 #pragma unroll 1
       for (int cc = 0; cc < DV / 32; ++cc) {
         uint32_t o[32];
@@ -470,6 +477,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
           const int c0 = vh * DV + cc * 32;
 #pragma unroll
           for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(o[e]) * (vsp[cc * 32 + e] * inv_l);
+          if (OPTS && vmp) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) of[e] = __fadd_rn(of[e], vmp[cc * 32 + e]);
+          }
           if (c0 + 32 <= p.m.d && p.vec_out) {
             uint32_t w[16];
 #pragma unroll
@@ -603,11 +614,14 @@ template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16>
 static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const FwdParams& p, cudaStream_t st) {
   using C = FwdCfg<DQK, DV, PV16>;
-  auto kern = p.m.seqs ? sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, true>
-                       : sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, false>;
-  static std::atomic<unsigned long long> attr_done_dense{0}, attr_done_packed{0};
-  std::atomic<unsigned long long>& attr_done = p.m.seqs ? attr_done_packed : attr_done_dense;
-  cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done);
+  const bool opts = p.q_gran_log2 != 7 || p.vm != nullptr;  // finer Q scales or smoothed V
+  const int which = (p.m.seqs ? 1 : 0) + (opts ? 2 : 0);
+  auto kern = which == 0 ? sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, false, false>
+            : which == 1 ? sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, true, false>
+            : which == 2 ? sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, false, true>
+                         : sage_fwd_kernel<DQK, DV, MODE, CAUSAL, OutT, PV16, true, true>;
+  static std::atomic<unsigned long long> attr_done[4] = {{0}, {0}, {0}, {0}};
+  cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done[which]);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nblk_q, p.m.Hq * p.n_vhalves, p.m.B);
   kern<<<grid, 192, C::SMEM, st>>>(tq, tk, tv, p);

@@ -125,8 +125,32 @@ __device__ __forceinline__ float block_max(float v, float* red) {
   return r;
 }
 
-// INT8 codes of this thread's tile, x(r, k) given by `val`; rows at or beyond `rows` (tokens
-// past N) get code 0 whatever `val` returns for them.
+// INT8 codes of this thread's tile, x(r, k) given by `val` and row r's 127 / amax by `inv_of`;
+// rows at or beyond `rows` (tokens past N) get code 0 whatever `val` returns for them.
+template <typename F, typename G>
+__device__ __forceinline__ void store_int8_tile_rows(int8_t* __restrict__ dst, int dp, const TileCoord& tc, G inv_of,
+                                                     int rows, F val) {
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const bool valid = tc.g * 16 + r < rows;
+    const float inv = inv_of(r);
+    uint32_t w[2];
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t packed = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        int code = __float2int_rn(__fmul_rn(val(r, half * 4 + e), inv));  // rint: ties to even
+        code = max(-127, min(127, code));
+        packed |= (uint32_t)(code & 0xFF) << (8 * e);
+      }
+      w[half] = valid ? packed : 0u;
+    }
+    *reinterpret_cast<uint2*>(dst + (size_t)(tc.g * 16 + r) * dp + tc.c0) = make_uint2(w[0], w[1]);
+  }
+}
+
+// The same with one 127 / amax for the whole tile.
 template <typename F>
 __device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp, const TileCoord& tc, float inv, int rows,
                                                 F val) {
@@ -162,8 +186,18 @@ __device__ __forceinline__ float tree8_max(const float* part, int dp, int c) {
   for (int g = 1; g < 8; ++g) m = fmaxf(m, p[g * dp]);
   return m;
 }
+__device__ __forceinline__ float tree8_min(const float* part, int dp, int c) {
+  const float* p = part + c;
+  float m = p[0];
+#pragma unroll
+  for (int g = 1; g < 8; ++g) m = fminf(m, p[g * dp]);
+  return m;
+}
 
-template <typename T>
+// FINE_Q: Q scales per token or per 32 tokens (else per 128-token block); SMOOTH_V: V's token
+// mean is subtracted before coding (pass 1 then gathers V's column sums, max and min).  Separate
+// instances keep the default path's register count (and occupancy) as low as before.
+template <typename T, bool FINE_Q, bool SMOOTH_V>
 __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
   __shared__ float red[8];
   __shared__ float part[8 * 256];
@@ -179,11 +213,42 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
     const int h = y;
     load_tile<T>(v, static_cast<const T*>(p.q) + sv.q_in + h * sv.q_head + n0 * sv.q_tok, sv.q_tok, d, rows, p.vec_q,
                  tc);
-    const float am = block_max(tile_absmax<T>(v), red);
-    const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
     const long long row = sv.q_row0 + h * p.m.q_head_rows + n0;
-    store_int8_tile(p.q8 + row * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); });
-    if (threadIdx.x == 0) p.qs[row / 128] = __fdiv_rn(am, 127.f);
+    if (!FINE_Q) {  // one scale for the 128-token block
+      const float am = block_max(tile_absmax<T>(v), red);
+      const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
+      store_int8_tile(p.q8 + row * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); });
+      if (threadIdx.x == 0) p.qs[row / 128] = __fdiv_rn(am, 127.f);
+    } else {  // one scale per token (q_gran 1) or per 32 tokens (q_gran 32)
+      // max |q| of each of this thread's 16 tokens over its 8 channels, then over the dp/8
+      // consecutive threads that hold the token's other channels
+      float ta[16];
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        const uint32_t a = __vmaxu2(__vmaxu2(v[r].x & 0x7FFF7FFFu, v[r].y & 0x7FFF7FFFu),
+                                    __vmaxu2(v[r].z & 0x7FFF7FFFu, v[r].w & 0x7FFF7FFFu));
+        ta[r] = bits_to_f32<T>(max(a & 0xFFFFu, a >> 16));
+      }
+      for (int o = 1; o < dp / 8; o <<= 1)
+#pragma unroll
+        for (int r = 0; r < 16; ++r) ta[r] = fmaxf(ta[r], __shfl_xor_sync(0xffffffffu, ta[r], o));
+      if (p.q_gran_log2 == 5) {  // tokens 32k..32k+31 = token groups 2k and 2k+1
+        float gm = ta[0];
+#pragma unroll
+        for (int r = 1; r < 16; ++r) gm = fmaxf(gm, ta[r]);
+        if (tc.cv == 0) red[tc.g] = gm;
+        __syncthreads();
+        gm = fmaxf(red[tc.g & ~1], red[tc.g | 1]);
+#pragma unroll
+        for (int r = 0; r < 16; ++r) ta[r] = gm;
+        if (tc.cv == 0 && (tc.g & 1) == 0) p.qs[(row + tc.g * 16) / 32] = __fdiv_rn(gm, 127.f);
+      } else if (tc.cv == 0) {
+#pragma unroll
+        for (int r = 0; r < 16; ++r) p.qs[row + tc.g * 16 + r] = __fdiv_rn(ta[r], 127.f);
+      }
+      store_int8_tile_rows(p.q8 + row * dp, dp, tc, [&](int r) { return ta[r] > 0.f ? __fdiv_rn(127.f, ta[r]) : 0.f; },
+                           rows, [&](int r, int e) { return elem<T>(v[r], e); });
+    }
   } else if (y < p.m.Hq + p.m.Hkv) {  // ---- K: per-block partial column sums
     const int h = y - p.m.Hq;
     load_tile<T>(v, static_cast<const T*>(p.k) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_k,
@@ -201,6 +266,38 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
     __syncthreads();
     const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
     p.ksum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
+  } else if (SMOOTH_V) {  // ---- V, smoothed: per-block partial column sums, max and min
+    const int h = y - p.m.Hq - p.m.Hkv;
+    load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
+                 tc);
+    float acc[8], hi[8], lo[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f, hi[e] = -INFINITY, lo[e] = INFINITY;
+#pragma unroll
+    for (int r = 0; r < 16; ++r)
+      if (tc.g * 16 + r < rows)  // tokens beyond N are skipped
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const float x = elem<T>(v[r], e);
+          acc[e] = __fadd_rn(acc[e], x);
+          hi[e] = fmaxf(hi[e], x);
+          lo[e] = fminf(lo[e], x);
+        }
+    const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = acc[e];
+    __syncthreads();
+    p.vsum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = hi[e];
+    __syncthreads();
+    p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
+    __syncthreads();
+#pragma unroll
+    for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = lo[e];
+    __syncthreads();
+    p.vmin_part[base + threadIdx.x] = tree8_min(part, dp, threadIdx.x);
   } else {  // ---- V: per-block partial column amax
     const int h = y - p.m.Hq - p.m.Hkv;
     load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
@@ -233,10 +330,29 @@ __global__ void quant_finalize_kernel(QuantParams p) {
     const float* ks = p.ksum_part + base + c;
     const float* vm = p.vmax_part + base + c;
     float acc = 0.f, am = 0.f;
+    if (p.smooth_v) {
+      // V - mean(V): its max |.| per channel is reached at the channel's largest or smallest v,
+      // since rounding v - mean to float32 is monotonic in v
+      const float* vsum = p.vsum_part + base + c;
+      const float* vmin = p.vmin_part + base + c;
+      float vacc = 0.f, hi = -INFINITY, lo = INFINITY;
 #pragma unroll 8
-    for (int i = 0; i < nblk; ++i) {  // sums stay in block order; the loads overlap
-      acc = __fadd_rn(acc, ks[(size_t)i * dp]);
-      am = fmaxf(am, vm[(size_t)i * dp]);
+      for (int i = 0; i < nblk; ++i) {  // sums stay in block order
+        acc = __fadd_rn(acc, ks[(size_t)i * dp]);
+        vacc = __fadd_rn(vacc, vsum[(size_t)i * dp]);
+        hi = fmaxf(hi, vm[(size_t)i * dp]);
+        lo = fminf(lo, vmin[(size_t)i * dp]);
+      }
+      const float mean = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(vacc, (float)sv.nk) : 0.f;
+      am = sv.nk > 0 ? fmaxf(fabsf(__fsub_rn(hi, mean)), fabsf(__fsub_rn(lo, mean))) : 0.f;
+      p.vm[(size_t)bh * dp + c] = mean;
+    } else {
+#pragma unroll 8
+      for (int i = 0; i < nblk; ++i) {  // sums stay in block order; the loads overlap
+        acc = __fadd_rn(acc, ks[(size_t)i * dp]);
+        am = fmaxf(am, vm[(size_t)i * dp]);
+      }
+      if (p.vm) p.vm[(size_t)bh * dp + c] = 0.f;
     }
     p.km[(size_t)bh * dp + c] = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(acc, (float)sv.nk) : 0.f;
     p.vs[(size_t)bh * dp + c] = __fdiv_rn(am, p.vmax_code);
@@ -249,7 +365,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   return __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3) & 0xFFFFu;
 }
 
-template <typename T>
+template <typename T, bool SMOOTH_V>
 __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
   __shared__ float red[8];
   const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
@@ -309,11 +425,19 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
   } else {  // ---- V: E4M3 or fp16 codes, transposed to [channel][token]
     const int h = y - p.m.Hkv;
     const size_t bh = (size_t)b * p.m.Hkv + h;
-    float inv[8];
+    float inv[8], mean[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) inv[e] = p.vinv[bh * dp + tc.c0 + e];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) mean[e] = SMOOTH_V ? p.vm[bh * dp + tc.c0 + e] : 0.f;
     load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
                  tc);
+    // (v - mean) * inv; tokens past N give 0 (with smoothing the subtraction would not)
+    auto vx = [&](int r, int e) -> float {
+      if (!SMOOTH_V) return __fmul_rn(elem<T>(v[r], e), inv[e]);  // tokens past N load as 0 -> code 0
+      const float x = __fsub_rn(elem<T>(v[r], e), mean[e]);
+      return (tc.g * 16 + r < rows) ? __fmul_rn(x, inv[e]) : 0.f;
+    };
     // V^T element (channel c, token t) of this sequence and head: row v_row0 + h*dp + c, column
     // v_col0 + t, rows k_head_rows codes apart
     const long long vrow = sv.v_row0 + (long long)h * dp + tc.c0, vcol = sv.v_col0 + n0 + tc.g * 16;
@@ -326,8 +450,7 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
         uint32_t w[8];
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-          const __half2 h2 = __floats2half2_rn(__fmul_rn(elem<T>(v[2 * q], e), inv[e]),
-                                               __fmul_rn(elem<T>(v[2 * q + 1], e), inv[e]));
+          const __half2 h2 = __floats2half2_rn(vx(2 * q, e), vx(2 * q + 1, e));
           w[q] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         uint4* dst = reinterpret_cast<uint4*>(vt + (vrow + e) * pitch + vcol);
@@ -341,10 +464,10 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
       uint32_t w[4];
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        const float a0 = __fmul_rn(elem<T>(v[4 * q + 0], e), inv[e]);
-        const float a1 = __fmul_rn(elem<T>(v[4 * q + 1], e), inv[e]);
-        const float a2 = __fmul_rn(elem<T>(v[4 * q + 2], e), inv[e]);
-        const float a3 = __fmul_rn(elem<T>(v[4 * q + 3], e), inv[e]);
+        const float a0 = vx(4 * q + 0, e);
+        const float a1 = vx(4 * q + 1, e);
+        const float a2 = vx(4 * q + 2, e);
+        const float a3 = vx(4 * q + 3, e);
         w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
       }
       *reinterpret_cast<uint4*>(p.v8t + (vrow + e) * pitch + vcol) =
@@ -356,9 +479,16 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
 template <typename T>
 static cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
   const int B = p.m.B, Hq = p.m.Hq, Hkv = p.m.Hkv, dp = p.m.dp;
-  quant_pass1_kernel<T><<<dim3(p.nblk_q > p.nblk_k ? p.nblk_q : p.nblk_k, Hq + 2 * Hkv, B), dp, 0, st>>>(p);
+  const dim3 grid1(p.nblk_q > p.nblk_k ? p.nblk_q : p.nblk_k, Hq + 2 * Hkv, B);
+  const bool fine = p.q_gran_log2 != 7;
+  if (fine && p.smooth_v) quant_pass1_kernel<T, true, true><<<grid1, dp, 0, st>>>(p);
+  else if (fine) quant_pass1_kernel<T, true, false><<<grid1, dp, 0, st>>>(p);
+  else if (p.smooth_v) quant_pass1_kernel<T, false, true><<<grid1, dp, 0, st>>>(p);
+  else quant_pass1_kernel<T, false, false><<<grid1, dp, 0, st>>>(p);
   quant_finalize_kernel<<<B * Hkv, dp, 0, st>>>(p);
-  quant_pass2_kernel<T><<<dim3(p.nblk_k > 0 ? p.nblk_k : 1, 2 * Hkv, B), dp, 0, st>>>(p);
+  const dim3 grid2(p.nblk_k > 0 ? p.nblk_k : 1, 2 * Hkv, B);
+  if (p.smooth_v) quant_pass2_kernel<T, true><<<grid2, dp, 0, st>>>(p);
+  else quant_pass2_kernel<T, false><<<grid2, dp, 0, st>>>(p);
   return cudaGetLastError();
 }
 

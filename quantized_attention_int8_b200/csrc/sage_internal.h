@@ -93,6 +93,11 @@ struct QuantParams {
   float* ksum_part;  // [k rows / 128][dp]: per 128-token block of K
   float* vmax_part;  // [k rows / 128][dp]
   float* vinv;       // [B][Hkv][dp]
+  float* vsum_part;  // [k rows / 128][dp] (V smoothing only)
+  float* vmin_part;  // [k rows / 128][dp] (V smoothing only; vmax_part then holds max v, not max |v|)
+  float* vm;         // [B][Hkv][dp] V's token mean (nullptr allowed when smooth_v is 0)
+  int smooth_v;      // code V - vm instead of V
+  int q_gran_log2;   // query tokens per Q scale: 7 (128), 5 (32) or 0 (1)
   float vmax_code;   // 448 (FP8 P.V, fp32 accumulation) or 1 (the other P.V modes)
   int v_fp16;        // V codes are fp16 (FP16 P.V) instead of E4M3; v8t then holds 2 bytes per code
 };
@@ -101,8 +106,10 @@ struct FwdParams {
   const float* qs;
   const float* ks;
   const float* vs;
+  const float* vm;  // V's token mean, added to the output (nullptr: V not smoothed)
   void* out;
   SeqMap m;
+  int q_gran_log2;  // query tokens per Q scale = 1 << q_gran_log2
   int nblk_q;     // 128-row query tiles of the longest sequence (grid x)
   int G;          // query heads per kv head
   int n_vhalves;  // output column halves handled by separate CTAs (2 when dp = 256)

@@ -87,10 +87,12 @@ def slice_heads(t: torch.Tensor, layout: str, b: int, heads) -> torch.Tensor:
 def oracle_to_device(qz: dict) -> dict:
     """Oracle codes/scales -> CUDA tensors in the library's layouts (V transposed)."""
     v8t = np.ascontiguousarray(qz["v8"].transpose(0, 1, 3, 2))
-    z = {k: torch.from_numpy(np.ascontiguousarray(qz[k])).cuda() for k in ("q8", "qs", "k8", "ks", "km", "vs")}
+    z = {k: torch.from_numpy(np.ascontiguousarray(qz[k])).cuda() for k in ("q8", "qs", "k8", "ks", "km", "vs", "vm")}
     z["v8t"] = torch.from_numpy(v8t).cuda()
     z.update({k: qz[k] for k in ("B", "Hq", "Hkv", "N", "d")})
     z["pv_dtype"] = "fp16" if qz["pv_mode"] & 2 else "fp8"
+    z["qk_quant_gran"] = {128: "per_block", 32: "per_warp", 1: "per_thread"}[qz.get("q_gran", 128)]
+    z["smooth_v"] = bool(qz.get("smooth_v", False))
     return z
 
 
@@ -110,6 +112,14 @@ def vmax_of(v) -> float:
 def pv_name(w: W.Workload) -> str:
     """pv_accum_dtype of the workload's P.V mode."""
     return "fp16+fp32" if w.pv_mode & 1 else "fp32"
+
+
+GRAN_NAME = {128: "per_block", 32: "per_warp", 1: "per_thread"}
+
+
+def opt_kw(w: W.Workload) -> dict:
+    """Keyword options of the Python binding for the workload's Q granularity and V smoothing."""
+    return dict(qk_quant_gran=GRAN_NAME[w.q_gran], smooth_v=w.smooth_v)
 
 
 def pv_dtype(w: W.Workload) -> str:

@@ -58,12 +58,24 @@ def test_sage_attn_argument_checks(lib):
 
 def test_other_entry_points_argument_checks(lib):
     c, E = lib.capi, lib.SAGE_ERR_INVALID_ARG
-    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, lib.SAGE_FP32, 0, 0, *([FAKE] * 7), None) == \
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, lib.SAGE_FP32, 0, 0, None, *([FAKE] * 8), None) == \
         lib.SAGE_ERR_UNSUPPORTED
-    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, None, *([FAKE] * 6), None) == E
-    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, FAKE + 1, *([FAKE] * 6), None) == E
-    assert c.sage_attn_quantized(*([FAKE] * 7), 1, 4, 3, 256, 64, 0, 0, 0, 0.0, 0, None) == E
-    assert c.sage_attn_quantized(*([FAKE] * 6), None, 1, 4, 2, 256, 64, 0, 0, 0, 0.0, 0, None) == E
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, None, None, *([FAKE] * 7), None) == E
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, None, FAKE + 1, *([FAKE] * 7), None) == E
+    assert c.sage_attn_quantized(*([FAKE] * 8), 1, 4, 3, 256, 64, 0, 0, 0, 0.0, 0, None, None) == E
+    assert c.sage_attn_quantized(*([FAKE] * 7), None, 1, 4, 2, 256, 64, 0, 0, 0, 0.0, 0, None, None) == E
+    # options: granularity must be 0, 128, 32 or 1; smooth_v 0 or 1; smoothing needs a vm buffer
+    bad = [lib.SageOpts(64, 0), lib.SageOpts(128, 2), lib.SageOpts(-1, 0)]
+    for o in bad:
+        assert c.sage_attn_ex(FAKE, FAKE + (1 << 34), FAKE + (2 << 34), FAKE + (3 << 34), 1, 2, 2, 256, 256, 64,
+                              0, 0, 0, 0.0, 0, ctypes.byref(o), None) == E
+        assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, ctypes.byref(o), *([FAKE] * 8),
+                               None) == E
+    sm = lib.SageOpts(1, 1)
+    assert c.sage_quantize(FAKE, FAKE, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, ctypes.byref(sm), *([FAKE] * 7), None,
+                           None) == E
+    assert c.sage_attn_quantized(*([FAKE] * 6), None, FAKE, 1, 2, 2, 256, 64, 0, 0, 0, 0.0, 0, ctypes.byref(sm),
+                                 None) == E
     assert c.sage_qk_int32(FAKE, FAKE, 1, 2, 2, 256, 64, None, 1, FAKE, None) == E
     assert c.sage_qk_int32(FAKE, FAKE, 1, 2, 2, 256, 300, FAKE, 1, FAKE, None) == E
     assert c.sage_qk_int32(FAKE, FAKE, 1, 2, 2, 256, 64, FAKE, 0, FAKE, None) == lib.SAGE_OK  # nothing to do
@@ -75,7 +87,9 @@ def test_workspace_bytes(lib):
     # 2 bytes of the FP16 P.V modes, the largest), plus fp32 scales and partial sums
     ws = lib.sage_workspace_bytes(2, 8, 2, 1000, 96)
     codes = 2 * (8 + 2 + 2 * 2) * 1024 * 128
-    assert codes < ws < codes + 2 * 2 * 8 * 128 * 4 * 2 + 64 * 1024
+    # the rest: per-token Q scales (the finest granularity, 2*8*1024 floats), four K/V partial-sum
+    # arrays (4 * 2*2*8 blocks * 128 floats), per-channel vectors and 1 KiB alignment per buffer
+    assert codes < ws < codes + 2 * 8 * 1024 * 4 + 4 * 2 * 2 * 8 * 128 * 4 + 96 * 1024
 
 
 def test_padded_dim(lib):
@@ -92,3 +106,11 @@ def test_pv_mode_names(lib):
     for bad in (("fp8", "fp16"), ("int8", "fp32"), ("fp16", "bf16")):
         with pytest.raises(ValueError):
             lib.pv_mode(*bad)
+
+
+def test_opts_names(lib):
+    assert (lib.opts().q_gran, lib.opts().smooth_v) == (128, 0)
+    assert (lib.opts("per_warp", True).q_gran, lib.opts("per_warp", True).smooth_v) == (32, 1)
+    assert lib.opts("per_thread").q_gran == 1
+    with pytest.raises(ValueError):
+        lib.opts("per_channel")

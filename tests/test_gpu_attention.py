@@ -6,7 +6,7 @@ import torch
 import workloads as W
 from oracle import attention, emulate, quant
 from tests._support import (check_vs_emulation, check_vs_exact, cuda, nkeys, oracle_to_device, out_hnd,
-                            pv_dtype, pv_name, slice_heads, vmax_of)
+                            opt_kw, pv_dtype, pv_name, slice_heads, vmax_of)
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +37,13 @@ SMALL = [
     W.TINY.with_(name="pv16_outlier_gqa4_causal_bf16", N=640, d=64, Hq=8, Hkv=2, dist="normal_koutlier",
                  dtype="bf16", causal=True, pv_mode=2),
     W.TINY.with_(name="pv16acc_d96_causal", N=1000, d=96, causal=True, pv_mode=3, dist="uniform2", sm_scale=None),
+    # Q scale granularity and V smoothing
+    W.TINY.with_(name="qgran32_causal_gqa_d64", N=640, Hq=8, Hkv=2, causal=True, q_gran=32),
+    W.TINY.with_(name="qgran1_d128_nhd_bf16", N=300, d=128, layout="NHD", dtype="bf16", q_gran=1, sm_scale=None),
+    W.TINY.with_(name="smoothv_koffset_d64_causal", N=700, d=64, dist="normal_koffset", causal=True, smooth_v=True),
+    W.TINY.with_(name="smoothv_qgran1_pv16_d256", N=300, d=256, pv_mode=2, q_gran=1, smooth_v=True, sm_scale=None),
+    W.TINY.with_(name="smoothv_qgran32_fp16acc_d96", N=513, d=96, pv_mode=1, q_gran=32, smooth_v=True,
+                 sm_scale=None),
 ]
 
 
@@ -48,7 +55,7 @@ def _scale(w):
 def test_attention_kernel_reproduces_method(lib, w):
     """sage_attn_quantized on the oracle's own codes vs the CPU emulation of the method."""
     q, k, v = W.make_inputs(w)
-    qz = quant.quantize(q, k, v, w.layout, w.pv_mode)
+    qz = quant.quantize(q, k, v, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
     z = oracle_to_device(qz)
     out = lib.sage_attn_quantized(z, q.dtype, w.layout, w.causal, _scale(w), pv_name(w))
     lib.sage_check_status()
@@ -59,21 +66,22 @@ def test_attention_kernel_reproduces_method(lib, w):
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
 def test_sage_attn_vs_exact_attention(lib, w):
     q, k, v = W.make_inputs(w)
-    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w))
+    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w),
+                        **opt_kw(w))
     lib.sage_check_status()
     ref = attention.attention_f64(q, k, v, w.layout, w.causal, _scale(w))
     em = None
     if w.dist == "normal_koutlier":  # not unit-variance: compare with the method's own accuracy
-        qz = quant.quantize(q, k, v, w.layout, w.pv_mode)
+        qz = quant.quantize(q, k, v, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
         em = emulate.emulate(qz, w.causal, _scale(w)).reshape(w.B, w.Hq, -1, w.d)[:, :, :w.N].astype(np.float64)
     check_vs_exact(out_hnd(out, w.layout), ref, nkeys(w.N, w.causal), vmax_of(v), w.name, emul=em)
 
 
-@pytest.mark.parametrize("w", SMALL[:6] + SMALL[10:13], ids=lambda w: w.name)
+@pytest.mark.parametrize("w", SMALL[:6] + SMALL[10:13] + SMALL[-5:], ids=lambda w: w.name)
 def test_end_to_end_equals_quantize_then_attend(lib, w):
     q, k, v = (cuda(t) for t in W.make_inputs(w))
-    a = lib.sage_attn(q, k, v, w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w))
-    z = lib.sage_quantize(q, k, v, w.layout, pv_name(w), pv_dtype(w))
+    a = lib.sage_attn(q, k, v, w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w), **opt_kw(w))
+    z = lib.sage_quantize(q, k, v, w.layout, pv_name(w), pv_dtype(w), **opt_kw(w))
     b = lib.sage_attn_quantized(z, q.dtype, w.layout, w.causal, _scale(w), pv_name(w))
     lib.sage_check_status()
     assert torch.equal(a.view(torch.int16), b.view(torch.int16))
@@ -105,7 +113,8 @@ def test_rejects_bad_inputs(lib):
 
 
 FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"],
-        W.BY_NAME["pad_sweep_b8_h16_n16384_d64_full"], W.BY_NAME["pad_sweep_b8_h16_n1024_d96_full"]] + W.FP16_PV
+        W.BY_NAME["pad_sweep_b8_h16_n16384_d64_full"], W.BY_NAME["pad_sweep_b8_h16_n1024_d96_full"]] + W.FP16_PV + \
+    W.OPTIONS
 
 
 def _rows(out, layout, b, h, rows):
@@ -117,7 +126,8 @@ def _rows(out, layout, b, h, rows):
 def test_full_size_sampled_rows(lib, w):
     """The full-size launch the bench times; the oracle checks sampled heads and 128-row blocks."""
     q, k, v = W.make_inputs(w)
-    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w))
+    out = lib.sage_attn(cuda(q), cuda(k), cuda(v), w.layout, w.causal, _scale(w), pv_name(w), pv_dtype=pv_dtype(w),
+                        **opt_kw(w))
     lib.sage_check_status()
     G = w.Hq // w.Hkv
     nb = (w.N + 127) // 128
@@ -132,7 +142,7 @@ def test_full_size_sampled_rows(lib, w):
         hk = hq // G
         qs, ks, vs = (slice_heads(t, w.layout, b, [hh]) for t, hh in ((q, hq), (k, hk), (v, hk)))
         got = _rows(out, w.layout, b, hq, torch.as_tensor(rows))
-        qz = quant.quantize(qs, ks, vs, w.layout, w.pv_mode)
+        qz = quant.quantize(qs, ks, vs, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
         em = emulate.emulate(qz, w.causal, _scale(w), heads=[(0, 0)], q_blocks=qbs)[0]
         em = np.concatenate([em[i * 128:i * 128 + min(128, w.N - qb * 128)] for i, qb in enumerate(qbs)])
         check_vs_emulation(got, em.astype(np.float64), vmax_of(vs), f"{w.name} b{b} h{hq}")

@@ -5,7 +5,7 @@ import torch
 
 import workloads as W
 from oracle import quant
-from tests._support import cuda, pv_dtype, pv_name, slice_heads
+from tests._support import cuda, opt_kw, pv_dtype, pv_name, slice_heads
 
 pytestmark = pytest.mark.gpu
 
@@ -20,13 +20,20 @@ SMALL = [
     W.TINY.with_(name="pv16_ragged_d40_gqa_bf16", N=300, d=40, Hq=4, Hkv=2, dtype="bf16", pv_mode=2),
     W.TINY.with_(name="pv16acc_nhd_koffset_d128", N=700, d=128, layout="NHD", dist="normal_koffset", pv_mode=3),
     W.TINY.with_(name="pv16_d256_outlier", B=2, N=129, d=256, dist="normal_koutlier", pv_mode=2),
+    # Q scale granularity and V smoothing
+    W.TINY.with_(name="qgran32_ragged_d40_gqa_bf16", N=300, d=40, Hq=4, Hkv=2, dtype="bf16", q_gran=32),
+    W.TINY.with_(name="qgran1_d128_nhd", N=257, d=128, layout="NHD", q_gran=1),
+    W.TINY.with_(name="qgran1_d256_smoothv", B=2, N=129, d=256, q_gran=1, smooth_v=True),
+    W.TINY.with_(name="smoothv_koffset_d64", N=700, d=64, dist="normal_koffset", smooth_v=True),
+    W.TINY.with_(name="smoothv_pv16acc_d96_ragged", N=333, d=96, pv_mode=3, smooth_v=True, q_gran=32),
+    W.TINY.with_(name="smoothv_fp16acc_d33", N=257, d=33, Hq=3, Hkv=1, pv_mode=1, smooth_v=True),
 ]
 
 
 def _gpu_codes(lib, w, q, k, v):
-    z = lib.sage_quantize(cuda(q), cuda(k), cuda(v), w.layout, pv_name(w), pv_dtype(w))
+    z = lib.sage_quantize(cuda(q), cuda(k), cuda(v), w.layout, pv_name(w), pv_dtype(w), **opt_kw(w))
     lib.sage_check_status()
-    out = {k2: z[k2].cpu().numpy() for k2 in ("q8", "qs", "k8", "ks", "km", "vs")}
+    out = {k2: z[k2].cpu().numpy() for k2 in ("q8", "qs", "k8", "ks", "km", "vs", "vm")}
     out["v8"] = z["v8t"].cpu().numpy().transpose(0, 1, 3, 2)
     return out
 
@@ -34,7 +41,7 @@ def _gpu_codes(lib, w, q, k, v):
 def _assert_same(got, ref, q_sel=slice(None), kv_sel=slice(None)):
     for key in ("q8", "qs"):
         assert np.array_equal(got[key][q_sel], ref[key]), key
-    for key in ("k8", "ks", "km", "v8", "vs"):
+    for key in ("k8", "ks", "km", "v8", "vs", "vm"):
         g, r = got[key][kv_sel], ref[key]
         if g.dtype == np.float32:
             ok = np.array_equal(g.view(np.uint32), r.view(np.uint32))
@@ -51,7 +58,7 @@ def _assert_same(got, ref, q_sel=slice(None), kv_sel=slice(None)):
 def test_quantize_bit_exact_small(lib, w):
     q, k, v = W.make_inputs(w)
     got = _gpu_codes(lib, w, q, k, v)
-    ref = quant.quantize(q, k, v, w.layout, w.pv_mode)
+    ref = quant.quantize(q, k, v, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
     _assert_same(got, ref)
 
 

@@ -108,7 +108,7 @@ def test_varlen_equal_lengths_is_the_dense_nhd_batch(lib, pv):
     # and Nq = Nk through sage_attn_ex is sage_attn
     ex = torch.empty_like(dense)
     st = lib.capi.sage_attn_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), ex.data_ptr(), 3, 4, 2, 300, 300, 64,
-                               lib.SAGE_FP16, lib.SAGE_NHD, 1, 0.125, pv, torch.cuda.current_stream().cuda_stream)
+                               lib.SAGE_FP16, lib.SAGE_NHD, 1, 0.125, pv, None, torch.cuda.current_stream().cuda_stream)
     assert st == lib.SAGE_OK
     lib.sage_check_status()
     assert torch.equal(dense.view(torch.int16), ex.view(torch.int16))

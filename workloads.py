@@ -53,6 +53,8 @@ class Workload:
     sm_scale: float | None = None  # None -> 1/sqrt(d)
     Nk: int | None = None          # key / value length when it differs from N (the query length)
     varlen: tuple = ()             # packed batch: ((nq, nk), ...) per sequence; then B = len(varlen)
+    q_gran: int = 128              # query tokens per Q scale: 128 (per block), 32 (per warp), 1 (per thread)
+    smooth_v: bool = False         # code V - mean_tokens(V), add the mean back
 
     @property
     def nk(self) -> int:
@@ -106,7 +108,11 @@ FP16_PV = [IMAGE_DIT.with_(name="image_dit_b2_h24_n4096_d64_pv16", pv_mode=2),
            VIDEO_DIT.with_(name="video_dit_b1_h24_n32768_d128_nhd_pv16", pv_mode=3),
            LLM_GQA.with_(name="llm_causal_gqa_b4_hq32_hkv8_n8192_d128_pv16", pv_mode=2)]
 
-ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV
+# The same inputs with finer Q scales and V smoothing.
+OPTIONS = [IMAGE_DIT.with_(name="image_dit_b2_h24_n4096_d64_qthread_smoothv", q_gran=1, smooth_v=True),
+           LLM_GQA.with_(name="llm_causal_gqa_b4_hq32_hkv8_n8192_d128_qwarp", q_gran=32)]
+
+ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV + OPTIONS
 BY_NAME = {w.name: w for w in ALL}
 
 
