@@ -31,6 +31,12 @@
 
 namespace sage {
 
+// Programmatic dependent launch: the finalize and pass-2 grids are launched while their
+// predecessor still runs; they wait here for it to complete (and its writes to be visible)
+// before reading what it wrote.
+__device__ __forceinline__ void wait_for_previous_grid() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void allow_next_grid() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 __device__ __forceinline__ float to_f32(__half x) { return __half2float(x); }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
 
@@ -199,6 +205,7 @@ __device__ __forceinline__ float tree8_min(const float* part, int dp, int c) {
 // instances keep the default path's register count (and occupancy) as low as before.
 template <typename T, bool FINE_Q, bool SMOOTH_V>
 __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
+  allow_next_grid();
   __shared__ float red[8];
   __shared__ float part[8 * 256];
   const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
@@ -322,6 +329,8 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
 }
 
 __global__ void quant_finalize_kernel(QuantParams p) {
+  allow_next_grid();
+  wait_for_previous_grid();  // pass 1's partial sums
   const int bh = blockIdx.x, b = bh / p.m.Hkv, h = bh - b * p.m.Hkv;
   const SeqView sv = seq_view(p.m, b);
   const int dp = p.m.dp, nblk = (sv.nk + 127) / 128;
@@ -368,7 +377,10 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 template <typename T, bool SMOOTH_V>
 __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
   __shared__ float red[8];
-  const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
+  wait_for_previous_grid();  // the finalize kernel's K mean and V scales
+  // Last-read-first: pass 1 read V after K and batch B-1 last, so those are the tiles most likely
+  // still in L2 when this pass reads them again.
+  const int blk = gridDim.x - 1 - blockIdx.x, y = gridDim.y - 1 - blockIdx.y, b = gridDim.z - 1 - blockIdx.z;
   const SeqView sv = seq_view(p.m, b);
   const int n0 = blk * 128, rows = min(128, sv.nk - n0);
   if (rows <= 0) return;  // past the end of this sequence (the whole CTA leaves)
@@ -476,6 +488,23 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
   }
 }
 
+// Launch `kern` so that it may start while the previous kernel in the stream still runs (it
+// waits with griddepcontrol.wait before reading that kernel's output).
+template <typename K>
+static cudaError_t launch_dependent(K kern, dim3 grid, dim3 block, cudaStream_t st, const QuantParams& p) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, p);
+}
+
 template <typename T>
 static cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
   const int B = p.m.B, Hq = p.m.Hq, Hkv = p.m.Hkv, dp = p.m.dp;
@@ -485,11 +514,13 @@ static cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
   else if (fine) quant_pass1_kernel<T, true, false><<<grid1, dp, 0, st>>>(p);
   else if (p.smooth_v) quant_pass1_kernel<T, false, true><<<grid1, dp, 0, st>>>(p);
   else quant_pass1_kernel<T, false, false><<<grid1, dp, 0, st>>>(p);
-  quant_finalize_kernel<<<B * Hkv, dp, 0, st>>>(p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  e = launch_dependent(quant_finalize_kernel, dim3(B * Hkv), dim3(dp), st, p);
+  if (e != cudaSuccess) return e;
   const dim3 grid2(p.nblk_k > 0 ? p.nblk_k : 1, 2 * Hkv, B);
-  if (p.smooth_v) quant_pass2_kernel<T, true><<<grid2, dp, 0, st>>>(p);
-  else quant_pass2_kernel<T, false><<<grid2, dp, 0, st>>>(p);
-  return cudaGetLastError();
+  return p.smooth_v ? launch_dependent(quant_pass2_kernel<T, true>, grid2, dim3(dp), st, p)
+                    : launch_dependent(quant_pass2_kernel<T, false>, grid2, dim3(dp), st, p);
 }
 
 cudaError_t launch_quantize(const QuantParams& p, cudaStream_t st) {
