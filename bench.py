@@ -139,8 +139,15 @@ def _flush(buf):
     buf.add_(1)
 
 
+HOST_AHEAD_CYCLES = 400_000  # ~0.2 ms of device-side sleep before each step's start event
+
+
 def time_steps(fn, steps, warmup, flush_buf):
-    """Per-step CUDA events on the current stream, L2 flushed before every step."""
+    """Per-step CUDA events on the current stream, L2 flushed before every step.
+
+    A short device-side sleep sits between the flush and the start event, so the device is still
+    busy while the host enqueues the step: the events then measure device time only, not the
+    host's launch latency (as when a program enqueues its steps ahead of the device)."""
     stream = torch.cuda.current_stream()
     for _ in range(warmup):
         _flush(flush_buf)
@@ -149,6 +156,7 @@ def time_steps(fn, steps, warmup, flush_buf):
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in ev:
         _flush(flush_buf)
+        torch.cuda._sleep(HOST_AHEAD_CYCLES)
         a.record(stream)
         fn()
         b.record(stream)
@@ -222,7 +230,8 @@ def _config(w):
             "layout": w.layout, "causal": w.causal, "pv_dtype": "fp16" if w.pv_mode & 2 else "fp8",
             "pv_accum": "fp16+fp32" if w.pv_mode & 1 else "fp32",
             "qk_quant_gran": {128: "per_block", 32: "per_warp", 1: "per_thread"}[w.q_gran], "smooth_v": w.smooth_v,
-            "values": w.dist, "l2": "flushed between steps (256 MiB write outside the events)"}
+            "values": w.dist, "l2": "flushed between steps (256 MiB write outside the events)",
+            "host": "each step enqueued while the device is busy (device sleep before the start event)"}
 
 
 def run_ours(args, w):

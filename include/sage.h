@@ -102,7 +102,10 @@ typedef struct {
  * creates on first use and that keeps its memory for later calls (it holds as
  * much device memory as the largest workspace in flight, until the process
  * exits); the workspace is released stream-ordered before return.
- * SAGE_ERR_OOM if it cannot be allocated.  out must not overlap q, k or v. */
+ * SAGE_ERR_OOM if it cannot be allocated.  out must not overlap q, k or v.
+ * The call may be captured in a CUDA graph (the workspace then becomes the
+ * graph's allocation nodes); the finalize / pass-2 / attention kernels are
+ * launched as programmatic dependents of the kernel before them. */
 sage_status sage_attn(const void* q, const void* k, const void* v, void* out, int B, int Hq, int Hkv, int N, int d,
                       sage_dtype dtype, sage_layout layout, int is_causal, float sm_scale, sage_pv_mode pv_mode,
                       void* stream);

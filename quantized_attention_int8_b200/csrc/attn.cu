@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     return;
   }
 
+  // launched as a programmatic dependent of the quantize pass: wait for it to finish (and its
+  // codes and scales to be visible) before anything below reads them
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   if (threadIdx.x == 0) {
     mbar_init(&bars->q_full, 1);
     for (int s = 0; s < C::ST; ++s) {
@@ -624,8 +627,19 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done[which]);
   if (e != cudaSuccess) return e;
   dim3 grid(p.nblk_q, p.m.Hq * p.n_vhalves, p.m.B);
-  kern<<<grid, 192, C::SMEM, st>>>(tq, tk, tv, p);
-  return cudaGetLastError();
+  // a programmatic dependent of whatever ran before on the stream (the quantize pass): the CTAs
+  // may start while it finishes and wait for it in griddepcontrol.wait
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = C::SMEM;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, tq, tk, tv, p);
 }
 
 template <int DQK, int DV, typename OutT, bool PV16>

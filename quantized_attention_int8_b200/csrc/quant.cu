@@ -377,6 +377,7 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 template <typename T, bool SMOOTH_V>
 __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
   __shared__ float red[8];
+  allow_next_grid();
   wait_for_previous_grid();  // the finalize kernel's K mean and V scales
   // Last-read-first: pass 1 read V after K and batch B-1 last, so those are the tiles most likely
   // still in L2 when this pass reads them again.

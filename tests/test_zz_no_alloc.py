@@ -58,3 +58,26 @@ def test_noalloc_rejects_workspace_beyond_the_static_array(lib):
     st = lib.capi.sage_attn_noalloc(fake, fake + (1 << 34), fake + (2 << 34), fake + (3 << 34), w.B, w.Hq, w.Hkv,
                                     w.N, w.d, lib.SAGE_FP16, lib.SAGE_HND, 1, 0.0, 0, None)
     assert st == lib.SAGE_ERR_INVALID_ARG
+
+
+def test_noalloc_captured_in_a_cuda_graph(lib):
+    # after one eager call (which looks the static array up), the allocation-free entry point
+    # can be captured and replayed
+    w = CASES[0]
+    q, k, v = (cuda(t) for t in W.make_inputs(w))
+    out = torch.empty_like(q)
+    assert _call(lib, lib.capi.sage_attn_noalloc, w, q, k, v, out) == lib.SAGE_OK
+    torch.cuda.synchronize()
+    ref = out.clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    with torch.cuda.graph(g, stream=s):
+        st = lib.capi.sage_attn_noalloc(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), w.B, w.Hq, w.Hkv,
+                                        w.N, w.d, _dt(lib, q), lib.SAGE_HND if w.layout == "HND" else lib.SAGE_NHD,
+                                        int(w.causal), float(W.sm_scale_of(w)), w.pv_mode, s.cuda_stream)
+    assert st == lib.SAGE_OK
+    out.zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    assert lib.capi.sage_check_status(torch.cuda.current_stream().cuda_stream) == lib.SAGE_OK
+    assert torch.equal(out.view(torch.int16), ref.view(torch.int16))
