@@ -267,6 +267,7 @@ def run_ours(args, w):
         times = time_steps(step, args.steps, args.warmup, flush)
     qa.sage_check_status()
     value, total_ms = job_throughput(sum(times), ops, args.steps, dist, "cuda")
+    step_stats = {"min_ms": min(times), "median_ms": statistics.median(times), "max_ms": max(times)}
 
     # ---- the fused attention kernel alone (roofline)
     z = qa.sage_quantize(qd, kd, vd, w.layout, pv, pvd, **okw)
@@ -332,8 +333,11 @@ def run_ours(args, w):
             "quantize": {"ms": q_ms, "algorithmic_bytes": q_bytes, "GB_per_s": q_bytes / (q_ms * 1e-3) / 1e9,
                          "hbm_peak_GB_per_s": peaks["hbm"], "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm"]},
             "cpu_baseline": cpu,
+            # d not in {64, 128, 256}: the kernels run on the zero-padded head dim
+            "padded_work_value": value * qa.padded_dim(w.d) / w.d if qa.padded_dim(w.d) != w.d else None,
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": in_bytes,
                     "d2h_bytes_per_step": out.numel() * out.element_size()},
+            "step_ms": step_stats,
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),
         }

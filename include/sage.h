@@ -190,6 +190,14 @@ sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t*
 sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int Hkv, int N, int d,
                           const int32_t* tiles, int n_tiles, int32_t* s_out, void* stream);
 
+/* Diagnostic for the failure path (no counterpart on the pages): launches one
+ * block whose bounded wait, the same wait every pipeline stage of the kernels
+ * uses, is on a barrier that nothing completes; it gives up after about
+ * budget_us microseconds (1 .. 100000) at the GPU's base clock, records the
+ * timeout and returns.  sage_check_status then reports SAGE_ERR_TIMEOUT, and
+ * the context stays usable.  SAGE_ERR_INVALID_ARG for a budget out of range. */
+sage_status sage_selftest_wait_timeout(int budget_us, void* stream);
+
 /* Synchronizes `stream`, then reports (and clears) the device-side error word:
  * SAGE_ERR_TIMEOUT if a kernel gave up on a bounded wait, SAGE_ERR_INVALID_ARG
  * for a flagged tile record, SAGE_ERR_CUDA for a pending CUDA error. */

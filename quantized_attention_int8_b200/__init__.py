@@ -95,6 +95,7 @@ def _load() -> ctypes.CDLL:
         "sage_device_supported": ([], I),
         "sage_attn_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
         "sage_attn_ex": ([P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P, P], I),
+        "sage_selftest_wait_timeout": ([I, P], I),
         "sage_attn_varlen": ([P, P, P, P, P, P, I, I, I, ctypes.c_longlong, ctypes.c_longlong, I, I, I, I, I, F, I, P,
                               P], I),
     }

@@ -496,6 +496,16 @@ sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int
   return from_cuda(launch_qk_dump(tq, tk, p, m.dp, static_cast<cudaStream_t>(stream)));
 }
 
+sage_status sage_selftest_wait_timeout(int budget_us, void* stream) {
+  if (budget_us < 1 || budget_us > 100000) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_device();
+  if (s != SAGE_OK) return s;
+  int dev = 0, khz = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev) != cudaSuccess || khz <= 0) return SAGE_ERR_CUDA;
+  return from_cuda(launch_wait_probe((long long)budget_us * (khz / 1000), static_cast<cudaStream_t>(stream)));
+}
+
 sage_status sage_check_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return SAGE_ERR_CUDA;

@@ -735,6 +735,25 @@ cudaError_t launch_seq_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int
   return cudaGetLastError();
 }
 
+// Failure-path check: one thread waits, with the library's bounded wait, on an mbarrier that
+// nothing completes.  The wait runs out after `budget_cycles`, records SAGE_DEVERR_TIMEOUT and
+// returns, exactly as a stalled pipeline stage of the fused kernel would.
+__global__ void sage_wait_probe_kernel(long long budget_cycles) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    mbar_wait(&bar, 0, &abort_flag, budget_cycles, 1000u /* re-check every ~1 us */);
+  }
+}
+
+cudaError_t launch_wait_probe(long long budget_cycles, cudaStream_t st) {
+  sage_wait_probe_kernel<<<1, 32, 0, st>>>(budget_cycles);
+  return cudaGetLastError();
+}
+
 cudaError_t read_clear_device_error(int* value) {
   cudaError_t e = cudaMemcpyFromSymbol(value, g_device_error, sizeof(int));
   if (e != cudaSuccess) return e;

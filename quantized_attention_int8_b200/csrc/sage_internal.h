@@ -132,6 +132,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 cudaError_t launch_seq_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int max_q, int max_k,
                             long long total_q, long long total_k, SeqDesc* seqs, cudaStream_t st);
 cudaError_t read_clear_device_error(int* value);
+cudaError_t launch_wait_probe(long long budget_cycles, cudaStream_t st);
 cudaError_t launch_qk_dump(const CUtensorMap& tq, const CUtensorMap& tk, const QkDumpParams& p, int dp,
                            cudaStream_t st);
 

@@ -76,13 +76,15 @@ constexpr uint32_t kSuspendHintNs = 1000000;  // 1 ms per suspension; the budget
 
 // Bounded wait for the phase with the given parity.  Returns false (and
 // records a timeout) if the budget runs out or *abort is already set.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
+                                          long long budget_cycles = kWaitBudgetCycles,
+                                          uint32_t hint_ns = kSuspendHintNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
-    if (mbar_try_wait_suspend(bar, parity, kSuspendHintNs)) return true;
+    if (mbar_try_wait_suspend(bar, parity, hint_ns)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) {
+    if (clock64() - t0 > budget_cycles) {
       atomicOr(&g_device_error, SAGE_DEVERR_TIMEOUT);
       *abort = 1;
       return false;

@@ -108,6 +108,11 @@ def test_pv_mode_names(lib):
             lib.pv_mode(*bad)
 
 
+def test_selftest_budget_checks(lib):
+    assert lib.capi.sage_selftest_wait_timeout(0, None) == lib.SAGE_ERR_INVALID_ARG
+    assert lib.capi.sage_selftest_wait_timeout(100001, None) == lib.SAGE_ERR_INVALID_ARG
+
+
 def test_opts_names(lib):
     assert (lib.opts().q_gran, lib.opts().smooth_v) == (128, 0)
     assert (lib.opts("per_warp", True).q_gran, lib.opts("per_warp", True).smooth_v) == (32, 1)
