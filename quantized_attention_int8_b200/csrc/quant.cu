@@ -23,6 +23,8 @@
 // vector cv = t % (dp/8) (channels 8cv .. 8cv+7)", loaded as sixteen 16-byte
 // vectors.  The K token sum of a block is the pairwise tree over its 8 group
 // sums, each group summed token by token.
+#include <algorithm>
+
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
@@ -121,6 +123,30 @@ __device__ __forceinline__ void load_tile(uint4 (&v)[16], const T* __restrict__ 
   }
 }
 
+// Prefetch of the next block's tile (vector path only): the same 16 x 16-byte loads as load_tile,
+// issued as asynchronous copies into this thread's slots of `stage` (slot r of thread t at
+// stage[r * blockDim.x + t]); tokens past `rows` and channels past d are zero-filled.
+__device__ __forceinline__ void prefetch_tile(uint4* stage, const void* x0, long long tok_stride_bytes, int d,
+                                              int rows, const TileCoord& tc) {
+  const unsigned char* base = static_cast<const unsigned char*>(x0);
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    const int n = tc.g * 16 + r;
+    const bool valid = n < rows && tc.c0 < d;
+    const unsigned char* src = valid ? base + (size_t)n * tok_stride_bytes + tc.c0 * 2 : base;
+    const uint32_t dst = static_cast<uint32_t>(__cvta_generic_to_shared(stage + r * blockDim.x + threadIdx.x));
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(valid ? 16 : 0)
+                 : "memory");
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+
+__device__ __forceinline__ void take_prefetched(uint4 (&v)[16], const uint4* stage) {
+  asm volatile("cp.async.wait_group 0;" ::: "memory");
+#pragma unroll
+  for (int r = 0; r < 16; ++r) v[r] = stage[r * blockDim.x + threadIdx.x];
+}
+
 __device__ __forceinline__ float block_max(float v, float* red) {
   for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
   const int w = threadIdx.x >> 5, nw = blockDim.x >> 5;
@@ -203,23 +229,42 @@ __device__ __forceinline__ float tree8_min(const float* part, int dp, int c) {
 // FINE_Q: Q scales per token or per 32 tokens (else per 128-token block); SMOOTH_V: V's token
 // mean is subtracted before coding (pass 1 then gathers V's column sums, max and min).  Separate
 // instances keep the default path's register count (and occupancy) as low as before.
+// Each CTA handles up to p.bpc consecutive 128-token blocks of one head; with p.prefetch the next
+// block's tile streams into shared memory (cp.async) while the current one is processed.
 template <typename T, bool FINE_Q, bool SMOOTH_V>
-__global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
+__global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
   allow_next_grid();
+  extern __shared__ uint4 stage[];  // p.prefetch: 16 slots per thread
   __shared__ float red[8];
   __shared__ float part[8 * 256];
-  const int blk = blockIdx.x, y = blockIdx.y, b = blockIdx.z;
+  const int y = blockIdx.y, b = blockIdx.z;
   const SeqView sv = seq_view(p.m, b);
-  const int n0 = blk * 128;
-  const int rows = min(128, (y < p.m.Hq ? sv.nq : sv.nk) - n0);
-  if (rows <= 0) return;  // past the end of this sequence (the whole CTA leaves)
   const int dp = p.m.dp, d = p.m.d;
   const TileCoord tc = tile_coord(dp);
+  // this CTA's head: its tokens in the caller's tensor
+  const T* src;
+  long long tstride;
+  int ntok;
+  bool vec;
+  if (y < p.m.Hq) {
+    src = static_cast<const T*>(p.q) + sv.q_in + y * sv.q_head, tstride = sv.q_tok, ntok = sv.nq, vec = p.vec_q;
+  } else if (y < p.m.Hq + p.m.Hkv) {
+    src = static_cast<const T*>(p.k) + sv.k_in + (y - p.m.Hq) * sv.k_head, tstride = sv.k_tok, ntok = sv.nk;
+    vec = p.vec_k;
+  } else {
+    src = static_cast<const T*>(p.v) + sv.k_in + (y - p.m.Hq - p.m.Hkv) * sv.k_head, tstride = sv.k_tok;
+    ntok = sv.nk, vec = p.vec_v;
+  }
+  const int blk0 = blockIdx.x * p.bpc, blk1 = min((ntok + 127) / 128, blk0 + p.bpc);
+  if (blk0 >= blk1) return;  // past the end of this sequence (the whole CTA leaves)
   uint4 v[16];
+  load_tile<T>(v, src + (long long)blk0 * 128 * tstride, tstride, d, min(128, ntok - blk0 * 128), vec, tc);
+  for (int blk = blk0; blk < blk1; ++blk) {
+  const int n0 = blk * 128, rows = min(128, ntok - n0);
+  const bool pref = p.prefetch && vec && blk + 1 < blk1;
+  if (pref) prefetch_tile(stage, src + (long long)(n0 + 128) * tstride, tstride * 2, d, min(128, ntok - n0 - 128), tc);
   if (y < p.m.Hq) {  // ---- Q: final INT8 codes and per-block scale
     const int h = y;
-    load_tile<T>(v, static_cast<const T*>(p.q) + sv.q_in + h * sv.q_head + n0 * sv.q_tok, sv.q_tok, d, rows, p.vec_q,
-                 tc);
     const long long row = sv.q_row0 + h * p.m.q_head_rows + n0;
     if (!FINE_Q) {  // one scale for the 128-token block
       const float am = block_max(tile_absmax<T>(v), red);
@@ -258,8 +303,6 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
     }
   } else if (y < p.m.Hq + p.m.Hkv) {  // ---- K: per-block partial column sums
     const int h = y - p.m.Hq;
-    load_tile<T>(v, static_cast<const T*>(p.k) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_k,
-                 tc);
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f;
@@ -275,8 +318,6 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
     p.ksum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
   } else if (SMOOTH_V) {  // ---- V, smoothed: per-block partial column sums, max and min
     const int h = y - p.m.Hq - p.m.Hkv;
-    load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
-                 tc);
     float acc[8], hi[8], lo[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.f, hi[e] = -INFINITY, lo[e] = INFINITY;
@@ -307,8 +348,6 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
     p.vmin_part[base + threadIdx.x] = tree8_min(part, dp, threadIdx.x);
   } else {  // ---- V: per-block partial column amax
     const int h = y - p.m.Hq - p.m.Hkv;
-    load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
-                 tc);
     uint32_t a[4] = {0, 0, 0, 0};  // channels (2e, 2e+1), |x| as bit patterns
 #pragma unroll
     for (int r = 0; r < 16; ++r) {
@@ -325,6 +364,14 @@ __global__ void __launch_bounds__(256) quant_pass1_kernel(QuantParams p) {
     __syncthreads();
     const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
     p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
+  }
+  __syncthreads();  // `part` and `red` are reused by the next block
+  if (blk + 1 < blk1) {
+    if (pref)
+      take_prefetched(v, stage);
+    else
+      load_tile<T>(v, src + (long long)(n0 + 128) * tstride, tstride, d, min(128, ntok - n0 - 128), vec, tc);
+  }
   }
 }
 
@@ -375,27 +422,35 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
 }
 
 template <typename T, bool SMOOTH_V>
-__global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
+__global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
+  extern __shared__ uint4 stage[];  // p.prefetch: 16 slots per thread
   __shared__ float red[8];
   allow_next_grid();
   wait_for_previous_grid();  // the finalize kernel's K mean and V scales
   // Last-read-first: pass 1 read V after K and batch B-1 last, so those are the tiles most likely
   // still in L2 when this pass reads them again.
-  const int blk = gridDim.x - 1 - blockIdx.x, y = gridDim.y - 1 - blockIdx.y, b = gridDim.z - 1 - blockIdx.z;
+  const int y = gridDim.y - 1 - blockIdx.y, b = gridDim.z - 1 - blockIdx.z;
   const SeqView sv = seq_view(p.m, b);
-  const int n0 = blk * 128, rows = min(128, sv.nk - n0);
-  if (rows <= 0) return;  // past the end of this sequence (the whole CTA leaves)
   const int dp = p.m.dp, d = p.m.d;
   const TileCoord tc = tile_coord(dp);
+  const bool isk = y < p.m.Hkv;
+  const T* src = static_cast<const T*>(isk ? p.k : p.v) + sv.k_in + (isk ? y : y - p.m.Hkv) * sv.k_head;
+  const long long tstride = sv.k_tok;
+  const bool vec = isk ? p.vec_k : p.vec_v;
+  const int blk0 = (gridDim.x - 1 - blockIdx.x) * p.bpc, blk1 = min((sv.nk + 127) / 128, blk0 + p.bpc);
+  if (blk0 >= blk1) return;  // past the end of this sequence (the whole CTA leaves)
   uint4 v[16];
+  load_tile<T>(v, src + (long long)blk0 * 128 * tstride, tstride, d, min(128, sv.nk - blk0 * 128), vec, tc);
+  for (int blk = blk0; blk < blk1; ++blk) {
+  const int n0 = blk * 128, rows = min(128, sv.nk - n0);
+  const bool pref = p.prefetch && vec && blk + 1 < blk1;
+  if (pref) prefetch_tile(stage, src + (long long)(n0 + 128) * tstride, tstride * 2, d, min(128, sv.nk - n0 - 128), tc);
   if (y < p.m.Hkv) {  // ---- K - mean(K): INT8 codes and per-block scale
     const int h = y;
     const size_t bh = (size_t)b * p.m.Hkv + h;
     float km[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) km[e] = p.km[bh * dp + tc.c0 + e];
-    load_tile<T>(v, static_cast<const T*>(p.k) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_k,
-                 tc);
     // padded channels read 0 and have mean 0; padded rows are masked by store_int8_tile
     auto x = [&](int r, int e) -> float { return __fsub_rn(elem<T>(v[r], e), km[e]); };
     // max |k - mean| per channel is reached at the channel's largest or smallest k, since
@@ -443,8 +498,6 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
     for (int e = 0; e < 8; ++e) inv[e] = p.vinv[bh * dp + tc.c0 + e];
 #pragma unroll
     for (int e = 0; e < 8; ++e) mean[e] = SMOOTH_V ? p.vm[bh * dp + tc.c0 + e] : 0.f;
-    load_tile<T>(v, static_cast<const T*>(p.v) + sv.k_in + h * sv.k_head + n0 * sv.k_tok, sv.k_tok, d, rows, p.vec_v,
-                 tc);
     // (v - mean) * inv; tokens past N give 0 (with smoothing the subtraction would not)
     auto vx = [&](int r, int e) -> float {
       if (!SMOOTH_V) return __fmul_rn(elem<T>(v[r], e), inv[e]);  // tokens past N load as 0 -> code 0
@@ -470,33 +523,41 @@ __global__ void __launch_bounds__(256) quant_pass2_kernel(QuantParams p) {
         dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
         dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
       }
-      return;
-    }
+    } else {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      uint32_t w[4];
+      for (int e = 0; e < 8; ++e) {
+        uint32_t w[4];
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float a0 = vx(4 * q + 0, e);
-        const float a1 = vx(4 * q + 1, e);
-        const float a2 = vx(4 * q + 2, e);
-        const float a3 = vx(4 * q + 3, e);
-        w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
+        for (int q = 0; q < 4; ++q) {
+          const float a0 = vx(4 * q + 0, e);
+          const float a1 = vx(4 * q + 1, e);
+          const float a2 = vx(4 * q + 2, e);
+          const float a3 = vx(4 * q + 3, e);
+          w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
+        }
+        *reinterpret_cast<uint4*>(p.v8t + (vrow + e) * pitch + vcol) = make_uint4(w[0], w[1], w[2], w[3]);
       }
-      *reinterpret_cast<uint4*>(p.v8t + (vrow + e) * pitch + vcol) =
-          make_uint4(w[0], w[1], w[2], w[3]);
     }
+  }
+  __syncthreads();  // `red` is reused by the next block
+  if (blk + 1 < blk1) {
+    if (pref)
+      take_prefetched(v, stage);
+    else
+      load_tile<T>(v, src + (long long)(n0 + 128) * tstride, tstride, d, min(128, sv.nk - n0 - 128), vec, tc);
+  }
   }
 }
 
 // Launch `kern` so that it may start while the previous kernel in the stream still runs (it
 // waits with griddepcontrol.wait before reading that kernel's output).
 template <typename K>
-static cudaError_t launch_dependent(K kern, dim3 grid, dim3 block, cudaStream_t st, const QuantParams& p) {
+static cudaError_t launch_dependent(K kern, dim3 grid, dim3 block, cudaStream_t st, const QuantParams& p,
+                                   size_t smem = 0) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
-  cfg.dynamicSmemBytes = 0;
+  cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -507,21 +568,34 @@ static cudaError_t launch_dependent(K kern, dim3 grid, dim3 block, cudaStream_t 
 }
 
 template <typename T>
-static cudaError_t launch_quant_t(const QuantParams& p, cudaStream_t st) {
+static cudaError_t launch_quant_t(const QuantParams& p_in, cudaStream_t st) {
+  QuantParams p = p_in;
   const int B = p.m.B, Hq = p.m.Hq, Hkv = p.m.Hkv, dp = p.m.dp;
-  const dim3 grid1(p.nblk_q > p.nblk_k ? p.nblk_q : p.nblk_k, Hq + 2 * Hkv, B);
+  const int nblk1 = p.nblk_q > p.nblk_k ? p.nblk_q : p.nblk_k;
+  // Blocks per CTA: with more than about four waves of blocks (some 8 CTAs resident per SM), each
+  // CTA walks a few consecutive blocks of its head, the next block's tile streaming in behind the
+  // current one (measured: 328 -> 305 us on a 604 MB pass); below that, one block per CTA (walking
+  // four blocks per CTA made a 113 MB pass slower, 60 -> 64 us).
+  int dev = 0, sms = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const long long blocks = (long long)nblk1 * (Hq + 2 * Hkv) * B, slots = (long long)sms * 8;
+  p.bpc = (int)std::min<long long>(8, std::max<long long>(1, blocks / (4 * slots)));
+  p.prefetch = (dp <= 128 && p.bpc > 1) ? 1 : 0;
+  const size_t smem = p.prefetch ? (size_t)dp * 16 * sizeof(uint4) : 0;  // 16 slots per thread
+  const dim3 grid1((nblk1 + p.bpc - 1) / p.bpc, Hq + 2 * Hkv, B);
   const bool fine = p.q_gran_log2 != 7;
-  if (fine && p.smooth_v) quant_pass1_kernel<T, true, true><<<grid1, dp, 0, st>>>(p);
-  else if (fine) quant_pass1_kernel<T, true, false><<<grid1, dp, 0, st>>>(p);
-  else if (p.smooth_v) quant_pass1_kernel<T, false, true><<<grid1, dp, 0, st>>>(p);
-  else quant_pass1_kernel<T, false, false><<<grid1, dp, 0, st>>>(p);
+  if (fine && p.smooth_v) quant_pass1_kernel<T, true, true><<<grid1, dp, smem, st>>>(p);
+  else if (fine) quant_pass1_kernel<T, true, false><<<grid1, dp, smem, st>>>(p);
+  else if (p.smooth_v) quant_pass1_kernel<T, false, true><<<grid1, dp, smem, st>>>(p);
+  else quant_pass1_kernel<T, false, false><<<grid1, dp, smem, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   e = launch_dependent(quant_finalize_kernel, dim3(B * Hkv), dim3(dp), st, p);
   if (e != cudaSuccess) return e;
-  const dim3 grid2(p.nblk_k > 0 ? p.nblk_k : 1, 2 * Hkv, B);
-  return p.smooth_v ? launch_dependent(quant_pass2_kernel<T, true>, grid2, dim3(dp), st, p)
-                    : launch_dependent(quant_pass2_kernel<T, false>, grid2, dim3(dp), st, p);
+  const int nblk2 = p.nblk_k > 0 ? p.nblk_k : 1;
+  const dim3 grid2((nblk2 + p.bpc - 1) / p.bpc, 2 * Hkv, B);
+  return p.smooth_v ? launch_dependent(quant_pass2_kernel<T, true>, grid2, dim3(dp), st, p, smem)
+                    : launch_dependent(quant_pass2_kernel<T, false>, grid2, dim3(dp), st, p, smem);
 }
 
 cudaError_t launch_quantize(const QuantParams& p, cudaStream_t st) {

@@ -98,6 +98,8 @@ struct QuantParams {
   float* vm;         // [B][Hkv][dp] V's token mean (nullptr allowed when smooth_v is 0)
   int smooth_v;      // code V - vm instead of V
   int q_gran_log2;   // query tokens per Q scale: 7 (128), 5 (32) or 0 (1)
+  int bpc;           // 128-token blocks per CTA of the two passes (grid x = ceil(blocks / bpc))
+  int prefetch;      // stream the next block into shared memory while one is processed (dp <= 128)
   float vmax_code;   // 448 (FP8 P.V, fp32 accumulation) or 1 (the other P.V modes)
   int v_fp16;        // V codes are fp16 (FP16 P.V) instead of E4M3; v8t then holds 2 bytes per code
 };
