@@ -29,6 +29,7 @@ __all__ = [
     "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
     "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
     "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode", "sage_attn_varlen", "SageOpts", "opts",
+    "sageattn", "sageattn_qk_int8_pv_fp8_cuda", "sageattn_qk_int8_pv_fp16_cuda", "sageattn_varlen",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
@@ -328,3 +329,34 @@ def sage_check_status() -> None:
 
 def sage_device_supported() -> bool:
     return bool(capi.sage_device_supported())
+
+
+# ---------------------------------------------------------------------------------------------
+# The entry-point names of the SageAttention README ("How to Use": sageattn(q, k, v,
+# tensor_layout="HND", is_causal=False); "Available APIs": the INT8-QK kernels with FP8 or FP16
+# P.V and the varlen one), mapped onto the calls above.
+# ---------------------------------------------------------------------------------------------
+def sageattn(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None, **kw):
+    """sage_attn under the README's name (FP8 P.V with fp32 accumulation unless told otherwise)."""
+    return sage_attn(q, k, v, tensor_layout, is_causal, sm_scale, **kw)
+
+
+def sageattn_qk_int8_pv_fp8_cuda(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None,
+                                 pv_accum_dtype="fp32", qk_quant_gran="per_block", smooth_v=False, out=None):
+    """INT8 Q.K^T and FP8 (E4M3) P.V; pv_accum_dtype "fp32" or "fp16+fp32" / "fp32+fp16"."""
+    return sage_attn(q, k, v, tensor_layout, is_causal, sm_scale, pv_accum_dtype, out=out, pv_dtype="fp8",
+                     qk_quant_gran=qk_quant_gran, smooth_v=smooth_v)
+
+
+def sageattn_qk_int8_pv_fp16_cuda(q, k, v, tensor_layout="HND", is_causal=False, sm_scale=None,
+                                  pv_accum_dtype="fp32", qk_quant_gran="per_block", smooth_v=False, out=None):
+    """INT8 Q.K^T and FP16 P.V; pv_accum_dtype "fp32", "fp16+fp32" or "fp16" (see pv_mode)."""
+    return sage_attn(q, k, v, tensor_layout, is_causal, sm_scale, pv_accum_dtype, out=out, pv_dtype="fp16",
+                     qk_quant_gran=qk_quant_gran, smooth_v=smooth_v)
+
+
+def sageattn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, is_causal=False, sm_scale=None,
+                    pv_dtype="fp16", **kw):
+    """sage_attn_varlen under the README's name; FP16 P.V by default, as the README lists it."""
+    return sage_attn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, is_causal, sm_scale,
+                            pv_dtype=pv_dtype, **kw)

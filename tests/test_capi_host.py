@@ -119,3 +119,13 @@ def test_opts_names(lib):
     assert lib.opts("per_thread").q_gran == 1
     with pytest.raises(ValueError):
         lib.opts("per_channel")
+
+
+def test_readme_entry_point_names(lib):
+    import inspect
+    for name in ("sageattn", "sageattn_qk_int8_pv_fp8_cuda", "sageattn_qk_int8_pv_fp16_cuda", "sageattn_varlen"):
+        assert callable(getattr(lib, name)) and name in lib.__all__
+    sig = inspect.signature(lib.sageattn)
+    assert list(sig.parameters)[:6] == ["q", "k", "v", "tensor_layout", "is_causal", "sm_scale"]
+    assert sig.parameters["tensor_layout"].default == "HND" and sig.parameters["is_causal"].default is False
+    assert inspect.signature(lib.sageattn_varlen).parameters["pv_dtype"].default == "fp16"

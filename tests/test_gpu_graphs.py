@@ -37,3 +37,19 @@ def test_sage_attn_captured_in_a_cuda_graph(lib, w):
     call(eager)
     lib.sage_check_status()
     assert torch.equal(out.view(torch.int16), eager.view(torch.int16))
+
+
+def test_readme_names_are_the_same_calls(lib):
+    w = W.TINY.with_(name="names", N=300, Hq=4, Hkv=2, causal=True)
+    q, k, v = (cuda(t) for t in W.make_inputs(w))
+    same = lambda a, b: torch.equal(a.view(torch.int16), b.view(torch.int16))
+    assert same(lib.sageattn(q, k, v, "HND", True), lib.sage_attn(q, k, v, "HND", True))
+    assert same(lib.sageattn_qk_int8_pv_fp8_cuda(q, k, v, is_causal=True, pv_accum_dtype="fp32+fp16"),
+                lib.sage_attn(q, k, v, "HND", True, None, "fp16+fp32"))
+    assert same(lib.sageattn_qk_int8_pv_fp16_cuda(q, k, v, is_causal=True),
+                lib.sage_attn(q, k, v, "HND", True, pv_dtype="fp16"))
+    cu = torch.tensor([0, 100, 300], dtype=torch.int32, device="cuda")
+    qp, kp, vp = (t[0].transpose(0, 1).contiguous() for t in (q, k, v))
+    assert same(lib.sageattn_varlen(qp, kp, vp, cu, cu, 200, 200, True),
+                lib.sage_attn_varlen(qp, kp, vp, cu, cu, 200, 200, True, pv_dtype="fp16"))
+    lib.sage_check_status()
