@@ -62,7 +62,12 @@ def test_quantize_bit_exact_small(lib, w):
     _assert_same(got, ref)
 
 
-FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"], W.FP16_PV[1]]
+FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"], W.FP16_PV[1],
+        # more than four waves of 128-token blocks: CTAs walk several blocks (ragged last block),
+        # with the next tile prefetched (16-byte rows) or loaded synchronously (d = 33)
+        W.TINY.with_(name="multiblock_prefetch_ragged_d64", B=4, Hq=8, Hkv=8, N=16381, d=64),
+        W.TINY.with_(name="multiblock_sync_d33_nhd_smoothv", B=4, Hq=8, Hkv=8, N=16300, d=33, layout="NHD",
+                     smooth_v=True, q_gran=32)]
 
 
 @pytest.mark.parametrize("w", FULL, ids=lambda w: w.name)
@@ -74,6 +79,6 @@ def test_quantize_bit_exact_full_size_sampled_heads(lib, w):
     for b, hk in {(0, 0), (w.B - 1, w.Hkv - 1)}:
         hq = list(range(hk * G, (hk + 1) * G))
         ref = quant.quantize(slice_heads(q, w.layout, b, hq), slice_heads(k, w.layout, b, [hk]),
-                             slice_heads(v, w.layout, b, [hk]), w.layout, w.pv_mode)
+                             slice_heads(v, w.layout, b, [hk]), w.layout, w.pv_mode, w.q_gran, w.smooth_v)
         _assert_same(got, ref, q_sel=(slice(b, b + 1), slice(hk * G, (hk + 1) * G)),
                      kv_sel=(slice(b, b + 1), slice(hk, hk + 1)))
