@@ -13,8 +13,11 @@ B=2, H=24, N=4096, d=64, bf16, HND, non-causal, K with a per-channel offset.
 * ``roofline``: the fused attention kernel alone (sage_attn_quantized on the
   same buffers, per-launch CUDA events, L2 flushed) against the dense INT8/FP8
   tensor peak (2x the measured bf16 cuBLAS peak, the B200 nominal ratio).
-* ``e2e``: the same metric through the public API with pinned HOST buffers:
-  H2D of q, k, v and D2H of the output inside the timed region.
+* ``e2e``: the same metric through the public API (``sage_attn``) with pinned
+  HOST buffers: every step uploads q, k, v and downloads its output inside the
+  timed region.  ``value`` streams the steps (three CUDA streams, two device
+  buffer sets: step i+1's upload and step i-1's download overlap step i);
+  ``serial`` runs them one at a time with per-step events.
 * ``cpu_baseline``: the CPU oracle (exact fp64 attention) on a bounded sample
   of the same workload's heads, on this host's cores.
 * ``--impl reference``: there is no reference implementation to run; the
@@ -164,6 +167,54 @@ def time_steps(fn, steps, warmup, flush_buf):
     return [a.elapsed_time(b) for a, b in ev]
 
 
+def time_e2e_streamed(qh, kh, vh, attn, steps, warmup, flush_buf):
+    """Device time of `steps` end-to-end steps fed from pinned host memory: each step uploads
+    q, k, v, runs `attn(q, k, v, out)` and downloads out, on three streams with two device
+    buffer sets, so that uploads, compute and downloads of neighbouring steps overlap.  Events
+    bracket the whole stream (first upload to last download); returns its milliseconds."""
+    s_in, s_cmp, s_out = torch.cuda.Stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    nb = 2
+    dev = [[torch.empty(t.shape, dtype=t.dtype, device="cuda") for t in (qh, kh, vh)] for _ in range(nb)]
+    douts = [torch.empty(qh.shape, dtype=qh.dtype, device="cuda") for _ in range(nb)]
+    houts = [torch.empty(qh.shape, dtype=qh.dtype).pin_memory() for _ in range(nb)]
+
+    def run(n, start=None, end=None):
+        up = [torch.cuda.Event() for _ in range(n)]
+        done = [torch.cuda.Event() for _ in range(n)]
+        down = [torch.cuda.Event() for _ in range(n)]
+        if start is not None:
+            start.record(s_in)
+        for i in range(n):
+            j = i % nb
+            with torch.cuda.stream(s_in):
+                if i >= nb:
+                    s_in.wait_event(done[i - nb])  # buffer set j's inputs consumed
+                for d, h in zip(dev[j], (qh, kh, vh)):
+                    d.copy_(h, non_blocking=True)
+                up[i].record(s_in)
+            with torch.cuda.stream(s_cmp):
+                s_cmp.wait_event(up[i])
+                if i >= nb:
+                    s_cmp.wait_event(down[i - nb])  # buffer set j's output read back
+                _flush(flush_buf)
+                attn(*dev[j], douts[j])
+                done[i].record(s_cmp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(done[i])
+                houts[j].copy_(douts[j], non_blocking=True)
+                down[i].record(s_out)
+        if end is not None:
+            end.record(s_out)  # after the last download, which follows every other step's work
+
+    torch.cuda.synchronize()
+    run(warmup)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    run(steps, a, b)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
 def cpu_oracle_sample(w: W.Workload, budget_s: float):
     """Exact fp64 attention (the oracle) on successive (b, hq) heads until the time budget is used."""
     from oracle import attention
@@ -311,8 +362,14 @@ def run_ours(args, w):
         o = qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv, pv_dtype=pvd, **okw)
         outh.copy_(o, non_blocking=True)
 
+    # one step at a time (copy in, compute, copy out), per-step events: the latency of a call
     etimes = time_steps(e2e_step, args.steps, args.warmup, flush)
-    e2e_value, e_ms = job_throughput(sum(etimes), ops, args.steps, dist, "cuda")
+    serial_value, serial_ms = job_throughput(sum(etimes), ops, args.steps, dist, "cuda")
+    # a stream of steps (the throughput of a job that feeds batches from host memory)
+    e_ms = time_e2e_streamed(qh, kh, vh, lambda a, b, c, o: qa.sage_attn(a, b, c, w.layout, w.causal, scale, pv, out=o,
+                                                                          pv_dtype=pvd, **okw),
+                             args.steps, args.warmup, flush)
+    e2e_value, e_ms = job_throughput(e_ms, ops, args.steps, dist, "cuda")
 
     line = None
     if rank == 0:
@@ -336,7 +393,12 @@ def run_ours(args, w):
             # d not in {64, 128, 256}: the kernels run on the zero-padded head dim
             "padded_work_value": value * qa.padded_dim(w.d) / w.d if qa.padded_dim(w.d) != w.d else None,
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": in_bytes,
-                    "d2h_bytes_per_step": out.numel() * out.element_size()},
+                    "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e_ms / args.steps,
+                    "mode": "streamed: every step copies its q, k, v from pinned host memory and its output back "
+                            "inside the timed region; step i+1's upload and step i-1's download overlap step i "
+                            "(three streams, two device buffer sets, L2 flushed before each step's compute)",
+                    "serial": {"value": serial_value, "ms_per_step": serial_ms / args.steps,
+                               "mode": "one step at a time: upload, compute, download, per-step events"}},
             "step_ms": step_stats,
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),
