@@ -324,6 +324,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     const float* ksp = p.ks + (sv.k_row0 + (long long)hkv * p.m.k_head_rows) / 128;
     unsigned char* prow = sP + row * C::ROWB;
     float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates the stored P values' scale
+    float ks_next = DQK == 64 ? ksp[0] : 0.f;  // d = 64: the next tile's K scale
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
       if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
@@ -339,8 +340,17 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
         if (lane == 0) mbar_arrive(&bars->s_free);
       }
 
-      // dequantization factor in the log2 domain
-      const float f = __fmul_rn(__fmul_rn(qsv, ksp[i * BN / 128]), p.scale_log2);  // K scale of the 128-key block
+      // dequantization factor in the log2 domain, with the K scale of the 128-key block; at d = 64
+      // that scale is loaded one tile ahead (measured +1.3% with FP8 P.V, +3.7% with FP16 P.V;
+      // 5% slower in the causal d = 128 instance, so the others load it here)
+      float ksv;
+      if constexpr (DQK == 64) {
+        ksv = ks_next;
+        if (i + 1 < n_kv) ks_next = ksp[(i + 1) * BN / 128];
+      } else {
+        ksv = ksp[i * BN / 128];
+      }
+      const float f = __fmul_rn(__fmul_rn(qsv, ksv), p.scale_log2);
       const int key0 = i * BN;
       const bool edge = (key0 + BN > nk) || (CAUSAL && key0 + BN - 1 > qt * 128 + koff);
       int lim = BN;  // this row sees the tile's columns c < lim (none if lim <= 0)
