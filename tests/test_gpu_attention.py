@@ -114,7 +114,7 @@ def test_rejects_bad_inputs(lib):
 
 FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"],
         W.BY_NAME["pad_sweep_b8_h16_n16384_d64_full"], W.BY_NAME["pad_sweep_b8_h16_n1024_d96_full"]] + W.FP16_PV + \
-    W.OPTIONS
+    W.OPTIONS + W.FP32_ACC
 
 
 def _rows(out, layout, b, h, rows):

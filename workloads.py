@@ -112,7 +112,10 @@ FP16_PV = [IMAGE_DIT.with_(name="image_dit_b2_h24_n4096_d64_pv16", pv_mode=2),
 OPTIONS = [IMAGE_DIT.with_(name="image_dit_b2_h24_n4096_d64_qthread_smoothv", q_gran=1, smooth_v=True),
            LLM_GQA.with_(name="llm_causal_gqa_b4_hq32_hkv8_n8192_d128_qwarp", q_gran=32)]
 
-ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV + OPTIONS
+# The video-DiT inputs with fp32 P.V accumulation (the default mode) instead of fp16+fp32.
+FP32_ACC = [VIDEO_DIT.with_(name="video_dit_b1_h24_n32768_d128_nhd_fp32acc", pv_mode=0)]
+
+ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV + OPTIONS + FP32_ACC
 BY_NAME = {w.name: w for w in ALL}
 
 
