@@ -1,0 +1,48 @@
+"""bench.py's reference arm (the CPU oracle timed on the host) and its JSON line, on CPU.
+
+Single process, and under torchrun with two ranks where rank 0 alone runs and prints.
+"""
+import json
+import os
+import socket
+import subprocess
+import sys
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+ARGS = ["--impl", "reference", "--workload", "tiny_b1_h2_n256_d64", "--steps", "1", "--warmup", "3"]
+
+
+def _lines(out: str):
+    return [json.loads(x) for x in out.splitlines() if x.startswith("{")]
+
+
+def _check(line, n_gpus):
+    assert line["impl"] == "reference"
+    assert line["unit"] == "TOPS" and line["value"] > 0 and line["higher_is_better"] is True
+    assert line["n_gpus"] == n_gpus and line["steps"] == 1 and line["warmup"] == 3
+    assert line["config"]["workload"] == "tiny_b1_h2_n256_d64"
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    assert line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"] == {"value": line["value"], "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert line["vs_baseline"] is None
+
+
+def test_reference_arm_single_process():
+    r = subprocess.run([sys.executable, "bench.py", *ARGS], cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _lines(r.stdout)
+    assert len(lines) == 1
+    _check(lines[0], 1)
+
+
+def test_reference_arm_two_ranks_prints_once():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        port = s.getsockname()[1]
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", "--nproc-per-node", "2",
+           "--master-addr", "127.0.0.1", "--master-port", str(port), "bench.py", "--gpus", "2", *ARGS]
+    r = subprocess.run(cmd, cwd=ROOT, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = _lines(r.stdout)
+    assert len(lines) == 1
+    _check(lines[0], 2)
