@@ -5,12 +5,9 @@ it predicts the error the method itself makes against exact attention, so a
 test can tell a kernel bug from the cost of 8-bit arithmetic.
 
 Steps, per (batch, query head, 128-row query block), over the key tiles in
-increasing order (the blockwise online softmax the fused kernels use;
-SageAttention README, "Current Features"; qwbw.cn article, pitfalls, for the
-``pv_accum_dtype`` options).  A key tile is 128 keys for FP8 P.V and 64 keys
-for FP16 P.V (the tile width is where the online softmax may move its
-reference and, with fp16+fp32 accumulation, how many keys one fp16 partial
-sums; the pages fix neither):
+increasing order (the blockwise online softmax; SageAttention README,
+"Current Features"; qwbw.cn article, pitfalls, for the ``pv_accum_dtype``
+options).  A key tile is ``tile`` keys, 128 by default: one INT8 K block.
 
 1. S = Q8 . K8^T exactly in integers (K8 holds codes of K - mean(K)).
 2. Dequantize in the log2 domain: s = S * f with
@@ -19,12 +16,13 @@ sums; the pages fix neither):
    j > i + (Nk - Nq) under the (bottom-right aligned) causal mask, are
    excluded; a row that sees no key at all outputs zeros.
 3. Online softmax against a reference max m: the reference moves to
-   m' = max(m, row max of s) only when that exceeds m by more than
-   tau = 2 (log2 units), else it stays (m' = m); p = 2^(s - m') <= 2^tau;
-   alpha = 2^(m - m') (1 when it stays); l = l * alpha + sum(p).  With
-   tau = 0 this is the textbook online softmax; tau = 2 is how the CUDA
-   kernel runs it (it rescales O only when the reference moves), and the
-   result is the same up to rounding because O and l share the reference.
+   m' = max(m, row max of s) when that exceeds m by more than ``tau``
+   (log2 units), else it stays (m' = m); p = 2^(s - m') <= 2^tau;
+   alpha = 2^(m - m') (1 when it stays); l = l * alpha + sum(p).
+   tau = 0 (the default) is the plain online softmax: the reference is
+   always the running max.  A larger tau is a lazy reference, which moves
+   (and rescales O) only when the running max has grown by more than tau;
+   O and l share the reference, so the result differs only in how P rounds.
 4. P is stored as E4M3(p * 448 * 2^-tau), so codes stay within +-448 (FP8
    P.V modes 0, 1), or as fp16(p) (FP16 P.V modes 2, 3).
 5. PV: modes 0 and 2 (fp32 accumulation) O = O * alpha + P . V;
@@ -43,21 +41,28 @@ from . import fp8
 from .quant import BLOCK, P_SCALE, PV_FP16, F32
 
 LOG2E = 1.4426950408889634
-TAU = 2.0  # reference-max slack of the CUDA kernel's online softmax (log2 units)
+TAU = 0.0  # the plain online softmax: the reference is the running max
 
 
-def kv_tile(pv_mode: int) -> int:
-    """Keys per online-softmax tile for a P.V mode: 128 (FP8 P.V) or 64 (FP16 P.V)."""
-    return 64 if pv_mode in PV_FP16 else BLOCK
+def lazy_reading(pv_mode: int) -> dict:
+    """The lazy-reference reading of steps 3-5 that the fused CUDA kernel takes: tau = 2 (O is
+    rescaled only when the running max has grown by more than 2 in log2 units) and key tiles of
+    128 keys for FP8 P.V, 64 for FP16 P.V (where a P row of fp16 values and a V^T row are each
+    128 bytes).  The pages fix neither; pass it as ``emulate(..., **lazy_reading(mode))``."""
+    return dict(tau=2.0, tile=64 if pv_mode in PV_FP16 else BLOCK)
 
 
-def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, tau: float = TAU):
+def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, tau: float = TAU,
+            tile: int = BLOCK):
     """Emulated output float32 (len(heads), len(q_blocks) * 128, d) in HND row order.
 
     ``qz`` is the dict from ``quant.quantize``.  ``heads`` lists (b, hq) pairs
     (default: all), ``q_blocks`` the 128-row query blocks (default: all).
-    Rows beyond N are returned as NaN.
+    ``tau`` and ``tile``: steps 3-5 (default: the plain online softmax over
+    128-key tiles).  Rows beyond N are returned as NaN.
     """
+    if tile not in (64, BLOCK):
+        raise ValueError("tile must be 64 or 128 keys")
     B, Hq, Hkv, N, d = qz["B"], qz["Hq"], qz["Hkv"], qz["N"], qz["d"]
     Nk = qz.get("Nk", N)
     off = Nk - N                      # causal: query i sees keys j <= i + off
@@ -69,7 +74,7 @@ def emulate(qz: dict, causal: bool, sm_scale: float, heads=None, q_blocks=None, 
     qbs = list(range(nb)) if q_blocks is None else list(q_blocks)
     c = F32(F32(sm_scale) * F32(LOG2E))
     fp16_pv = mode in PV_FP16
-    T = kv_tile(mode)
+    T = tile
     pscale = F32(1.0) if fp16_pv else F32(P_SCALE * 2.0 ** -tau)  # exact: 448 * 2^-tau
     out = np.full((len(hs), len(qbs) * BLOCK, d), np.nan, F32)
     for n, (b, h) in enumerate(hs):

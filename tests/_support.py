@@ -11,23 +11,33 @@ from oracle import quant
 # ---------------------------------------------------------------------------------------------
 # Tolerances
 #
-# * North-star accuracy: cosine similarity >= 0.999 against exact fp64 attention.
-# * The 9070XT bench of the trdm.cn article reports max |sage - sdpa| between 1e-1 and 1e-2;
-#   0.1 is asserted on rows that attend to >= 128 keys.  Rows with fewer keys (early rows under
-#   the causal mask) average only a few FP8 values: one E4M3 code of V is off by up to 2^-4
-#   relative, and the P code of each key by up to 2^-4 relative, so for any row
-#   |out - exact| <= 2^-4 max|V| + 2^-4 (1 + 2^-4) max|V| + (score error) < 2^-3 max|V|
-#   for these unit-scale inputs; that derived bound is asserted on every row.
-# * Against the CPU emulation of the method (same codes, same tile order): the only differences
-#   are the output rounding (bf16 half ulp = 2^-9 relative), float32 summation order and the
-#   GPU's ex2.approx (a few ulp).  The last one can, rarely, move p*448 across an E4M3
-#   rounding boundary (probability ~2^-17 per score), changing one P code by one step
-#   (<= 2^-3 of that p).  So >= 99.99% of elements must lie within 2^-7 |emul| + 2e-3, and
-#   every element within the per-row bound 2^-3 max|V|.
+# Against the CPU emulation of the method (same codes, the fused kernel's lazy-reference reading:
+# emulate(..., **emulate.lazy_reading(mode))): the only differences are the output rounding (bf16
+# half ulp = 2^-9 relative), float32 summation order and the GPU's ex2.approx (a few ulp).  The
+# last one can, rarely, move p*448 across an E4M3 rounding boundary (probability ~2^-17 per
+# score), changing one P code by one step (<= 2^-3 of that p).  So >= 99.99% of elements must lie
+# within 2^-7 |emul| + 2e-3, and every element within 2^-3 max|V| (one flipped code of a key whose
+# weight is close to 1).
+#
+# Against exact fp64 attention, anchored on the method's own error on the same rows:
+# * every element: |gpu - exact| <= |emul - exact| + 2^-7 |emul| + 2e-3 (>= 99.99% of elements;
+#   the rest within |emul - exact| + 2^-3 max|V|, the code flips above);
+# * cosine similarity >= 0.999 (inputs with x8 K outlier channels: the method itself can fall
+#   below it, as the shared per-block K scale grows; there >= cos(emul, exact) - 2e-4);
+# * the target accuracy, max |gpu - exact| <= 2e-2, for unit-variance inputs (Q, K, V ~ N(0, 1),
+#   K also with a per-channel offset, which smoothing removes): on every row with FP16 P.V, and
+#   on rows that see >= 512 keys with FP8 P.V.  The relaxation for FP8 P on shorter rows is the
+#   method's, not the kernel's: each E4M3 code of P and of V is off by up to 2^-4 relative, and a
+#   row that averages fewer keys averages that error less; the emulation alone reaches 0.028
+#   (tiny workload, 256 keys) and 0.031 (rows with 128..511 keys of the causal GQA workload),
+#   while every sampled row with >= 512 keys stays below 0.006.
+# Quantization codes, scales, K mean and int32 scores: bit-exact (other tests).
 # ---------------------------------------------------------------------------------------------
 COS_MIN = 0.999
-PAGES_MAX_ABS = 0.1
+TARGET_MAX_ABS = 2e-2
+FP8_TARGET_MIN_KEYS = 512
 TIGHT_REL, TIGHT_ABS, TIGHT_FRAC = 2.0 ** -7, 2e-3, 0.9999
+UNIT_VARIANCE = ("normal", "normal_koffset")
 
 
 def cos_sim(a, b) -> float:
@@ -36,31 +46,30 @@ def cos_sim(a, b) -> float:
     return float(a @ b / np.sqrt((a @ a) * (b @ b)))
 
 
-def check_vs_exact(out, ref, nkeys, vmax, what="", emul=None):
-    """out, ref: (..., rows, d) float64; nkeys: (rows,) number of visible keys of each row.
-
-    The 0.999 cosine bound is stated for unit-variance inputs.  For inputs
-    with K outlier channels (``emul`` given: the method's own output on the
-    same rows), a x8 channel inflates the shared per-block INT8 scale of K
-    and the method itself can fall below these bounds (both were measured on
-    unit-variance inputs); the GPU must then be at least as accurate as the
-    method: cos >= min(0.999, cos(emul, exact) - 2e-4) and, on rows with
-    >= 128 keys, max abs <= max(0.1, max |emul - exact| + 0.02).
-    """
+def check_vs_exact(out, ref, emul, nkeys, vmax, what="", dist="normal", pv_mode=0):
+    """out, ref, emul: (..., rows, d) float64 -- the GPU output, exact attention and the method's
+    emulation (lazy reading) on the same rows; nkeys: (rows,) visible keys of each row; dist: the
+    inputs' value recipe (workloads.py); pv_mode: the P.V mode.  Returns the measured figures."""
+    out, ref, emul = (np.asarray(x, np.float64) for x in (out, ref, emul))
     err = np.abs(out - ref)
+    own = np.abs(emul - ref)
     c = cos_sim(out, ref)
-    cmin = COS_MIN if emul is None else min(COS_MIN, cos_sim(emul, ref) - 2e-4)
+    cmin = COS_MIN if dist != "normal_koutlier" else min(COS_MIN, cos_sim(emul, ref) - 2e-4)
     assert c >= cmin, f"{what}: cosine {c:.6f} < {cmin:.6f}"
-    big = np.asarray(nkeys) >= 128
-    if big.any():
-        m = err[..., big, :].max()
-        bound = PAGES_MAX_ABS
-        if emul is not None:
-            bound = max(bound, float(np.abs(emul - ref)[..., big, :].max()) + 0.02)
-        assert m <= bound, f"{what}: max abs {m:.4f} > {bound:.4f} on rows with >= 128 keys"
-    m_all = err.max()
-    assert m_all <= 0.125 * vmax, f"{what}: max abs {m_all:.4f} > 2^-3 max|V| = {0.125 * vmax:.4f}"
-    return dict(cos=c, max_abs=float(m_all), max_abs_128=float(err[..., big, :].max()) if big.any() else 0.0)
+    band = own + TIGHT_REL * np.abs(emul) + TIGHT_ABS
+    frac = float((err <= band).mean())
+    assert frac >= TIGHT_FRAC, f"{what}: only {frac:.6f} of elements within the method's own error + " \
+                               f"2^-7|emul| + 2e-3 (worst excess {float((err - band).max()):.4g})"
+    worst = float((err - own).max())
+    assert worst <= 0.125 * vmax, f"{what}: {worst:.4f} beyond the method's own error > 2^-3 max|V|"
+    nk = np.asarray(nkeys)
+    rows = np.ones(len(nk), bool) if pv_mode & 2 else nk >= FP8_TARGET_MIN_KEYS
+    target = None
+    if dist in UNIT_VARIANCE and rows.any():
+        target = float(err[..., rows, :].max())
+        assert target <= TARGET_MAX_ABS, f"{what}: max abs {target:.4f} > {TARGET_MAX_ABS} on " \
+                                         f"{'all rows' if pv_mode & 2 else 'rows with >= 512 keys'}"
+    return dict(cos=c, max_abs=float(err.max()), max_abs_target_rows=target, frac_in_band=frac)
 
 
 def check_vs_emulation(out, emul, vmax, what=""):

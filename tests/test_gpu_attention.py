@@ -59,8 +59,8 @@ def test_attention_kernel_reproduces_method(lib, w):
     z = oracle_to_device(qz)
     out = lib.sage_attn_quantized(z, q.dtype, w.layout, w.causal, _scale(w), pv_name(w))
     lib.sage_check_status()
-    em = emulate.emulate(qz, w.causal, _scale(w)).reshape(w.B, w.Hq, -1, w.d)[:, :, :w.N]
-    check_vs_emulation(out_hnd(out, w.layout), em.astype(np.float64), vmax_of(v), w.name)
+    em = emulate.emulate(qz, w.causal, _scale(w), **emulate.lazy_reading(w.pv_mode)).reshape(w.B, w.Hq, -1, w.d)
+    check_vs_emulation(out_hnd(out, w.layout), em[:, :, :w.N].astype(np.float64), vmax_of(v), w.name)
 
 
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
@@ -70,11 +70,10 @@ def test_sage_attn_vs_exact_attention(lib, w):
                         **opt_kw(w))
     lib.sage_check_status()
     ref = attention.attention_f64(q, k, v, w.layout, w.causal, _scale(w))
-    em = None
-    if w.dist == "normal_koutlier":  # not unit-variance: compare with the method's own accuracy
-        qz = quant.quantize(q, k, v, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
-        em = emulate.emulate(qz, w.causal, _scale(w)).reshape(w.B, w.Hq, -1, w.d)[:, :, :w.N].astype(np.float64)
-    check_vs_exact(out_hnd(out, w.layout), ref, nkeys(w.N, w.causal), vmax_of(v), w.name, emul=em)
+    qz = quant.quantize(q, k, v, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
+    em = emulate.emulate(qz, w.causal, _scale(w), **emulate.lazy_reading(w.pv_mode)).reshape(w.B, w.Hq, -1, w.d)
+    check_vs_exact(out_hnd(out, w.layout), ref, em[:, :, :w.N], nkeys(w.N, w.causal), vmax_of(v), w.name, w.dist,
+                   w.pv_mode)
 
 
 @pytest.mark.parametrize("w", SMALL[:6] + SMALL[10:13] + SMALL[-5:], ids=lambda w: w.name)
@@ -143,9 +142,9 @@ def test_full_size_sampled_rows(lib, w):
         qs, ks, vs = (slice_heads(t, w.layout, b, [hh]) for t, hh in ((q, hq), (k, hk), (v, hk)))
         got = _rows(out, w.layout, b, hq, torch.as_tensor(rows))
         qz = quant.quantize(qs, ks, vs, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
-        em = emulate.emulate(qz, w.causal, _scale(w), heads=[(0, 0)], q_blocks=qbs)[0]
+        em = emulate.emulate(qz, w.causal, _scale(w), heads=[(0, 0)], q_blocks=qbs, **emulate.lazy_reading(w.pv_mode))[0]
         em = np.concatenate([em[i * 128:i * 128 + min(128, w.N - qb * 128)] for i, qb in enumerate(qbs)])
         check_vs_emulation(got, em.astype(np.float64), vmax_of(vs), f"{w.name} b{b} h{hq}")
         ref = attention.attention_f64(qs, ks, vs, w.layout, w.causal, _scale(w), heads=[(0, 0)], rows=rows)[0]
-        check_vs_exact(got, ref, nkeys(w.N, w.causal, rows), vmax_of(vs), f"{w.name} b{b} h{hq}",
-                       emul=em.astype(np.float64) if w.dist == "normal_koutlier" else None)
+        check_vs_exact(got, ref, em, nkeys(w.N, w.causal, rows), vmax_of(vs), f"{w.name} b{b} h{hq}", w.dist,
+                       w.pv_mode)

@@ -43,11 +43,12 @@ def test_rectangular_vs_method_and_exact(lib, w):
     lib.sage_check_status()
     got = out_hnd(out, w.layout)
     qz = quant.quantize(q, k, v, w.layout, w.pv_mode)
-    em = emulate.emulate(qz, w.causal, scale).reshape(w.B, w.Hq, -1, w.d)[:, :, :w.N].astype(np.float64)
+    em = emulate.emulate(qz, w.causal, scale, **emulate.lazy_reading(w.pv_mode)).reshape(w.B, w.Hq, -1, w.d)
+    em = em[:, :, :w.N].astype(np.float64)
     check_vs_emulation(got, em, vmax_of(v), w.name)
     ref = attention.attention_f64(q, k, v, w.layout, w.causal, scale)
     nk = _nkeys(w.N, w.nk, w.causal)
-    check_vs_exact(got, ref, nk, vmax_of(v), w.name)
+    check_vs_exact(got, ref, em, nk, vmax_of(v), w.name, w.dist, w.pv_mode)
     assert np.all(got[:, :, nk == 0] == 0), "rows that see no key must be zero"
 
 
@@ -85,10 +86,11 @@ def test_varlen_per_sequence_vs_method_and_exact(lib, w):
             continue
         qs, ks, vs = (t[c[b]:c[b + 1]][None] for t, c in ((q, cq), (k, ck), (v, ck)))  # (1, n, H, d)
         qz = quant.quantize(qs, ks, vs, "NHD", w.pv_mode)
-        em = emulate.emulate(qz, w.causal, scale).reshape(1, w.Hq, -1, w.d)[:, :, :nq].astype(np.float64)
+        em = emulate.emulate(qz, w.causal, scale, **emulate.lazy_reading(w.pv_mode)).reshape(1, w.Hq, -1, w.d)
+        em = em[:, :, :nq].astype(np.float64)
         check_vs_emulation(g, em, vmax_of(vs), f"{w.name} seq {b}")
         ref = attention.attention_f64(qs, ks, vs, "NHD", w.causal, scale)
-        check_vs_exact(g, ref, _nkeys(nq, nk, w.causal), vmax_of(vs), f"{w.name} seq {b}")
+        check_vs_exact(g, ref, em, _nkeys(nq, nk, w.causal), vmax_of(vs), f"{w.name} seq {b}", w.dist, w.pv_mode)
     # the whole packed output against the packed oracle definition as well
     ex = attention.attention_varlen_f64(q, k, v, cq.numpy(), ck.numpy(), w.causal, scale)
     assert np.abs(got - ex).max() <= 0.125 * float(v.float().abs().max())
@@ -154,10 +156,10 @@ def test_varlen_full_size_sampled_rows(lib):
             qs = q[cq[b]:cq[b + 1], hq:hq + 1][None]
             ks, vs = (t[ck[b]:ck[b + 1], hk:hk + 1][None] for t in (k, v))
             qz = quant.quantize(qs, ks, vs, "NHD", w.pv_mode)
-            em = emulate.emulate(qz, w.causal, scale, heads=[(0, 0)], q_blocks=qbs)[0]
+            em = emulate.emulate(qz, w.causal, scale, heads=[(0, 0)], q_blocks=qbs, **emulate.lazy_reading(w.pv_mode))[0]
             em = np.concatenate([em[i * 128:i * 128 + min(128, nq - qb * 128)] for i, qb in enumerate(qbs)])
             g = got[cq[b] + rows, hq]
             what = f"seq {b} ({nq}x{nk}) h{hq}"
             check_vs_emulation(g, em.astype(np.float64), vmax_of(vs), what)
             ref = attention.attention_f64(qs, ks, vs, "NHD", w.causal, scale, heads=[(0, 0)], rows=rows)[0]
-            check_vs_exact(g, ref, _nkeys(nq, nk, w.causal, rows), vmax_of(vs), what, emul=em.astype(np.float64))
+            check_vs_exact(g, ref, em, _nkeys(nq, nk, w.causal, rows), vmax_of(vs), what, w.dist, w.pv_mode)
