@@ -70,12 +70,21 @@ typedef enum { SAGE_FP16 = 0, SAGE_BF16 = 1, SAGE_FP32 = 2 } sage_dtype;
  *                       [-1, 1]); fp32 accumulation.  Key tiles of 64.
  *   SAGE_PV16_FP16_FP32 FP16 P and V; each 64-key tile's P.V in a fresh fp16
  *                       accumulator (|partial| <= 64 * 4 * 1), added into fp32 O.
- * Bit 0 of the value selects fp16+fp32 accumulation, bit 1 FP16 operands. */
+ *   SAGE_PV16_FP16      FP16 P and V accumulated in fp16 across all key tiles
+ *                       (pitfalls section: pv_accum_dtype "fp16", the fastest and
+ *                       least overflow-safe option on the GPUs the pages target).
+ *                       Not offered: every entry point returns
+ *                       SAGE_ERR_UNSUPPORTED.  On sm_100a a tcgen05.mma issues at the
+ *                       same rate with an F16 as with an F32 accumulator, so the
+ *                       mode would only add rounding error and overflow risk.
+ * Bit 0 of the value selects fp16+fp32 accumulation, bit 1 FP16 operands, bit 2
+ * pure fp16 accumulation. */
 typedef enum {
   SAGE_PV_FP32 = 0,
   SAGE_PV_FP16_FP32 = 1,
   SAGE_PV16_FP32 = 2,
-  SAGE_PV16_FP16_FP32 = 3
+  SAGE_PV16_FP16_FP32 = 3,
+  SAGE_PV16_FP16 = 6
 } sage_pv_mode;
 
 /* Optional quantization settings (SageAttention README, "Current Features":
@@ -160,8 +169,13 @@ size_t sage_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * Padded tokens and channels hold code 0 (and km 0, vs 0, vm 0).  Codes and scales
  * follow: amax over the block's real tokens and channels, inv = 127 / amax,
  * code = clamp(rint_even(x * inv), -127, 127), scale = amax / 127 (0 when amax
- * is 0); K is smoothed as x = k - km, km summed in fp32 block by block (tokens
- * in order inside a block, then the block sums in order) and divided by N;
+ * is 0); K is smoothed as x = k - km, km summed in fp32 in this order: each
+ * 128-token block is split into 8 groups of 16 consecutive tokens, each group is
+ * summed token by token from +0.0 (tokens >= N skipped), the block's partial is
+ * the pairwise tree ((g0 + g1) + (g2 + g3)) + ((g4 + g5) + (g6 + g7)), the block
+ * partials are added one by one in block order from +0.0, and the total is
+ * divided by (float)N with one IEEE division (every add and the division round
+ * to nearest even); the order is part of the bit-exact contract;
  * V: inv = VMAX / amax_channel, code = E4M3_rne_satfinite(v * inv) (FP8 modes)
  * or fp16_rne(v * inv) (FP16 modes), vs = amax / VMAX with VMAX = 448
  * (SAGE_PV_FP32) or 1 (the other modes); with smooth_v, v - vm in place of v
@@ -198,9 +212,25 @@ sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int
  * the context stays usable.  SAGE_ERR_INVALID_ARG for a budget out of range. */
 sage_status sage_selftest_wait_timeout(int budget_us, void* stream);
 
+/* Diagnostic (no counterpart on the pages): measures nothing itself, but launches
+ * one CTA per SM whose single thread issues `iters` x 4 back-to-back tcgen05.mma of
+ * M = 128, N = 256 and 32 bytes of K per operand row (kind 0: kind::i8, K = 32;
+ * kind 1: kind::f8f6f4 with E4M3 operands, K = 32; kind 2: kind::f16, K = 16) into
+ * one tensor-memory accumulator, and waits for them.  *ops receives the
+ * operations the launch performs (SMs x iters x 4 x 2 x 128 x 256 x K); the caller
+ * times the launch on `stream` (CUDA events) to get the GPU's tensor-core rate for
+ * that kind.  SAGE_ERR_INVALID_ARG for a kind outside 0..2, iters outside
+ * 1..1000000 or a NULL ops. */
+sage_status sage_mma_probe(int kind, int iters, double* ops, void* stream);
+
 /* Synchronizes `stream`, then reports (and clears) the device-side error word:
  * SAGE_ERR_TIMEOUT if a kernel gave up on a bounded wait, SAGE_ERR_INVALID_ARG
- * for a flagged tile record, SAGE_ERR_CUDA for a pending CUDA error. */
+ * for a flagged tile record or cu_seqlens table, SAGE_ERR_CUDA for a pending CUDA
+ * error.  The error word is one per device, not per stream: it collects the
+ * flags of every call on the current device since it was last read, whatever
+ * stream they ran on, and the first sage_check_status to read it (on any stream)
+ * reports and clears them.  Only `stream` is synchronized, so a call still
+ * running on another stream may flag an error after the read. */
 sage_status sage_check_status(void* stream);
 
 /* Static description of a status code. */
@@ -209,8 +239,17 @@ const char* sage_status_string(sage_status s);
 /* 1 if the current CUDA device can run this library (compute capability 10.0). */
 int sage_device_supported(void);
 
+/* Test hook for the failure paths (no counterpart on the pages): host-side
+ * injection, with no GPU fault and no device call.  fake_cc > 0: the device check
+ * reports that compute capability (major * 10 + minor) instead of querying the
+ * device -- 100 passes as a B200, anything else gives SAGE_ERR_ARCH; 0 restores the
+ * real query.  fail_allocs > 0: that many of the following workspace allocations
+ * fail with SAGE_ERR_OOM before touching the device (0 clears it).  Process-wide;
+ * not for use outside tests. */
+void sage_test_inject(int fake_cc, int fail_allocs);
+
 /* Largest workspace sage_attn_noalloc can hold: 64 MiB (for example B=2, H=24,
- * N=4096, d=64 needs about 38 MiB; sage_workspace_bytes() gives the exact need). */
+ * N=4096, d=64 with pv_mode SAGE_PV_FP32 needs about 38 MiB). */
 #define SAGE_NOALLOC_MAX_BYTES (64u << 20)
 
 /* sage_attn without any device allocation.  The paper has no counterpart: this
@@ -222,8 +261,12 @@ int sage_device_supported(void);
  *
  * Its workspace is one static device array of SAGE_NOALLOC_MAX_BYTES inside this
  * library: every GPU that loads the library holds that memory until the process
- * exits.  Problems whose workspace (sage_workspace_bytes) exceeds the maximum are
- * rejected with SAGE_ERR_INVALID_ARG before any GPU work.  The first call on each
+ * exits.  A call whose own workspace -- the quantized Q, K, V, their scales and
+ * the quantize pass's partial sums for these sizes and this pv_mode, default
+ * options -- exceeds the maximum is rejected with SAGE_ERR_INVALID_ARG before any
+ * GPU work.  sage_workspace_bytes() is an upper bound of that figure (it takes the
+ * largest P.V mode and options), so sizes it keeps within the maximum are always
+ * accepted.  The first call on each
  * device looks up the array's device address (cudaGetSymbolAddress) with that
  * device current; make that first call before any stream capture.  All calls
  * share the one array and it keeps the previous call's contents (every byte a call

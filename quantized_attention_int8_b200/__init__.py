@@ -38,24 +38,25 @@ SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_ARCH, SAGE_ERR_CUD
     SAGE_ERR_TIMEOUT = range(7)
 SAGE_HND, SAGE_NHD = 0, 1
 SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
-SAGE_PV_FP32, SAGE_PV_FP16_FP32, SAGE_PV16_FP32, SAGE_PV16_FP16_FP32 = 0, 1, 2, 3
+SAGE_PV_FP32, SAGE_PV_FP16_FP32, SAGE_PV16_FP32, SAGE_PV16_FP16_FP32, SAGE_PV16_FP16 = 0, 1, 2, 3, 6
 
 _LAYOUTS = {"HND": SAGE_HND, "NHD": SAGE_NHD}
 _DTYPES = {torch.float16: SAGE_FP16, torch.bfloat16: SAGE_BF16, torch.float32: SAGE_FP32}
 _PV = {("fp8", "fp32"): SAGE_PV_FP32, ("fp8", "fp16+fp32"): SAGE_PV_FP16_FP32,
        ("fp8", "fp32+fp16"): SAGE_PV_FP16_FP32,
        ("fp16", "fp32"): SAGE_PV16_FP32, ("fp16", "fp16+fp32"): SAGE_PV16_FP16_FP32,
-       ("fp16", "fp16"): SAGE_PV16_FP32}
+       ("fp16", "fp16"): SAGE_PV16_FP16}
 
 
 def pv_mode(pv_dtype: str = "fp8", pv_accum_dtype: str = "fp32") -> int:
     """The sage_pv_mode value for P.V operands ``pv_dtype`` and accumulation ``pv_accum_dtype``.
 
     "fp32+fp16" is the README's spelling of the two-level (fp16 tile, fp32 total)
-    accumulation of the FP8 kernel.  "fp16" (pure fp16 accumulation, offered for the
-    FP16 kernel as the fastest and least overflow-safe option) runs with the fp32 TMEM
-    accumulator: on sm_100a a tcgen05 MMA issues at the same rate with an F16 or an F32
-    accumulator, so fp16 accumulation would buy no speed and only add error.
+    accumulation of the FP8 kernel.  "fp16" (pure fp16 accumulation with FP16 operands,
+    the fastest and least overflow-safe option on the GPUs the pages target) maps to
+    SAGE_PV16_FP16, which the library rejects with SAGE_ERR_UNSUPPORTED: on sm_100a a
+    tcgen05 MMA issues at the same rate with an F16 or an F32 accumulator, so fp16
+    accumulation would buy no speed and only add error and overflow risk.
     """
     try:
         return _PV[(pv_dtype, pv_accum_dtype)]
@@ -97,6 +98,8 @@ def _load() -> ctypes.CDLL:
         "sage_attn_noalloc": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
         "sage_attn_ex": ([P, P, P, P, I, I, I, I, I, I, I, I, I, F, I, P, P], I),
         "sage_selftest_wait_timeout": ([I, P], I),
+        "sage_mma_probe": ([I, I, ctypes.POINTER(ctypes.c_double), P], I),
+        "sage_test_inject": ([I, I], None),
         "sage_attn_varlen": ([P, P, P, P, P, P, I, I, I, ctypes.c_longlong, ctypes.c_longlong, I, I, I, I, I, F, I, P,
                               P], I),
     }

@@ -3,6 +3,7 @@
 #include <cmath>
 #include <cstdint>
 #include <cstring>
+#include <atomic>
 #include <mutex>
 
 #include "sage_internal.h"
@@ -117,7 +118,14 @@ sage_status from_cuda(cudaError_t e) {
   return e == cudaErrorMemoryAllocation ? SAGE_ERR_OOM : SAGE_ERR_CUDA;
 }
 
+// Host-side failure injection (sage_test_inject): a compute capability reported instead of the
+// device's (0: query the device), and a number of workspace allocations to fail.
+std::atomic<int> g_fake_cc{0};
+std::atomic<int> g_fail_allocs{0};
+
 sage_status check_device() {
+  const int fake = g_fake_cc.load(std::memory_order_relaxed);
+  if (fake) return fake == 100 ? SAGE_OK : SAGE_ERR_ARCH;
   int dev = 0, major = 0, minor = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess) return SAGE_ERR_CUDA;
@@ -197,6 +205,8 @@ sage_status parse_opts(const sage_opts* o, Opts* out) {
 // memory it has handed out (release threshold = unlimited), so that repeated calls reuse
 // it instead of mapping fresh device memory each time.
 cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t st) {
+  for (int n = g_fail_allocs.load(); n > 0;)  // an injected failure, before any device call
+    if (g_fail_allocs.compare_exchange_weak(n, n - 1)) return cudaErrorMemoryAllocation;
   constexpr int kMaxDevices = 128;
   static std::mutex mu;
   static cudaMemPool_t pools[kMaxDevices] = {};
@@ -240,7 +250,7 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
                     int pv_mode, const Opts& o, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   const uint32_t ksub = m.dp >= 128 ? 128 : 64;
-  const uint32_t dv = m.dp == 64 ? 64 : 128;
+  const uint32_t dv = m.dp;  // V^T rows (channels) per tile: all of the padded head dim
   const bool pv16 = pv_mode_fp16_operands(pv_mode);
   const uint32_t bn = pv16 ? 64 : 128;  // keys per KV tile of the fused kernel
   const uint64_t vpitch = (uint64_t)m.k_head_rows * (pv16 ? 2 : 1);  // bytes per V^T row (one channel)
@@ -256,7 +266,6 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
   p.m = seq_map(m, layout, qb.seqs);
   p.nblk_q = m.nblk_q;
   p.G = m.G;
-  p.n_vhalves = m.dp == 256 ? 2 : 1;
   p.vec_out = (m.d % 8 == 0) && aligned16(out);
   p.scale_log2 = resolve_scale(sm_scale, m.d) * 1.4426950408889634f;
   return from_cuda(launch_fwd(tq, tk, tv, p, dtype, causal, pv_mode, st));
@@ -315,6 +324,7 @@ sage_status check_common(const void* q, const void* k, const void* v, int dtype,
   sage_status s = check_dtype(dtype);
   if (s != SAGE_OK) return s;
   if (layout != SAGE_HND && layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
+  if (pv_mode == SAGE_PV16_FP16) return SAGE_ERR_UNSUPPORTED;
   if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
   return SAGE_OK;
 }
@@ -462,6 +472,7 @@ sage_status sage_attn_quantized(const int8_t* q8, const float* qs, const int8_t*
   sage_status s = check_dtype(out_dtype);
   if (s != SAGE_OK) return s;
   if (out_layout != SAGE_HND && out_layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
+  if (pv_mode == SAGE_PV16_FP16) return SAGE_ERR_UNSUPPORTED;
   if (!pv_mode_valid(pv_mode)) return SAGE_ERR_INVALID_ARG;
   Opts o;
   if ((s = parse_opts(opts, &o)) != SAGE_OK) return s;
@@ -494,6 +505,19 @@ sage_status sage_qk_int32(const int8_t* q8, const int8_t* k8, int B, int Hq, int
   p.tiles = tiles, p.n_tiles = n_tiles, p.out = s_out;
   p.B = m.B, p.Hq = m.Hq, p.Hkv = m.Hkv, p.Np = (int)m.q_head_rows, p.nblk = m.nblk_q, p.G = m.G;
   return from_cuda(launch_qk_dump(tq, tk, p, m.dp, static_cast<cudaStream_t>(stream)));
+}
+
+sage_status sage_mma_probe(int kind, int iters, double* ops, void* stream) {
+  if (kind < 0 || kind > 2 || iters < 1 || iters > 1000000 || !ops) return SAGE_ERR_INVALID_ARG;
+  sage_status s = check_device();
+  if (s != SAGE_OK) return s;
+  int dev = 0, n_sm = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm <= 0)
+    return SAGE_ERR_CUDA;
+  const double k = kind == 2 ? 16.0 : 32.0;
+  *ops = (double)n_sm * iters * 4.0 * 2.0 * 128.0 * 256.0 * k;
+  return from_cuda(launch_mma_probe(kind, iters, n_sm, static_cast<cudaStream_t>(stream)));
 }
 
 sage_status sage_selftest_wait_timeout(int budget_us, void* stream) {
@@ -530,6 +554,11 @@ const char* sage_status_string(sage_status s) {
 }
 
 int sage_device_supported(void) { return check_device() == SAGE_OK ? 1 : 0; }
+
+void sage_test_inject(int fake_cc, int fail_allocs) {
+  g_fake_cc.store(fake_cc > 0 ? fake_cc : 0);
+  g_fail_allocs.store(fail_allocs > 0 ? fail_allocs : 0);
+}
 
 }  // extern "C"
 

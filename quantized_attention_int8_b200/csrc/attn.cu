@@ -1,7 +1,7 @@
 // Fused INT8-QK / FP8-PV (or FP16-PV) attention for sm_100a (tcgen05 + TMA + TMEM).
 //
-// One CTA computes one 128-row query tile of one (batch, query head) and, when
-// the padded head dim is 256, one 128-column half of the output.  Six warps:
+// One CTA computes one 128-row query tile of one (batch, query head), all of its
+// output columns (a 256-column O at padded head dim 256).  Six warps:
 //
 //   warps 0-3  softmax / correction / epilogue; thread t owns query row t
 //              (TMEM lane t), so row max and row sum need no shuffles;
@@ -10,7 +10,8 @@
 //   warp 5     TMEM allocator and UMMA issuer (one elected thread).
 //
 // Per key tile j of BN keys (the blockwise online softmax of the method):
-//   S_j  = Q8 . K8_j^T                    tcgen05.mma kind::i8 -> int32 in TMEM
+//   S_j  = Q8 . K8_j^T                    tcgen05.mma kind::i8 -> int32 in TMEM, added to a
+//                                         bias that makes each score a float (kSBiasBits)
 //   s    = S_j * (qs * ks_j * sm_scale * log2 e), causal / length mask
 //   m'   = max(m, rowmax s), p = 2^(s - m'), alpha = 2^(m - m'), l = l alpha + sum p
 //   P    = E4M3(p * 448) (FP8 P.V, BN = 128) or fp16(p) (FP16 P.V, BN = 64), written to
@@ -32,7 +33,6 @@
 #include <cuda_fp8.h>
 
 #include <atomic>
-#include <climits>
 
 #include "sage_internal.h"
 #include "sm100.cuh"
@@ -55,14 +55,14 @@ struct FwdCfg {
   static constexpr int V_BYTES = DV * ROWB;
   static constexpr int P_BYTES = 128 * ROWB;
   static constexpr int ST = PV16 ? (DQK == 64 ? 4 : DQK == 128 ? 3 : 2) : (DQK == 64 ? 5 : 2);  // ring depth
-  static constexpr int CTAS_PER_SM = DQK <= 128 ? 2 : 1;       // two CTAs share an SM when they fit
+  static constexpr int CTAS_PER_SM = DQK <= 128 ? 2 : 1;  // two CTAs share an SM when they fit (d <= 128)
   static constexpr int BAR_BYTES = 256;
   static constexpr int SMEM = 1024 + Q_BYTES + ST * (K_BYTES + V_BYTES) + P_BYTES + BAR_BYTES;
   // TMEM: S (int32 scores, BN columns) and O (fp32, DV columns).  In fp16+fp32 mode the
   // per-tile fp16 accumulator T (DV columns) reuses S's columns (and those up to O) once the
   // scores are in registers.
   static constexpr uint32_t S_COL = 0, T_COL = 0, O_COL = BN > DV ? BN : DV;
-  static constexpr uint32_t TMEM_COLS = O_COL + DV <= 128 ? 128 : 256;
+  static constexpr uint32_t TMEM_COLS = O_COL + DV <= 128 ? 128 : (O_COL + DV <= 256 ? 256 : 512);
   static_assert(ROWB == 128, "P and V^T rows are one 128-byte swizzle span");
   static_assert(O_COL + DV <= TMEM_COLS, "TMEM plan");
   static_assert(ST <= 8, "barrier array size");
@@ -134,6 +134,14 @@ __device__ __forceinline__ void add_f16x2_f32(uint32_t t, float& a0, float& a1) 
 constexpr float kLog2_448 = 8.807354922057604f;  // p * 448 = 2^(log2 p + log2 448)
 constexpr float kTau = 2.0f;                       // reference-max slack of the online softmax (log2 units)
 
+// The Q.K^T accumulator is armed with the bit pattern of 1.5 * 2^23 before each tile's MMAs, which
+// then add the int32 products to it.  Every score satisfies |S| <= 256 * 127^2 < 2^22, so the sum
+// is the bit pattern of the float 1.5 * 2^23 + S: the scores arrive as floats in [2^23, 2^24), where
+// float order is integer order (the row max needs no conversion) and S = value - 1.5 * 2^23 is one
+// exact subtraction, with no int-to-float conversion.
+constexpr uint32_t kSBiasBits = 0x4B400000u;
+constexpr float kSBias = 12582912.0f;  // 1.5 * 2^23
+
 template <int DQK, int DV, int MODE, bool CAUSAL, typename OutT, bool PV16, bool PACKED, bool OPTS>
 __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     sage_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -159,7 +167,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
   int qt = blockIdx.x;
   if (CAUSAL) qt = nblk_q - 1 - qt;  // longest rows first
   if (qt < 0 || qt >= nblk_q) return;  // past the end of this sequence (the whole CTA leaves)
-  const int hq = blockIdx.y / p.n_vhalves, vh = blockIdx.y - hq * p.n_vhalves;
+  const int hq = blockIdx.y;
   const int hkv = hq / p.G;
   // Causal mask, bottom-right aligned: query i sees keys j <= i + (nk - nq).
   const int koff = nk - nq;
@@ -175,7 +183,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
   if (n_kv == 0) {
     // no row of this tile sees a key (nk = 0, or the causal offset leaves the tile empty): zeros
     if (warp < 4 && grow < nq)
-      for (int c = vh * DV; c < min(p.m.d, vh * DV + DV); ++c) store_elem(out + orow + c, 0.f);
+      for (int c = 0; c < p.m.d; ++c) store_elem(out + orow + c, 0.f);
     return;
   }
 
@@ -214,7 +222,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       tma_prefetch_desc(&tmV);
       const int q_row = (int)(sv.q_row0 + (long long)hq * p.m.q_head_rows) + qt * 128;
       const int k_row = (int)(sv.k_row0 + (long long)hkv * p.m.k_head_rows);
-      const int v_row = (int)(sv.v_row0 + (long long)hkv * p.m.dp) + vh * DV;
+      const int v_row = (int)(sv.v_row0 + (long long)hkv * p.m.dp);
       const int v_col = (int)sv.v_col0;
       mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
       for (int s = 0; s < C::NSUB; ++s) tma_load_2d(sQ + s * 128 * C::KSUB, &tmQ, &bars->q_full, s * C::KSUB, q_row);
@@ -239,9 +247,9 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     }
   } else if (warp == 5) {
     // ------------------------------------------------------------------ UMMA issuer
-    // fp32 mode: QK(j) is issued as soon as S is free (the softmax has it in registers),
-    // ahead of PV(j-1).  fp16+fp32 mode: T(j) lives in S's columns, so QK(j+1) waits
-    // until the softmax has merged T(j) into O, and the order is QK(j), PV(j).
+    // fp32 mode: QK(j) is issued as soon as S is free (the softmax has it in registers and has
+    // re-armed it), ahead of PV(j-1).  fp16+fp32 mode: T(j) lives in S's columns, so QK(j+1)
+    // waits until the softmax has taken T(j) into registers, and the order is QK(j), PV(j).
     if (lane == 0) {
       constexpr uint32_t idesc_qk = make_idesc(2 /*S32*/, 1 /*S8*/, 128, C::BN);
       // A = P, B = V^T, both E4M3 (kind::f8f6f4) or both F16 (kind::f16): format code 0 either way
@@ -275,14 +283,15 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
         for (int j = 0; j < n_kv && ok; ++j) {
           const int st = j % C::ST;
           if (!mbar_wait(&bars->k_full[st], (j / C::ST) & 1, abort)) { ok = false; break; }
-          if (j > 0 && !mbar_wait(&bars->s_free, (j - 1) & 1, abort)) { ok = false; break; }
+          // S armed with the score bias (phase j: before tile 0, then after each tile's scores left)
+          if (!mbar_wait(&bars->s_free, j & 1, abort)) { ok = false; break; }
           tc_fence_after();
           const uint32_t ka = smem_u32(sK + st * C::K_BYTES);
 #pragma unroll
           for (int k = 0; k < DQK / 32; ++k) {
             const int sub = (k * 32) / C::KSUB, off = (k * 32) % C::KSUB;
             umma_i8(tmem + C::S_COL, smem_desc_kmajor(qa + sub * 128 * C::KSUB + off, C::KSUB),
-                    smem_desc_kmajor(ka + sub * C::BN * C::KSUB + off, C::KSUB), idesc_qk, (uint32_t)(k > 0));
+                    smem_desc_kmajor(ka + sub * C::BN * C::KSUB + off, C::KSUB), idesc_qk, 1u);
           }
           umma_commit(&bars->s_full);
           if (MODE == 0) {
@@ -299,6 +308,19 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     }
   } else {
     // ------------------------------------------------------------------ softmax warps 0-3
+    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    const uint32_t scol = tmem + lane_base + C::S_COL;
+    const uint32_t ocol = tmem + lane_base + C::O_COL;
+    // arm S with the score bias, then release it to the first Q.K^T
+    auto arm_s = [&]() {
+#pragma unroll
+      for (int cc = 0; cc < C::BN / 4; ++cc) tmem_fill4(scol + cc * 4, kSBiasBits);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars->s_free);
+    };
+    arm_s();
     {
       // Co-resident CTAs share an SM and its MUFU units.  Started together they stay in step,
       // all in their exponential loops at once (each at a fraction of the MUFU rate) and all in
@@ -313,9 +335,6 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       asm volatile("bar.sync 1, 128;" ::: "memory");
       if (slot) __nanosleep(slot * (600u / C::CTAS_PER_SM));
     }
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t scol = tmem + lane_base + C::S_COL;
-    const uint32_t ocol = tmem + lane_base + C::O_COL;
     // the Q scale of this row's group (its 128-token block, or with finer scales (OPTS) its 32-token
     // warp group or the row itself).  Instances without the options keep the plain block index:
     // changing it was measured to slow the tile loop's schedule by 2%.
@@ -330,15 +349,12 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
       tc_fence_after();
       constexpr int BN = C::BN;
+      // scores as float bit patterns 1.5 * 2^23 + S (see kSBiasBits)
       uint32_t s[BN];
 #pragma unroll
       for (int cc = 0; cc < BN / 32; ++cc) tmem_ld32(scol + cc * 32, *reinterpret_cast<uint32_t(*)[32]>(&s[cc * 32]));
       tmem_wait_ld();
-      if (MODE == 0) {  // S is in registers: the next QK may overwrite it
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free);
-      }
+      if (MODE == 0) arm_s();  // S is in registers: re-arm it for the next Q.K^T
 
       // dequantization factor in the log2 domain, with the K scale of the 128-key block; at d = 64
       // that scale is loaded one tile ahead (measured +1.3% with FP8 P.V, +3.7% with FP16 P.V;
@@ -354,46 +370,25 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       const int key0 = i * BN;
       const bool edge = (key0 + BN > nk) || (CAUSAL && key0 + BN - 1 > qt * 128 + koff);
       int lim = BN;  // this row sees the tile's columns c < lim (none if lim <= 0)
-      float mt;  // the tile's row max, scaled
-      if constexpr (MODE == 1) {
-        // scores as floats first (exact: |S| < 2^24), then three-input float maxima; measured
-        // 7% faster with the fp16+fp32 merge below, and 5% slower than the integer maxima in
-        // the fp32-accumulation instances
+      if (edge) {
+        lim = min(nk - key0, BN);
+        if (CAUSAL) lim = min(lim, grow + koff - key0 + 1);
 #pragma unroll
-        for (int c = 0; c < BN; ++c) s[c] = __float_as_uint((float)(int)s[c]);
-        if (edge) {
-          lim = min(nk - key0, BN);
-          if (CAUSAL) lim = min(lim, grow + koff - key0 + 1);
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c >= lim) s[c] = __float_as_uint(-INFINITY);
-        }
-        float mx4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) mx4[e] = fmaxf(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1]));
-#pragma unroll
-        for (int c = 8; c < BN; c += 8)
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            mx4[e] = fmax3(mx4[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
-        const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
-        mt = (mx == -INFINITY) ? -INFINITY : __fmul_rn(mx, f);
-      } else {
-        if (edge) {
-          lim = min(nk - key0, BN);
-          if (CAUSAL) lim = min(lim, grow + koff - key0 + 1);
-#pragma unroll
-          for (int c = 0; c < BN; ++c)
-            if (c >= lim) s[c] = (uint32_t)INT_MIN;
-        }
-        int mx8[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = (int)s[e];
-#pragma unroll
-        for (int c = 8; c < BN; ++c) mx8[c & 7] = max(mx8[c & 7], (int)s[c]);
-        const int mx = max(max(max(mx8[0], mx8[1]), max(mx8[2], mx8[3])), max(max(mx8[4], mx8[5]), max(mx8[6], mx8[7])));
-        mt = (mx == INT_MIN) ? -INFINITY : __fmul_rn((float)mx, f);
+        for (int c = 0; c < BN; ++c)
+          if (c >= lim) s[c] = __float_as_uint(-INFINITY);
       }
+      // row max with three-input float maxima on the biased scores (their float order is the
+      // scores' order); 1.5 * 2^23 + S - 1.5 * 2^23 recovers S exactly
+      float mx4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) mx4[e] = fmaxf(__uint_as_float(s[2 * e]), __uint_as_float(s[2 * e + 1]));
+#pragma unroll
+      for (int c = 8; c < BN; c += 8)
+#pragma unroll
+        for (int e = 0; e < 4; ++e)
+          mx4[e] = fmax3(mx4[e], __uint_as_float(s[c + 2 * e]), __uint_as_float(s[c + 2 * e + 1]));
+      const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]);
+      const float mt = (mx == -INFINITY) ? -INFINITY : __fmul_rn(__fsub_rn(mx, kSBias), f);  // the tile's row max, scaled
       // The reference max m moves only when the running max exceeds it by more than kTau,
       // so O is rescaled rarely; p = 2^(s - m) <= 2^kTau is stored as E4M3(p * 448 * 2^-kTau)
       // (FP8 P.V) or as fp16(p) (FP16 P.V).
@@ -403,8 +398,6 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       const float alpha = upd ? ((m == -INFINITY) ? 0.f : ex2_approx(m - m_new)) : 1.f;
       const float bias = (m_new == -INFINITY) ? 0.f : (PV16 ? 0.f : kLog2_448 - kTau) - m_new;
       const bool rescale = MODE == 0 && i > 0 && __any_sync(0xffffffffu, alpha != 1.f);
-      // a score as float: held as int32 bits (fp32 accumulation) or already converted (fp16+fp32)
-      auto score = [](uint32_t v) { return MODE == 1 ? __uint_as_float(v) : (float)(int)v; };
       // p * 448 * 2^-kTau = 2^(s*f - m + log2 448 - kTau) -> E4M3, 4 keys per 32-bit word;
       // FP16 P.V: p = 2^(s*f - m) -> fp16, 2 keys per word
       // row sums: four scalar partial sums, or in the non-causal d = 128 fp32-accumulation FP8
@@ -421,14 +414,17 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
         for (int e = 0; e < 4; e += 2) {
           const int c = c4 * 4 + e;
           float x0, x1;
+          // the exact score S = (1.5 * 2^23 + S) - 1.5 * 2^23 (same binade: no rounding), then
+          // S * f + bias with one rounding, as the scores were integers converted to float
           if (DQK >= 128 && MODE == 0) {  // packed FMA measured faster only in this configuration
-            const float2 x = __ffma2_rn(make_float2(score(s[c]), score(s[c + 1])), make_float2(f, f),
-                                        make_float2(bias, bias));
+            const float2 sc = __fadd2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
+                                         make_float2(-kSBias, -kSBias));
+            const float2 x = __ffma2_rn(sc, make_float2(f, f), make_float2(bias, bias));
             x0 = x.x;
             x1 = x.y;
           } else {
-            x0 = fmaf(score(s[c]), f, bias);
-            x1 = fmaf(score(s[c + 1]), f, bias);
+            x0 = fmaf(__fsub_rn(__uint_as_float(s[c]), kSBias), f, bias);
+            x1 = fmaf(__fsub_rn(__uint_as_float(s[c + 1]), kSBias), f, bias);
           }
           pv[e] = ex2_approx(x0);
           pv[e + 1] = ex2_approx(x1);
@@ -490,52 +486,41 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       if (lane == 0) mbar_arrive(&bars->p_full);
 
       if (MODE == 1) {
-        // O = O * alpha + T(i), T being this tile's fresh fp16 accumulator (in S's columns)
+        // O = O * alpha + T(i), T being this tile's fresh fp16 accumulator (in S's columns).  T is
+        // taken into registers first, so S is re-armed and released to the next Q.K^T before the
+        // merge, which then overlaps that MMA.
         if (!warp_wait(&bars->pv_done, i & 1, abort)) { ok = false; break; }
         tc_fence_after();
         const uint32_t tcol = tmem + lane_base + C::T_COL;
-        // warp-uniform form of the merge: tile 0 (O = T), no row rescaled (O += T), or O = O * alpha + T
-        const int form = i == 0 ? 0 : (__any_sync(0xffffffffu, alpha != 1.f) ? 2 : 1);
-#pragma unroll 1
+        uint32_t t[DV / 2];
+#pragma unroll
+        for (int cc = 0; cc < DV / 32; ++cc) tmem_ld16_pack16(tcol + cc * 32, *reinterpret_cast<uint32_t(*)[16]>(&t[cc * 16]));
+        tmem_wait_ld();
+        arm_s();
+        // O = O * alpha + T (tile 0: O = T; rows whose reference did not move have alpha = 1)
+        const float am = i == 0 ? 0.f : alpha;
+#pragma unroll
         for (int cc = 0; cc < DV / 32; ++cc) {
-          uint32_t t[16], o[32];
-          tmem_ld16_pack16(tcol + cc * 32, t);
-          tmem_ld32(ocol + cc * 32, o);  // loaded on tile 0 too (unused there): conditional loads spill
-          tmem_wait_ld();
-          if (form == 0) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float a0 = 0.f, a1 = 0.f;
-              add_f16x2_f32(t[e], a0, a1);
-              o[2 * e] = __float_as_uint(a0);
-              o[2 * e + 1] = __float_as_uint(a1);
-            }
-          } else if (form == 1) {
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float a0 = __uint_as_float(o[2 * e]), a1 = __uint_as_float(o[2 * e + 1]);
-              add_f16x2_f32(t[e], a0, a1);
-              o[2 * e] = __float_as_uint(a0);
-              o[2 * e + 1] = __float_as_uint(a1);
-            }
+          uint32_t o[32];
+          if (i > 0) {
+            tmem_ld32(ocol + cc * 32, o);
+            tmem_wait_ld();
           } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float a0 = __uint_as_float(o[2 * e]) * alpha, a1 = __uint_as_float(o[2 * e + 1]) * alpha;
-              add_f16x2_f32(t[e], a0, a1);
-              o[2 * e] = __float_as_uint(a0);
-              o[2 * e + 1] = __float_as_uint(a1);
-            }
+            for (int e = 0; e < 32; ++e) o[e] = 0u;
+          }
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            float a0 = __uint_as_float(o[2 * e]) * am, a1 = __uint_as_float(o[2 * e + 1]) * am;
+            add_f16x2_f32(t[cc * 16 + e], a0, a1);
+            o[2 * e] = __float_as_uint(a0);
+            o[2 * e + 1] = __float_as_uint(a1);
           }
           tmem_st32(ocol + cc * 32, o);
         }
         tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars->s_free);
       }
     }
-
     // ---------------------------------------------------------------- epilogue
     if (ok && MODE == 0) {
       ok = warp_wait(&bars->pv_done, (n_kv - 1) & 1, abort);
@@ -543,10 +528,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     }
     if (ok) {
       const float inv_l = l > 0.f ? __fdiv_rn(1.f, l) : 0.f;  // a row that saw no key outputs zeros
-      const float* vsp = p.vs + ((size_t)b * p.m.Hkv + hkv) * p.m.dp + vh * DV;
+      const float* vsp = p.vs + ((size_t)b * p.m.Hkv + hkv) * p.m.dp;
       // smoothed V: its token mean goes back on (rows that saw a key)
       const float* vmp =
-          (OPTS && p.vm && l > 0.f) ? p.vm + ((size_t)b * p.m.Hkv + hkv) * p.m.dp + vh * DV : nullptr;
+          (OPTS && p.vm && l > 0.f) ? p.vm + ((size_t)b * p.m.Hkv + hkv) * p.m.dp : nullptr;
 #pragma unroll 1
       for (int cc = 0; cc < DV / 32; ++cc) {
         uint32_t o[32];
@@ -554,7 +539,7 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
         tmem_ld32(ocol + cc * 32, o);
         tmem_wait_ld();
         if (grow < nq) {
-          const int c0 = vh * DV + cc * 32;
+          const int c0 = cc * 32;
 #pragma unroll
           for (int e = 0; e < 32; ++e) of[e] = __uint_as_float(o[e]) * (vsp[cc * 32 + e] * inv_l);
           if (OPTS && vmp) {
@@ -675,6 +660,64 @@ __global__ void __launch_bounds__(128, 1)
 }
 
 // ------------------------------------------------------------------------------------------------
+// Diagnostic: the tcgen05.mma issue rate of this GPU.  One CTA per SM; one thread issues `iters`
+// rounds of 4 back-to-back MMAs (M = 128, N = 256, 32 bytes of K per row: K = 32 for kind::i8 and
+// kind::f8f6f4, K = 16 for kind::f16) from one zeroed shared-memory tile pair into one TMEM
+// accumulator, then waits for them (bounded).  The operand data play no part in the rate.
+// ------------------------------------------------------------------------------------------------
+template <int KIND>
+__global__ void __launch_bounds__(128, 1) sage_mma_probe_kernel(int iters) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  const uint32_t pad = (1024u - (smem_u32(smem_raw) & 1023u)) & 1023u;
+  unsigned char* a = smem_raw + pad;  // 128 rows x 128 bytes
+  unsigned char* bt = a + 128 * 128;  // 256 rows x 128 bytes
+  __shared__ uint64_t bar;
+  __shared__ uint32_t tbase;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5;
+  for (int i = threadIdx.x; i < (128 + 256) * 128 / 16; i += blockDim.x)
+    reinterpret_cast<uint4*>(a)[i] = make_uint4(0, 0, 0, 0);
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(&tbase, 256);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (threadIdx.x == 0) {
+    // kind::i8: S32 accumulator, S8 operands; kind::f8f6f4: F32, E4M3; kind::f16: F32, F16
+    constexpr uint32_t idesc = make_idesc(KIND == 0 ? 2 : 1, KIND == 0 ? 1 : 0, 128, 256);
+    const uint32_t aa = smem_u32(a), bb = smem_u32(bt);
+    for (int it = 0; it < iters; ++it) {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint64_t ad = smem_desc_kmajor(aa + k * 32, 128), bd = smem_desc_kmajor(bb + k * 32, 128);
+        if (KIND == 0)
+          umma_i8(tbase, ad, bd, idesc, 1u);
+        else if (KIND == 1)
+          umma_f8(tbase, ad, bd, idesc, 1u);
+        else
+          umma_f16(tbase, ad, bd, idesc, 1u);
+      }
+    }
+    umma_commit(&bar);
+    if (!mbar_wait(&bar, 0, &abort_flag)) drain_wait(&bar, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 0) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 256);
+  }
+}
+
+// ------------------------------------------------------------------------------------------------
 // launchers
 // ------------------------------------------------------------------------------------------------
 // Sets a kernel's dynamic shared-memory limit once per device (the attribute is per device).
@@ -703,7 +746,7 @@ static cudaError_t launch_fwd_t(const CUtensorMap& tq, const CUtensorMap& tk, co
   static std::atomic<unsigned long long> attr_done[4] = {{0}, {0}, {0}, {0}};
   cudaError_t e = ensure_smem_limit(kern, C::SMEM, attr_done[which]);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.nblk_q, p.m.Hq * p.n_vhalves, p.m.B);
+  dim3 grid(p.nblk_q, p.m.Hq, p.m.B);
   // a programmatic dependent of whatever ran before on the stream (the quantize pass): the CTAs
   // may start while it finishes and wait for it in griddepcontrol.wait
   cudaLaunchConfig_t cfg = {};
@@ -743,7 +786,7 @@ static cudaError_t launch_fwd_o(const CUtensorMap& tq, const CUtensorMap& tk, co
   switch (p.m.dp) {
     case 64: return launch_fwd_d<64, 64, OutT>(tq, tk, tv, p, causal, mode, st);
     case 128: return launch_fwd_d<128, 128, OutT>(tq, tk, tv, p, causal, mode, st);
-    case 256: return launch_fwd_d<256, 128, OutT>(tq, tk, tv, p, causal, mode, st);
+    case 256: return launch_fwd_d<256, 256, OutT>(tq, tk, tv, p, causal, mode, st);
     default: return cudaErrorInvalidValue;
   }
 }
@@ -848,6 +891,25 @@ static cudaError_t launch_qk_dump_t(const CUtensorMap& tq, const CUtensorMap& tk
   if (e != cudaSuccess) return e;
   sage_qk_dump_kernel<DQK><<<p.n_tiles, 128, smem, st>>>(tq, tk, p);
   return cudaGetLastError();
+}
+
+template <int KIND>
+static cudaError_t launch_mma_probe_t(int iters, int n_sm, cudaStream_t st) {
+  const int smem = 1024 + (128 + 256) * 128;
+  static std::atomic<unsigned long long> attr_done{0};
+  cudaError_t e = ensure_smem_limit(sage_mma_probe_kernel<KIND>, smem, attr_done);
+  if (e != cudaSuccess) return e;
+  sage_mma_probe_kernel<KIND><<<n_sm, 128, smem, st>>>(iters);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_mma_probe(int kind, int iters, int n_sm, cudaStream_t st) {
+  switch (kind) {
+    case 0: return launch_mma_probe_t<0>(iters, n_sm, st);
+    case 1: return launch_mma_probe_t<1>(iters, n_sm, st);
+    case 2: return launch_mma_probe_t<2>(iters, n_sm, st);
+    default: return cudaErrorInvalidValue;
+  }
 }
 
 cudaError_t launch_qk_dump(const CUtensorMap& tq, const CUtensorMap& tk, const QkDumpParams& p, int dp,

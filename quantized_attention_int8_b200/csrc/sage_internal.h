@@ -114,7 +114,6 @@ struct FwdParams {
   int q_gran_log2;  // query tokens per Q scale = 1 << q_gran_log2
   int nblk_q;     // 128-row query tiles of the longest sequence (grid x)
   int G;          // query heads per kv head
-  int n_vhalves;  // output column halves handled by separate CTAs (2 when dp = 256)
   int vec_out;    // 16-byte output stores allowed (d % 8 == 0 and 16-byte aligned out)
   float scale_log2;  // sm_scale * log2(e)
 };
@@ -135,6 +134,8 @@ cudaError_t launch_seq_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int
                             long long total_q, long long total_k, SeqDesc* seqs, cudaStream_t st);
 cudaError_t read_clear_device_error(int* value);
 cudaError_t launch_wait_probe(long long budget_cycles, cudaStream_t st);
+// tcgen05.mma issue-rate probe: kind 0 = kind::i8, 1 = kind::f8f6f4, 2 = kind::f16; one CTA per SM.
+cudaError_t launch_mma_probe(int kind, int iters, int n_sm, cudaStream_t st);
 cudaError_t launch_qk_dump(const CUtensorMap& tq, const CUtensorMap& tk, const QkDumpParams& p, int dp,
                            cudaStream_t st);
 
