@@ -4,24 +4,32 @@
 
 A step is one pass of the whole path over one batch of synthetic input:
 the quantize/smooth pass plus the fused INT8-QK / FP8-PV attention kernel
-(``sage_attn``).  The default workload is the image-DiT self-attention shape
-B=2, H=24, N=4096, d=64, bf16, HND, non-causal, K with a per-channel offset.
+(``sage_attn``).  The default workload is the video-DiT long-sequence shape
+B=1, H=24, N=32768, d=128, bf16, NHD, non-causal, K with a per-channel offset,
+fp16+fp32 P.V accumulation (the largest of the five workloads, N >= 8K and
+d = 128).  The image-DiT (B=2, H=24, N=4096, d=64) and causal GQA prefill
+(B=4, Hq=32, Hkv=8, N=8192, d=128) workloads are measured in the same run and
+reported under ``also``, each with its own roofline.
 
 * ``value``: whole-job attention TOPS, 4*B*Hq*N^2*d (halved under the causal
   mask) per step, inputs resident in HBM, per-step CUDA events with an L2
   flush between steps (outside the events), max over ranks.
 * ``roofline``: the fused attention kernel alone (sage_attn_quantized on the
   same buffers, per-launch CUDA events, L2 flushed) against the dense INT8/FP8
-  tensor peak (2x the measured bf16 cuBLAS peak, the B200 nominal ratio).
+  tensor peak (2x the measured bf16 cuBLAS peak, the B200 nominal ratio); the
+  tcgen05.mma rate this GPU measures for kind::i8 and kind::f8f6f4
+  (sage_mma_probe) is reported beside it with the fraction against it.
 * ``e2e``: the same metric through the public API (``sage_attn``) with pinned
   HOST buffers: every step uploads q, k, v and downloads its output inside the
   timed region.  ``value`` streams the steps (three CUDA streams, two device
   buffer sets: step i+1's upload and step i-1's download overlap step i);
   ``serial`` runs them one at a time with per-step events.
-* ``cpu_baseline``: the CPU oracle (exact fp64 attention) on a bounded sample
-  of the same workload's heads, on this host's cores.
+* ``cpu_baseline``: the CPU oracle on this host's cores, on a bounded sample of
+  the same workload: exact fp64 attention of 512-row query chunks of successive
+  heads (TOPS), and the quantization emulation of one head (GB/s).
 * ``--impl reference``: there is no reference implementation to run; the
-  reference arm times the CPU oracle on the same workload instead.
+  reference arm times the CPU oracle (exact fp64 attention, bounded row
+  samples) on the same workload instead.
 
 Multi-GPU (torchrun): replicas only, one independent copy of the workload per
 rank, no collective on the data path (weak scaling).
@@ -46,7 +54,8 @@ sys.path.insert(0, ROOT)
 import workloads as W  # noqa: E402
 
 METRIC = "attention TOPS on 1 B200 (N=1K-32K, d=64/128) and % of dense INT8/FP8 tensor peak"
-DEFAULT_WORKLOAD = W.IMAGE_DIT.name
+DEFAULT_WORKLOAD = W.VIDEO_DIT.name
+ALSO = [W.IMAGE_DIT.name, W.LLM_GQA.name]
 L2_FLUSH_BYTES = 256 << 20
 
 
@@ -215,26 +224,52 @@ def time_e2e_streamed(qh, kh, vh, attn, steps, warmup, flush_buf):
     return a.elapsed_time(b)
 
 
-def cpu_oracle_sample(w: W.Workload, budget_s: float):
-    """Exact fp64 attention (the oracle) on successive (b, hq) heads until the time budget is used."""
-    from oracle import attention
-    from oracle.quant import to_hnd
-    q, k, v = W.make_inputs(w.with_(B=1))
-    qf, kf, vf = (to_hnd(t, w.layout) for t in (q, k, v))
-    G = w.Hq // w.Hkv
-    heads, t0 = 0, time.perf_counter()
-    while time.perf_counter() - t0 < budget_s and heads < w.Hq:
-        attention.attention_f64(qf[:, heads:heads + 1], kf[:, heads // G:heads // G + 1],
-                                vf[:, heads // G:heads // G + 1], "HND", w.causal, W.sm_scale_of(w))
-        heads += 1
-    dt = time.perf_counter() - t0
-    ops = w.with_(B=1, Hq=heads, Hkv=heads).ops()
+def _threads():
     try:
         import threadpoolctl
-        threads = max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] or [1])
+        return max([i.get("num_threads", 1) for i in threadpoolctl.threadpool_info()] or [1])
     except Exception:
-        threads = os.cpu_count()
-    return ops / dt / 1e12, threads, heads, dt
+        return os.cpu_count()
+
+
+def _head(t, layout, b, h):
+    t = t[b:b + 1]
+    return (t[:, h:h + 1] if layout == "HND" else t[:, :, h:h + 1]).contiguous()
+
+
+def cpu_oracle_sample(w: W.Workload, q, k, v, budget_s: float, start: int = 0):
+    """Exact fp64 attention (the oracle) of 512-row query chunks of successive (b=0, hq) heads, from
+    chunk `start` on, until the time budget is used (at least one chunk).  Returns (TOPS, threads,
+    rows, seconds, next start)."""
+    from oracle import attention
+    G = w.Hq // w.Hkv
+    nchunk = (w.N + 511) // 512
+    done, pairs, t0, i = 0, 0, time.perf_counter(), start
+    while done == 0 or time.perf_counter() - t0 < budget_s:
+        h, c = (i // nchunk) % w.Hq, i % nchunk
+        rows = np.arange(c * 512, min(w.N, c * 512 + 512))
+        qh, kh, vh = _head(q, w.layout, 0, h), _head(k, w.layout, 0, h // G), _head(v, w.layout, 0, h // G)
+        attention.attention_f64(qh, kh, vh, w.layout, w.causal, W.sm_scale_of(w), heads=[(0, 0)], rows=rows)
+        done += len(rows)
+        pairs += int((rows + 1).sum()) if w.causal else len(rows) * w.N
+        i += 1
+    dt = time.perf_counter() - t0
+    # the metric counts 4*d operations per visible (query, key) pair (causal: half of N^2 per head)
+    ops = 4.0 * w.d * pairs
+    return ops / dt / 1e12, _threads(), done, dt, i
+
+
+def cpu_quantize_sample(w: W.Workload, q, k, v):
+    """The quantization emulation (oracle) of one (b=0) kv head with its first query head: GB/s of
+    the algorithmic bytes (2 B read + 1 B written per Q, K element; V 1 or 2 B written)."""
+    from oracle import quant
+    qh, kh, vh = _head(q, w.layout, 0, 0), _head(k, w.layout, 0, 0), _head(v, w.layout, 0, 0)
+    t0 = time.perf_counter()
+    quant.quantize(qh, kh, vh, w.layout, w.pv_mode, w.q_gran, w.smooth_v)
+    dt = time.perf_counter() - t0
+    n = qh.numel()
+    nbytes = 3 * 2 * n + (4 if w.pv_mode & 2 else 3) * n
+    return nbytes / dt / 1e9, dt
 
 
 def job_throughput(local_ms: float, ops_per_step: float, steps: int, dist=None, device=None):
@@ -255,22 +290,24 @@ def run_reference(args, w):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
         return
-    budget = 8.0
-    vals = []
+    q, k, v = W.make_inputs(w.with_(B=1))
+    budget = args.ref_seconds / max(1, args.warmup + args.steps)  # split the run's CPU budget over its steps
+    vals, start = [], 0
     for i in range(args.warmup + args.steps):
-        tops, threads, heads, dt = cpu_oracle_sample(w, budget / max(1, args.steps))
+        tops, threads, rows, dt, start = cpu_oracle_sample(w, q, k, v, budget, start)
         if i >= args.warmup:
-            vals.append((tops, heads, dt))
-    v = statistics.median(t for t, _, _ in vals)
+            vals.append((tops, rows, dt))
+    val = statistics.median(t for t, _, _ in vals)
     ms = statistics.mean(dt for _, _, dt in vals) * 1e3
     line = {
-        "impl": "reference", "metric": METRIC, "value": v, "unit": "TOPS", "n_gpus": args.gpus, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "f64", "data": "synthetic",
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": _config(w),
-        "cpu_baseline": {"value": v, "unit": "TOPS", "cores": threads, "kind": "oracle",
-                         "sample": f"exact fp64 attention of {vals[-1][1]} (b=0, hq) head(s) of the workload per step"},
-        "e2e": {"value": v, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "cpu_baseline": {"value": val, "unit": "TOPS", "cores": threads, "kind": "oracle",
+                         "sample": f"exact fp64 attention of {vals[-1][1]} query rows (512-row chunks of successive "
+                                   f"(b=0, hq) heads) of the workload per step, {budget:.1f} s budget"},
+        "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "no reference implementation exists for this path; the reference arm is the CPU oracle",
     }
     print(json.dumps(line), flush=True)
@@ -283,6 +320,117 @@ def _config(w):
             "qk_quant_gran": {128: "per_block", 32: "per_warp", 1: "per_thread"}[w.q_gran], "smooth_v": w.smooth_v,
             "values": w.dist, "l2": "flushed between steps (256 MiB write outside the events)",
             "host": "each step enqueued while the device is busy (device sleep before the start event)"}
+
+
+def _modes(w):
+    pv = "fp16+fp32" if w.pv_mode & 1 else "fp32"
+    pvd = "fp16" if w.pv_mode & 2 else "fp8"
+    okw = dict(qk_quant_gran={128: "per_block", 32: "per_warp", 1: "per_thread"}[w.q_gran], smooth_v=w.smooth_v)
+    return pv, pvd, okw
+
+
+def _peak(w, peaks):
+    if w.pv_mode & 2:
+        # half the operations (Q.K^T) at the INT8 rate 2P, half (P.V, fp16) at the fp16 rate P:
+        # the blended peak for all of them is 4P/3
+        return 4.0 / 3.0 * peaks["bf16"], (f"4/3 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s (half "
+                                           "the operations at the INT8 rate 2x bf16, half at the fp16 rate 1x bf16)")
+    return 2.0 * peaks["bf16"], (f"2 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s "
+                                 "(dense INT8/FP8 = 2x bf16 on B200)")
+
+
+def mma_rates(qa, reps=5, iters=10000):
+    """tcgen05.mma rate of this GPU per kind (sage_mma_probe: one CTA per SM issuing MMAs back to
+    back), best of `reps` launches timed with CUDA events: TOPS for kind::i8 and kind::f8f6f4,
+    TFLOP/s for kind::f16."""
+    st = torch.cuda.current_stream()
+    out = {}
+    for kind, name in ((0, "i8"), (1, "f8f6f4"), (2, "f16")):
+        ops = ctypes.c_double(0.0)
+        best = 0.0
+        for r in range(reps + 2):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            s = qa.capi.sage_mma_probe(kind, iters, ctypes.byref(ops), st.cuda_stream)
+            b.record(st)
+            if s != qa.SAGE_OK:
+                raise RuntimeError(f"sage_mma_probe: {qa.sage_status_string(s)}")
+            torch.cuda.synchronize()
+            if r >= 2:
+                best = max(best, ops.value / (a.elapsed_time(b) * 1e-3) / 1e12)
+        out[name] = best
+    qa.sage_check_status()
+    return out
+
+
+def measure(qa, w, args, flush, dist, rates, clk_sampler=None):
+    """One workload: the whole path per step, the fused kernel alone, the quantize pass alone.
+    Returns (result dict, device inputs, CPU inputs)."""
+    pv, pvd, okw = _modes(w)
+    scale = W.sm_scale_of(w)
+    q, k, v = W.make_inputs(w)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    out = torch.empty_like(qd)
+    ops = w.ops()
+
+    # ---- whole path (quantize + attention), device-resident inputs
+    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out, pv_dtype=pvd, **okw)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    if clk_sampler is not None:
+        with clk_sampler:
+            times = time_steps(step, args.steps, args.warmup, flush)
+    else:
+        times = time_steps(step, args.steps, args.warmup, flush)
+    qa.sage_check_status()
+    value, total_ms = job_throughput(sum(times), ops, args.steps, dist, "cuda")
+
+    # ---- the fused attention kernel alone (roofline)
+    z = qa.sage_quantize(qd, kd, vd, w.layout, pv, pvd, **okw)
+    kern = lambda: qa.sage_attn_quantized(z, qd.dtype, w.layout, w.causal, scale, pv, out=out)
+    ktimes = time_steps(kern, args.steps, args.warmup, flush)
+    qa.sage_check_status()
+    k_ms = statistics.mean(ktimes)
+    peaks = _peaks()
+    peak_tops, peak_src = _peak(w, peaks)
+    achieved = ops / (k_ms * 1e-3) / 1e12
+    # the same against the tcgen05.mma rate measured on this GPU: Q.K^T at the kind::i8 rate, P.V at
+    # the kind::f8f6f4 (FP8 P.V) or kind::f16 (FP16 P.V) rate, half of the operations each
+    pv_rate = rates["f16"] if w.pv_mode & 2 else rates["f8f6f4"]
+    mma_peak = 1.0 / (0.5 / rates["i8"] + 0.5 / pv_rate)
+
+    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element
+    # (V: 2 B written in the FP16 P.V modes); the C entry point on preallocated outputs, so the Python
+    # allocations are not timed
+    qopts = qa.opts(**okw)  # kept alive while qargs points at it
+    qargs = [qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), w.B, w.Hq, w.Hkv, w.N, w.d,
+             qa.SAGE_BF16 if qd.dtype == torch.bfloat16 else qa.SAGE_FP16,
+             qa.SAGE_HND if w.layout == "HND" else qa.SAGE_NHD, w.pv_mode, ctypes.byref(qopts),
+             *(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "km", "v8t", "vs", "vm")),
+             torch.cuda.current_stream().cuda_stream]
+    qtimes = time_steps(lambda: qa.capi.sage_quantize(*qargs), max(3, args.steps // 2), 3, flush)
+    qa.sage_check_status()
+    q_ms = statistics.mean(qtimes)
+    q_bytes = 3 * (q.numel() + k.numel()) + (4 if w.pv_mode & 2 else 3) * v.numel()
+    del z
+    res = {
+        "value": value, "ms_per_step": total_ms / args.steps,
+        "step_ms": {"min_ms": min(times), "median_ms": statistics.median(times), "max_ms": max(times)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
+                     "frac": achieved / peak_tops, "traffic": _traffic(w.name),
+                     "kernel": "sage_fwd_kernel", "kernel_ms": k_ms, "peak_source": peak_src,
+                     "tcgen05_measured": {"peak": mma_peak, "frac": achieved / mma_peak,
+                                          "rates": rates,
+                                          "how": "sage_mma_probe (back-to-back tcgen05.mma, every SM) on this GPU; "
+                                                 "half the operations at the kind::i8 rate, half at the P.V kind's "
+                                                 "rate; frac above uses the bf16-derived peak"}},
+        "quantize": {"ms": q_ms, "algorithmic_bytes": q_bytes, "GB_per_s": q_bytes / (q_ms * 1e-3) / 1e9,
+                     "hbm_peak_GB_per_s": peaks["hbm"], "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm"]},
+        # d not in {64, 128, 256}: the kernels run on the zero-padded head dim
+        "padded_work_value": value * qa.padded_dim(w.d) / w.d if qa.padded_dim(w.d) != w.d else None,
+    }
+    return res, (qd, kd, vd, out), (q, k, v)
 
 
 def run_ours(args, w):
@@ -298,60 +446,17 @@ def run_ours(args, w):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     if not qa.sage_device_supported():
         raise SystemExit("this device is not a B200 (compute capability 10.0)")
-    pv = "fp16+fp32" if w.pv_mode & 1 else "fp32"
-    pvd = "fp16" if w.pv_mode & 2 else "fp8"
-    okw = dict(qk_quant_gran={128: "per_block", 32: "per_warp", 1: "per_thread"}[w.q_gran], smooth_v=w.smooth_v)
-    scale = W.sm_scale_of(w)
-    q, k, v = W.make_inputs(w)
-    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
-    qd, kd, vd = (t.cuda() for t in (q, k, v))
-    out = torch.empty_like(qd)
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    ops = w.ops()
-
-    # ---- whole path (quantize + attention), device-resident inputs
-    step = lambda: qa.sage_attn(qd, kd, vd, w.layout, w.causal, scale, pv, out=out, pv_dtype=pvd, **okw)
-    if dist:
-        dist.barrier()
-    torch.cuda.synchronize()
-    with ClockSampler(torch.cuda.current_device()) as clk:
-        times = time_steps(step, args.steps, args.warmup, flush)
-    qa.sage_check_status()
-    value, total_ms = job_throughput(sum(times), ops, args.steps, dist, "cuda")
-    step_stats = {"min_ms": min(times), "median_ms": statistics.median(times), "max_ms": max(times)}
-
-    # ---- the fused attention kernel alone (roofline)
-    z = qa.sage_quantize(qd, kd, vd, w.layout, pv, pvd, **okw)
-    kern = lambda: qa.sage_attn_quantized(z, qd.dtype, w.layout, w.causal, scale, pv, out=out)
-    ktimes = time_steps(kern, args.steps, args.warmup, flush)
-    qa.sage_check_status()
-    k_ms = statistics.mean(ktimes)
-    peaks = _peaks()
-    if w.pv_mode & 2:
-        # half the operations (Q.K^T) at the INT8 rate 2P, half (P.V, fp16) at the fp16 rate P:
-        # the blended peak for all of them is 4P/3
-        peak_tops = 4.0 / 3.0 * peaks["bf16"]
-        peak_src = (f"4/3 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s (half the operations "
-                    "at the INT8 rate 2x bf16, half at the fp16 rate 1x bf16)")
-    else:
-        peak_tops = 2.0 * peaks["bf16"]
-        peak_src = f"2 x {peaks['source']} bf16 cuBLAS burst {peaks['bf16']} TF/s (dense INT8/FP8 = 2x bf16 on B200)"
-    achieved = ops / (k_ms * 1e-3) / 1e12
-
-    # ---- quantize pass alone (HBM-bound): algorithmic bytes = 2 B read + 1 B written per Q/K/V element
-    # (V: 2 B written in the FP16 P.V modes);
-    # the C entry point on preallocated outputs, so the Python allocations are not timed
-    qopts = qa.opts(**okw)  # kept alive while qargs points at it
-    qargs = [qd.data_ptr(), kd.data_ptr(), vd.data_ptr(), w.B, w.Hq, w.Hkv, w.N, w.d,
-             qa.SAGE_BF16 if qd.dtype == torch.bfloat16 else qa.SAGE_FP16,
-             qa.SAGE_HND if w.layout == "HND" else qa.SAGE_NHD, w.pv_mode, ctypes.byref(qopts),
-             *(z[n].data_ptr() for n in ("q8", "qs", "k8", "ks", "km", "v8t", "vs", "vm")),
-             torch.cuda.current_stream().cuda_stream]
-    qtimes = time_steps(lambda: qa.capi.sage_quantize(*qargs), max(3, args.steps // 2), 3, flush)
-    q_ms = statistics.mean(qtimes)
-    q_bytes = 3 * (q.numel() + k.numel()) + (4 if w.pv_mode & 2 else 3) * v.numel()
+    rates = mma_rates(qa)
+    clk = ClockSampler(torch.cuda.current_device())
+    main_res, (qd, kd, vd, out), (q, k, v) = measure(qa, w, args, flush, dist, rates, clk)
 
     # ---- end to end through the public API with pinned host buffers
+    pv, pvd, okw = _modes(w)
+    scale = W.sm_scale_of(w)
+    ops = w.ops()
+    in_bytes = sum(t.numel() * t.element_size() for t in (q, k, v))
+    del qd, kd, vd
     qh, kh, vh = (t.pin_memory() for t in (q, k, v))
     outh = torch.empty(q.shape, dtype=q.dtype).pin_memory()
 
@@ -370,28 +475,42 @@ def run_ours(args, w):
                                                                           pv_dtype=pvd, **okw),
                              args.steps, args.warmup, flush)
     e2e_value, e_ms = job_throughput(e_ms, ops, args.steps, dist, "cuda")
+    qa.sage_check_status()
+    del qh, kh, vh, outh
+    torch.cuda.empty_cache()
 
-    line = None
+    # ---- the other workloads, same measurements (no e2e)
+    also = {}
+    for name in ALSO:
+        if name == w.name or args.no_also:
+            continue
+        res, dev, _ = measure(qa, W.BY_NAME[name], args, flush, dist, rates)
+        res["config"] = _config(W.BY_NAME[name])
+        also[name] = res
+        del dev
+        torch.cuda.empty_cache()
+
     if rank == 0:
         cpu = None
         if world == 1:
-            tops, threads, heads, dt = cpu_oracle_sample(w, 12.0)
+            tops, threads, rows, dt, _ = cpu_oracle_sample(w, q, k, v, 12.0)
+            qgbs, qdt = cpu_quantize_sample(w, q, k, v)
             cpu = {"value": tops, "unit": "TOPS", "cores": threads, "kind": "oracle",
-                   "sample": f"exact fp64 attention of {heads} (b=0, hq) head(s), {dt:.1f} s"}
+                   "sample": f"exact fp64 attention of {rows} query rows (512-row chunks of successive (b=0, hq) "
+                             f"heads), {dt:.1f} s",
+                   "quantize": {"value": qgbs, "unit": "GB/s", "kind": "oracle",
+                                "sample": f"quantization emulation of one (b=0) head of Q, K and V, {qdt:.2f} s; "
+                                          "bytes counted as for the GPU quantize pass"}}
         line = {
-            "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "i8+f16" if w.pv_mode & 2 else "i8+f8e4m3", "data": "synthetic",
+            "metric": METRIC, "value": main_res["value"], "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"], "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "i8+f16" if w.pv_mode & 2 else "i8+f8e4m3",
+            "data": "synthetic",
             "config": _config(w),
-            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak_tops, "unit": "TFLOP/s",
-                         "frac": achieved / peak_tops, "traffic": _traffic(w.name),
-                         "kernel": "sage_fwd_kernel", "kernel_ms": k_ms,
-                         "peak_source": peak_src},
-            "quantize": {"ms": q_ms, "algorithmic_bytes": q_bytes, "GB_per_s": q_bytes / (q_ms * 1e-3) / 1e9,
-                         "hbm_peak_GB_per_s": peaks["hbm"], "frac": q_bytes / (q_ms * 1e-3) / 1e9 / peaks["hbm"]},
+            "roofline": main_res["roofline"],
+            "quantize": main_res["quantize"],
             "cpu_baseline": cpu,
-            # d not in {64, 128, 256}: the kernels run on the zero-padded head dim
-            "padded_work_value": value * qa.padded_dim(w.d) / w.d if qa.padded_dim(w.d) != w.d else None,
+            "padded_work_value": main_res["padded_work_value"],
             "e2e": {"value": e2e_value, "unit": "TOPS", "h2d_bytes_per_step": in_bytes,
                     "d2h_bytes_per_step": out.numel() * out.element_size(), "ms_per_step": e_ms / args.steps,
                     "mode": "streamed: every step copies its q, k, v from pinned host memory and its output back "
@@ -399,9 +518,10 @@ def run_ours(args, w):
                             "(three streams, two device buffer sets, L2 flushed before each step's compute)",
                     "serial": {"value": serial_value, "ms_per_step": serial_ms / args.steps,
                                "mode": "one step at a time: upload, compute, download, per-step events"}},
-            "step_ms": step_stats,
+            "step_ms": main_res["step_ms"],
             "gpu_launches": 4 * args.steps,
             "clocks": clk.summary(),
+            "also": also,
         }
         print(json.dumps(line), flush=True)
     if dist:
@@ -416,6 +536,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(W.BY_NAME))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-also", action="store_true", help="measure only --workload")
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="reference arm: CPU seconds for the whole run (warm-up and timed steps)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)  # at least 3 untimed warm-up steps
     w = W.BY_NAME[args.workload]

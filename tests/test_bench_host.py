@@ -9,7 +9,8 @@ import subprocess
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-ARGS = ["--impl", "reference", "--workload", "tiny_b1_h2_n256_d64", "--steps", "1", "--warmup", "3"]
+ARGS = ["--impl", "reference", "--workload", "tiny_b1_h2_n256_d64", "--steps", "1", "--warmup", "3",
+        "--ref-seconds", "2"]
 
 
 def _lines(out: str):

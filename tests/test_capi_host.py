@@ -101,11 +101,52 @@ def test_padded_dim(lib):
 def test_pv_mode_names(lib):
     assert lib.pv_mode() == lib.SAGE_PV_FP32 == 0
     assert lib.pv_mode("fp8", "fp16+fp32") == lib.pv_mode("fp8", "fp32+fp16") == lib.SAGE_PV_FP16_FP32 == 1
-    assert lib.pv_mode("fp16", "fp32") == lib.pv_mode("fp16", "fp16") == lib.SAGE_PV16_FP32 == 2
+    assert lib.pv_mode("fp16", "fp32") == lib.SAGE_PV16_FP32 == 2
     assert lib.pv_mode("fp16", "fp16+fp32") == lib.SAGE_PV16_FP16_FP32 == 3
+    assert lib.pv_mode("fp16", "fp16") == lib.SAGE_PV16_FP16 == 6  # named, and rejected by the library
     for bad in (("fp8", "fp16"), ("int8", "fp32"), ("fp16", "bf16")):
         with pytest.raises(ValueError):
             lib.pv_mode(*bad)
+
+
+def test_pure_fp16_accumulation_is_rejected_not_substituted(lib):
+    # pv_accum_dtype "fp16" with FP16 operands: SAGE_ERR_UNSUPPORTED from every entry point that
+    # takes a P.V mode, before any GPU work (no silent fp32 accumulation in its place)
+    U = lib.SAGE_ERR_UNSUPPORTED
+    assert _attn(lib, pv=lib.SAGE_PV16_FP16) == U
+    c = lib.capi
+    assert c.sage_attn_noalloc(FAKE, FAKE + 0x100000000, FAKE + 0x200000000, FAKE + 0x300000000, 1, 2, 2, 256, 64,
+                               lib.SAGE_FP16, lib.SAGE_HND, 0, 0.0, lib.SAGE_PV16_FP16, None) == U
+    assert c.sage_attn_quantized(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE, None, FAKE + 0x300000000, 1, 2, 2, 256, 64,
+                                 lib.SAGE_FP16, lib.SAGE_HND, 0, 0.0, lib.SAGE_PV16_FP16, None, None) == U
+
+
+def test_mma_probe_argument_checks(lib):
+    ops = ctypes.c_double(0.0)
+    E = lib.SAGE_ERR_INVALID_ARG
+    assert lib.capi.sage_mma_probe(3, 10, ctypes.byref(ops), None) == E
+    assert lib.capi.sage_mma_probe(0, 0, ctypes.byref(ops), None) == E
+    assert lib.capi.sage_mma_probe(0, 10, None, None) == E
+
+
+def test_injected_arch_and_allocation_failures(lib):
+    """SAGE_ERR_ARCH and SAGE_ERR_OOM through the host-side test hook, with no GPU: the checks run in
+    their documented order (arguments, device, workspace) and nothing reaches the device."""
+    c = lib.capi
+    try:
+        c.sage_test_inject(90, 0)                         # an sm_90 device
+        assert _attn(lib) == lib.SAGE_ERR_ARCH
+        assert lib.sage_device_supported() is False
+        assert _attn(lib, d=0) == lib.SAGE_ERR_INVALID_ARG  # argument checks still come first
+        c.sage_test_inject(100, 2)                        # a B200 whose next two allocations fail
+        assert c.sage_device_supported() == 1
+        assert _attn(lib) == lib.SAGE_ERR_OOM
+        fake = [FAKE + (i << 32) for i in range(9)]
+        assert c.sage_quantize(fake[0], fake[1], fake[2], 1, 2, 2, 256, 64, lib.SAGE_FP16, lib.SAGE_HND, 0, None,
+                               *fake[3:], FAKE, None, None) == lib.SAGE_ERR_OOM
+    finally:
+        c.sage_test_inject(0, 0)
+    assert c.sage_device_supported() in (0, 1)
 
 
 def test_selftest_budget_checks(lib):

@@ -111,9 +111,9 @@ def test_rejects_bad_inputs(lib):
     assert e.value.status == lib.SAGE_ERR_INVALID_ARG
 
 
-FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA, W.BY_NAME["pad_sweep_b8_h16_n16384_d96_causal"],
-        W.BY_NAME["pad_sweep_b8_h16_n16384_d64_full"], W.BY_NAME["pad_sweep_b8_h16_n1024_d96_full"]] + W.FP16_PV + \
-    W.OPTIONS + W.FP32_ACC
+# every point of the head-dim padding sweep (N in {1K, 2K, 4K, 16K}, d in {96, 64}, both masks) at full size
+FULL = [W.IMAGE_DIT, W.VIDEO_DIT, W.LLM_GQA] + list(W.pad_sweep()) + W.FP16_PV + W.OPTIONS + W.FP32_ACC + \
+    W.HEAD_DIM_256
 
 
 def _rows(out, layout, b, h, rows):

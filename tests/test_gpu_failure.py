@@ -25,3 +25,26 @@ def test_wait_timeout_is_reported_and_the_context_survives(lib):
     em = emulate.emulate(quant.quantize(q, k, v, "HND", 0), True, 0.125, **emulate.lazy_reading(0))
     check_vs_exact(out_hnd(out, "HND"), attention.attention_f64(q, k, v, "HND", True, 0.125),
                    em.reshape(1, 2, -1, w.d)[:, :, :w.N], nkeys(w.N, True), vmax_of(v), w.name, w.dist, 0)
+
+
+def test_injected_allocation_failure_is_reported_and_the_next_call_runs(lib):
+    # the workspace allocation of the first call fails (host-side injection, nothing reaches the
+    # device); the call reports SAGE_ERR_OOM and queues no work, and the next call is whole
+    w = W.TINY.with_(name="after_oom", N=300)
+    q, k, v = (cuda(t) for t in W.make_inputs(w))
+    out = torch.full_like(q, 7.0)
+    try:
+        lib.capi.sage_test_inject(0, 1)
+        with pytest.raises(lib.SageError) as e:
+            lib.sage_attn(q, k, v, "HND", False, 0.125, out=out)
+        assert e.value.status == lib.SAGE_ERR_OOM
+    finally:
+        lib.capi.sage_test_inject(0, 0)
+    torch.cuda.synchronize()
+    assert bool((out == 7.0).all())  # nothing was written
+    assert lib.capi.sage_check_status(torch.cuda.current_stream().cuda_stream) == lib.SAGE_OK
+    ref = lib.sage_attn(q, k, v, "HND", False, 0.125)
+    lib.sage_check_status()
+    again = lib.sage_attn(q, k, v, "HND", False, 0.125, out=out)
+    lib.sage_check_status()
+    assert torch.equal(again.view(torch.int16), ref.view(torch.int16))

@@ -82,3 +82,30 @@ def test_quantize_bit_exact_full_size_sampled_heads(lib, w):
                              slice_heads(v, w.layout, b, [hk]), w.layout, w.pv_mode, w.q_gran, w.smooth_v)
         _assert_same(got, ref, q_sel=(slice(b, b + 1), slice(hk * G, (hk + 1) * G)),
                      kv_sel=(slice(b, b + 1), slice(hk, hk + 1)))
+
+
+def test_k_mean_follows_the_header_contract(lib):
+    """km from sage_quantize through the C ABI, against the summation order include/sage.h states,
+    written out here in plain Python float32 arithmetic on a ragged N (the last block holds 45 tokens,
+    so its last groups are partial or empty): groups of 16 tokens summed in order from +0.0, the
+    pairwise tree over a block's 8 groups, the block partials in block order, one division by N."""
+    w = W.TINY.with_(name="km_contract", N=300, d=40, Hq=2, Hkv=1, dist="normal_koffset")
+    q, k, v = W.make_inputs(w)
+    z = lib.sage_quantize(cuda(q), cuda(k), cuda(v), w.layout, "fp32")
+    lib.sage_check_status()
+    got = z["km"].cpu().numpy()[0, 0, :w.d]
+    f32 = np.float32
+    kk = k[0, 0].float().numpy()  # (N, d), exact widening of the fp16 inputs
+    for c in range(w.d):
+        total = f32(0.0)
+        for b0 in range(0, w.N, 128):
+            g = []
+            for g0 in range(b0, b0 + 128, 16):
+                acc = f32(0.0)
+                for n in range(g0, min(g0 + 16, w.N)):
+                    acc = f32(acc + f32(kk[n, c]))
+                g.append(acc)
+            part = f32(f32(f32(g[0] + g[1]) + f32(g[2] + g[3])) + f32(f32(g[4] + g[5]) + f32(g[6] + g[7])))
+            total = f32(total + part)
+        want = f32(total / f32(w.N))
+        assert got[c].view(np.uint32) == np.asarray(want).view(np.uint32), (c, got[c], want)

@@ -115,7 +115,11 @@ OPTIONS = [IMAGE_DIT.with_(name="image_dit_b2_h24_n4096_d64_qthread_smoothv", q_
 # The video-DiT inputs with fp32 P.V accumulation (the default mode) instead of fp16+fp32.
 FP32_ACC = [VIDEO_DIT.with_(name="video_dit_b1_h24_n32768_d128_nhd_fp32acc", pv_mode=0)]
 
-ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV + OPTIONS + FP32_ACC
+# Head dim 256 (the largest padded size): the kernel's 256-column output tile.
+HEAD_DIM_256 = [Workload("d256_b2_h16_n8192", 2, 16, 16, 8192, 256, "fp16", "HND", False, "normal", 0, 6),
+                Workload("d256_b2_h16_n8192_causal", 2, 16, 16, 8192, 256, "fp16", "HND", True, "normal", 0, 6)]
+
+ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV + OPTIONS + FP32_ACC + HEAD_DIM_256
 BY_NAME = {w.name: w for w in ALL}
 
 
