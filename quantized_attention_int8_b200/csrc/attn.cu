@@ -400,12 +400,8 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       const bool rescale = MODE == 0 && i > 0 && __any_sync(0xffffffffu, alpha != 1.f);
       // p * 448 * 2^-kTau = 2^(s*f - m + log2 448 - kTau) -> E4M3, 4 keys per 32-bit word;
       // FP16 P.V: p = 2^(s*f - m) -> fp16, 2 keys per word
-      // row sums: four scalar partial sums, or in the non-causal d = 128 fp32-accumulation FP8
-      // instance the same four as two packed f32x2 adds (each lane rounds as the scalar add does;
-      // measured +7% there, and 10-24% slower at d = 64 and in fp16+fp32 mode)
-      constexpr bool PACKED_SUM = DQK == 128 && MODE == 0 && !CAUSAL && !PV16;
+      // four scalar partial row sums (packed f32x2 adds measured slower in every instance)
       float rs[4] = {0.f, 0.f, 0.f, 0.f};
-      float2 rs01 = make_float2(0.f, 0.f), rs23 = make_float2(0.f, 0.f);
       uint32_t pw[C::ROWB / 4];
 #pragma unroll
       for (int c4 = 0; c4 < BN / 4; ++c4) {
@@ -416,7 +412,9 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
           float x0, x1;
           // the exact score S = (1.5 * 2^23 + S) - 1.5 * 2^23 (same binade: no rounding), then
           // S * f + bias with one rounding, as the scores were integers converted to float
-          if (DQK >= 128 && MODE == 0) {  // packed FMA measured faster only in this configuration
+          // packed f32x2 math measured faster only in the causal fp32-accumulation instances
+          // (scalar: +13% non-causal at d = 128, +18% at d = 256, -8% causal)
+          if (DQK >= 128 && MODE == 0 && CAUSAL) {
             const float2 sc = __fadd2_rn(make_float2(__uint_as_float(s[c]), __uint_as_float(s[c + 1])),
                                          make_float2(-kSBias, -kSBias));
             const float2 x = __ffma2_rn(sc, make_float2(f, f), make_float2(bias, bias));
@@ -432,14 +430,8 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
             pv[e] = (c < lim) ? pv[e] : 0.f;
             pv[e + 1] = (c + 1 < lim) ? pv[e + 1] : 0.f;
           }
-          if (!PACKED_SUM) {
-            rs[e] += pv[e];
-            rs[e + 1] += pv[e + 1];
-          }
-        }
-        if (PACKED_SUM) {
-          rs01 = __fadd2_rn(rs01, make_float2(pv[0], pv[1]));
-          rs23 = __fadd2_rn(rs23, make_float2(pv[2], pv[3]));
+          rs[e] += pv[e];
+          rs[e + 1] += pv[e + 1];
         }
         if (PV16) {
           pw[2 * c4] = pack2<__half>(pv[0], pv[1]);
@@ -448,7 +440,6 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
           pw[c4] = e4m3x2(pv[0], pv[1]) | (e4m3x2(pv[2], pv[3]) << 16);
         }
       }
-      if (PACKED_SUM) rs[0] = rs01.x, rs[1] = rs01.y, rs[2] = rs23.x, rs[3] = rs23.y;
       l = l * alpha + ((rs[0] + rs[1]) + (rs[2] + rs[3]));
       m = m_new;
       if (MODE == 0 && i > 0) {

@@ -375,6 +375,41 @@ __global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
   }
 }
 
+// K mean of channel c of one (batch, kv head) from pass 1's per-block partial sums: added one by one
+// in block order from +0.0, then one division by the token count (the bit-exact contract's order).
+__device__ __forceinline__ float k_mean_of(const QuantParams& p, long long base, int nblk, int nk, int c) {
+  const float* ks = p.ksum_part + base + c;
+  float acc = 0.f;
+#pragma unroll 8
+  for (int i = 0; i < nblk; ++i) acc = __fadd_rn(acc, ks[(size_t)i * p.m.dp]);  // the loads overlap
+  return (c < p.m.d && nk > 0) ? __fdiv_rn(acc, (float)nk) : 0.f;
+}
+
+// V's channel amax (of v, or with smoothing of v - mean: its max |.| is reached at the channel's
+// largest or smallest v, since rounding v - mean to float32 is monotonic in v) and token mean.
+__device__ __forceinline__ float v_amax_of(const QuantParams& p, long long base, int nblk, int nk, int c, float* mean) {
+  const float* vmx = p.vmax_part + base + c;
+  if (p.smooth_v) {
+    const float* vsum = p.vsum_part + base + c;
+    const float* vmin = p.vmin_part + base + c;
+    float vacc = 0.f, hi = -INFINITY, lo = INFINITY;
+#pragma unroll 8
+    for (int i = 0; i < nblk; ++i) {  // sums stay in block order
+      vacc = __fadd_rn(vacc, vsum[(size_t)i * p.m.dp]);
+      hi = fmaxf(hi, vmx[(size_t)i * p.m.dp]);
+      lo = fminf(lo, vmin[(size_t)i * p.m.dp]);
+    }
+    const float m = (c < p.m.d && nk > 0) ? __fdiv_rn(vacc, (float)nk) : 0.f;
+    *mean = m;
+    return nk > 0 ? fmaxf(fabsf(__fsub_rn(hi, m)), fabsf(__fsub_rn(lo, m))) : 0.f;
+  }
+  float am = 0.f;
+#pragma unroll 8
+  for (int i = 0; i < nblk; ++i) am = fmaxf(am, vmx[(size_t)i * p.m.dp]);
+  *mean = 0.f;
+  return am;
+}
+
 __global__ void quant_finalize_kernel(QuantParams p) {
   allow_next_grid();
   wait_for_previous_grid();  // pass 1's partial sums
@@ -383,34 +418,10 @@ __global__ void quant_finalize_kernel(QuantParams p) {
   const int dp = p.m.dp, nblk = (sv.nk + 127) / 128;
   const long long base = (sv.k_row0 + h * p.m.k_head_rows) / 128 * dp;
   for (int c = threadIdx.x; c < dp; c += blockDim.x) {
-    const float* ks = p.ksum_part + base + c;
-    const float* vm = p.vmax_part + base + c;
-    float acc = 0.f, am = 0.f;
-    if (p.smooth_v) {
-      // V - mean(V): its max |.| per channel is reached at the channel's largest or smallest v,
-      // since rounding v - mean to float32 is monotonic in v
-      const float* vsum = p.vsum_part + base + c;
-      const float* vmin = p.vmin_part + base + c;
-      float vacc = 0.f, hi = -INFINITY, lo = INFINITY;
-#pragma unroll 8
-      for (int i = 0; i < nblk; ++i) {  // sums stay in block order
-        acc = __fadd_rn(acc, ks[(size_t)i * dp]);
-        vacc = __fadd_rn(vacc, vsum[(size_t)i * dp]);
-        hi = fmaxf(hi, vm[(size_t)i * dp]);
-        lo = fminf(lo, vmin[(size_t)i * dp]);
-      }
-      const float mean = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(vacc, (float)sv.nk) : 0.f;
-      am = sv.nk > 0 ? fmaxf(fabsf(__fsub_rn(hi, mean)), fabsf(__fsub_rn(lo, mean))) : 0.f;
-      p.vm[(size_t)bh * dp + c] = mean;
-    } else {
-#pragma unroll 8
-      for (int i = 0; i < nblk; ++i) {  // sums stay in block order; the loads overlap
-        acc = __fadd_rn(acc, ks[(size_t)i * dp]);
-        am = fmaxf(am, vm[(size_t)i * dp]);
-      }
-      if (p.vm) p.vm[(size_t)bh * dp + c] = 0.f;
-    }
-    p.km[(size_t)bh * dp + c] = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(acc, (float)sv.nk) : 0.f;
+    float mean;
+    const float am = v_amax_of(p, base, nblk, sv.nk, c, &mean);
+    if (p.vm) p.vm[(size_t)bh * dp + c] = mean;
+    p.km[(size_t)bh * dp + c] = k_mean_of(p, base, nblk, sv.nk, c);
     p.vs[(size_t)bh * dp + c] = __fdiv_rn(am, p.vmax_code);
     p.vinv[(size_t)bh * dp + c] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
   }
@@ -439,6 +450,31 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
   const bool vec = isk ? p.vec_k : p.vec_v;
   const int blk0 = (gridDim.x - 1 - blockIdx.x) * p.bpc, blk1 = min((sv.nk + 127) / 128, blk0 + p.bpc);
   if (blk0 >= blk1) return;  // past the end of this sequence (the whole CTA leaves)
+  // Short sequences (p.fold): no finalize launch; every CTA computes its head's K mean, or V's
+  // scales and mean, from pass 1's partials in the same order, and the head's first CTA writes
+  // them out.  Otherwise the finalize kernel has written them.
+  __shared__ float hv[2][256];  // K: mean; V: 1 / scale, mean
+  const int hh = isk ? y : y - p.m.Hkv;
+  const size_t bhh = (size_t)b * p.m.Hkv + hh;
+  if (p.fold) {
+    const int c = threadIdx.x, nblk = (sv.nk + 127) / 128;
+    const long long base = (sv.k_row0 + hh * p.m.k_head_rows) / 128 * dp;
+    if (isk) {
+      const float km = k_mean_of(p, base, nblk, sv.nk, c);
+      hv[0][c] = km;
+      if (blk0 == 0) p.km[bhh * dp + c] = km;
+    } else {
+      float mean;
+      const float am = v_amax_of(p, base, nblk, sv.nk, c, &mean);
+      hv[0][c] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
+      hv[1][c] = mean;
+      if (blk0 == 0) {
+        p.vs[bhh * dp + c] = __fdiv_rn(am, p.vmax_code);
+        if (p.vm) p.vm[bhh * dp + c] = mean;
+      }
+    }
+    __syncthreads();
+  }
   uint4 v[16];
   load_tile<T>(v, src + (long long)blk0 * 128 * tstride, tstride, d, min(128, sv.nk - blk0 * 128), vec, tc);
   for (int blk = blk0; blk < blk1; ++blk) {
@@ -450,7 +486,7 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
     const size_t bh = (size_t)b * p.m.Hkv + h;
     float km[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) km[e] = p.km[bh * dp + tc.c0 + e];
+    for (int e = 0; e < 8; ++e) km[e] = p.fold ? hv[0][tc.c0 + e] : p.km[bh * dp + tc.c0 + e];
     // padded channels read 0 and have mean 0; padded rows are masked by store_int8_tile
     auto x = [&](int r, int e) -> float { return __fsub_rn(elem<T>(v[r], e), km[e]); };
     // max |k - mean| per channel is reached at the channel's largest or smallest k, since
@@ -495,9 +531,9 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
     const size_t bh = (size_t)b * p.m.Hkv + h;
     float inv[8], mean[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) inv[e] = p.vinv[bh * dp + tc.c0 + e];
+    for (int e = 0; e < 8; ++e) inv[e] = p.fold ? hv[0][tc.c0 + e] : p.vinv[bh * dp + tc.c0 + e];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) mean[e] = SMOOTH_V ? p.vm[bh * dp + tc.c0 + e] : 0.f;
+    for (int e = 0; e < 8; ++e) mean[e] = SMOOTH_V ? (p.fold ? hv[1][tc.c0 + e] : p.vm[bh * dp + tc.c0 + e]) : 0.f;
     // (v - mean) * inv; tokens past N give 0 (with smoothing the subtraction would not)
     auto vx = [&](int r, int e) -> float {
       if (!SMOOTH_V) return __fmul_rn(elem<T>(v[r], e), inv[e]);  // tokens past N load as 0 -> code 0
@@ -590,8 +626,13 @@ static cudaError_t launch_quant_t(const QuantParams& p_in, cudaStream_t st) {
   else quant_pass1_kernel<T, false, false><<<grid1, dp, smem, st>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  e = launch_dependent(quant_finalize_kernel, dim3(B * Hkv), dim3(dp), st, p);
-  if (e != cudaSuccess) return e;
+  // Up to 64 blocks per sequence pass 2 folds the finalize step in (each of its CTAs reads its head's
+  // partials; measured faster than a separate launch there), beyond that a finalize launch.
+  p.fold = nblk1 <= 64 ? 1 : 0;
+  if (!p.fold) {
+    e = launch_dependent(quant_finalize_kernel, dim3(B * Hkv), dim3(dp), st, p);
+    if (e != cudaSuccess) return e;
+  }
   const int nblk2 = p.nblk_k > 0 ? p.nblk_k : 1;
   const dim3 grid2((nblk2 + p.bpc - 1) / p.bpc, 2 * Hkv, B);
   return p.smooth_v ? launch_dependent(quant_pass2_kernel<T, true>, grid2, dim3(dp), st, p, smem)

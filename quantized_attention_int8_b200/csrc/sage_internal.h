@@ -102,6 +102,7 @@ struct QuantParams {
   int prefetch;      // stream the next block into shared memory while one is processed (dp <= 128)
   float vmax_code;   // 448 (FP8 P.V, fp32 accumulation) or 1 (the other P.V modes)
   int v_fp16;        // V codes are fp16 (FP16 P.V) instead of E4M3; v8t then holds 2 bytes per code
+  int fold;          // pass 2 computes the K mean and V scales itself (no finalize launch)
 };
 
 struct FwdParams {
