@@ -50,7 +50,8 @@ typedef enum {
   SAGE_ERR_ARCH = 3,
   SAGE_ERR_CUDA = 4,
   SAGE_ERR_OOM = 5,
-  SAGE_ERR_TIMEOUT = 6
+  SAGE_ERR_TIMEOUT = 6,
+  SAGE_ERR_BOUNDS = 7
 } sage_status;
 
 typedef enum { SAGE_HND = 0, SAGE_NHD = 1 } sage_layout;
@@ -224,9 +225,10 @@ sage_status sage_selftest_wait_timeout(int budget_us, void* stream);
 sage_status sage_mma_probe(int kind, int iters, double* ops, void* stream);
 
 /* Synchronizes `stream`, then reports (and clears) the device-side error word:
- * SAGE_ERR_TIMEOUT if a kernel gave up on a bounded wait, SAGE_ERR_INVALID_ARG
- * for a flagged tile record or cu_seqlens table, SAGE_ERR_CUDA for a pending CUDA
- * error.  The error word is one per device, not per stream: it collects the
+ * SAGE_ERR_TIMEOUT if a kernel gave up on a bounded wait, SAGE_ERR_BOUNDS if a
+ * kernel of the checked build skipped a store outside its buffer (see
+ * sage_checked_build), SAGE_ERR_INVALID_ARG for a flagged tile record or
+ * cu_seqlens table, SAGE_ERR_CUDA for a pending CUDA error.  The error word is one per device, not per stream: it collects the
  * flags of every call on the current device since it was last read, whatever
  * stream they ran on, and the first sage_check_status to read it (on any stream)
  * reports and clears them.  Only `stream` is synchronized, so a call still
@@ -247,6 +249,25 @@ int sage_device_supported(void);
  * fail with SAGE_ERR_OOM before touching the device (0 clears it).  Process-wide;
  * not for use outside tests. */
 void sage_test_inject(int fake_cc, int fail_allocs);
+
+/* 1 for the checked build of this library (compiled with -DSAGE_CHECKED, shipped
+ * beside the normal one as libsage_b200_checked.so), else 0.  In the checked build
+ * every global-memory store of the quantize kernels and of the fused attention
+ * kernel first tests that its bytes lie inside the buffer they belong to (sized as
+ * this header states: out, the sage_quantize outputs, the workspace's parts); a
+ * store outside is skipped, never made, and sage_check_status reports
+ * SAGE_ERR_BOUNDS.  (The per-sequence table of packed batches and the tiles of
+ * sage_qk_int32 are written at indices that their launch bounds: not checked.)
+ * Results are bit-identical to the normal build's; the normal build compiles the
+ * tests out. */
+int sage_checked_build(void);
+
+/* Test hook for the checked build (no counterpart on the pages): bytes > 0
+ * narrows the extent the kernels take for `out` to its first `bytes` bytes, so a
+ * call's stores past them are skipped and reported (SAGE_ERR_BOUNDS); 0 restores
+ * the full size.  No effect on the normal build.  Process-wide; not for use
+ * outside tests. */
+void sage_test_out_limit(long long bytes);
 
 /* Largest workspace sage_attn_noalloc can hold: 64 MiB (for example B=2, H=24,
  * N=4096, d=64 with pv_mode SAGE_PV_FP32 needs about 38 MiB). */

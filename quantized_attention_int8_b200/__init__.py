@@ -28,14 +28,16 @@ import torch
 __all__ = [
     "SageError", "sage_attn", "sage_quantize", "sage_attn_quantized", "sage_qk_int32", "sage_check_status",
     "sage_workspace_bytes", "sage_device_supported", "sage_status_string", "padded_dim", "LIB_PATH", "capi",
-    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "pv_mode", "sage_attn_varlen", "SageOpts", "opts",
+    "sage_attn_noalloc", "SAGE_NOALLOC_MAX_BYTES", "load_checked", "CHECKED_LIB_PATH", "pv_mode", "sage_attn_varlen", "SageOpts", "opts",
     "sageattn", "sageattn_qk_int8_pv_fp8_cuda", "sageattn_qk_int8_pv_fp16_cuda", "sageattn_varlen",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200.so")
+# the same library compiled with -DSAGE_CHECKED: every kernel store tests its extent first
+CHECKED_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsage_b200_checked.so")
 
 SAGE_OK, SAGE_ERR_INVALID_ARG, SAGE_ERR_UNSUPPORTED, SAGE_ERR_ARCH, SAGE_ERR_CUDA, SAGE_ERR_OOM, \
-    SAGE_ERR_TIMEOUT = range(7)
+    SAGE_ERR_TIMEOUT, SAGE_ERR_BOUNDS = range(8)
 SAGE_HND, SAGE_NHD = 0, 1
 SAGE_FP16, SAGE_BF16, SAGE_FP32 = 0, 1, 2
 SAGE_PV_FP32, SAGE_PV_FP16_FP32, SAGE_PV16_FP32, SAGE_PV16_FP16_FP32, SAGE_PV16_FP16 = 0, 1, 2, 3, 6
@@ -79,12 +81,12 @@ def opts(qk_quant_gran: str = "per_block", smooth_v: bool = False) -> SageOpts:
     return SageOpts(_GRANS[qk_quant_gran], 1 if smooth_v else 0)
 
 
-def _load() -> ctypes.CDLL:
-    if not os.path.exists(LIB_PATH):
+def _load(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
         raise ImportError(
-            f"{LIB_PATH} is not built; run `python quantized_attention_int8_b200/build_lib.py` "
+            f"{path} is not built; run `python quantized_attention_int8_b200/build_lib.py` "
             "(this package has no CPU fallback)")
-    lib = ctypes.CDLL(LIB_PATH)
+    lib = ctypes.CDLL(path)
     P, I, F, Z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     sig = {
         "sage_attn": ([P, P, P, P, I, I, I, I, I, I, I, I, F, I, P], I),
@@ -100,6 +102,8 @@ def _load() -> ctypes.CDLL:
         "sage_selftest_wait_timeout": ([I, P], I),
         "sage_mma_probe": ([I, I, ctypes.POINTER(ctypes.c_double), P], I),
         "sage_test_inject": ([I, I], None),
+        "sage_test_out_limit": ([ctypes.c_longlong], None),
+        "sage_checked_build": ([], I),
         "sage_attn_varlen": ([P, P, P, P, P, P, I, I, I, ctypes.c_longlong, ctypes.c_longlong, I, I, I, I, I, F, I, P,
                               P], I),
     }
@@ -110,6 +114,15 @@ def _load() -> ctypes.CDLL:
 
 
 capi = _load()
+
+
+def load_checked() -> ctypes.CDLL:
+    """The checked build (``libsage_b200_checked.so``) with the same signatures as ``capi``.
+
+    Its kernels test every global store against the buffer it belongs to, skip one that falls
+    outside and report it through ``sage_check_status`` (SAGE_ERR_BOUNDS).  A second, independent
+    copy of the library: its device state (error words, no-alloc workspace) is its own."""
+    return _load(CHECKED_LIB_PATH)
 
 
 class SageError(RuntimeError):

@@ -1,6 +1,7 @@
-"""Builds the CUDA library (libsage_b200.so) in-tree with nvcc for sm_100a.
+"""Builds the CUDA library in-tree with nvcc for sm_100a: libsage_b200.so and its checked
+twin libsage_b200_checked.so (-DSAGE_CHECKED: every kernel store tests its extent first).
 
-Usage: python quantized_attention_int8_b200/build_lib.py [--force] [--ptxas-info]
+Usage: python quantized_attention_int8_b200/build_lib.py [--force] [--ptxas-info] [--no-checked]
 
 Run it as a script (not as a module of the package): importing the package
 loads the library, which may not exist yet or may be stale.
@@ -17,6 +18,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libsage_b200.so")
+LIB_CHECKED = os.path.join(PKG, "libsage_b200_checked.so")
 SOURCES = ["api.cu", "attn.cu", "quant.cu"]
 HEADERS = ["sm100.cuh", "sage_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -29,20 +31,20 @@ def _nvcc() -> str:
     return cand
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = [os.path.join(CSRC, f) for f in SOURCES + HEADERS] + [os.path.join(INCLUDE, "sage.h")]
     return any(os.path.getmtime(p) > t for p in deps)
 
 
-def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) -> str:
-    if not force and not _stale():
-        return LIB
-    tmp = LIB + ".tmp"
+def _build_one(lib: str, defines: list[str], force: bool, ptxas_info: bool, verbose: bool) -> str:
+    if not force and not _stale(lib):
+        return lib
+    tmp = lib + ".tmp"
     cmd = [_nvcc(), "-O3", "-std=c++17", *ARCH, "-lineinfo", "-Xcompiler", "-fPIC,-O2", "-shared",
-           "--threads", "4", f"-I{INCLUDE}", f"-I{CSRC}", "-o", tmp,
+           "--threads", "4", *defines, f"-I{INCLUDE}", f"-I{CSRC}", "-o", tmp,
            *[os.path.join(CSRC, f) for f in SOURCES]]
     if ptxas_info:
         cmd[1:1] = ["-Xptxas", "-v"]
@@ -53,9 +55,18 @@ def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False) 
         raise RuntimeError(f"nvcc failed ({r.returncode}):\n{r.stdout}\n{r.stderr}")
     if ptxas_info or verbose:
         sys.stderr.write(r.stdout + r.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+    return lib
+
+
+def build(force: bool = False, ptxas_info: bool = False, verbose: bool = False, checked: bool = True) -> str:
+    """Builds the library (and, unless checked=False, its checked twin); returns the library's path."""
+    _build_one(LIB, [], force, ptxas_info, verbose)
+    if checked:
+        _build_one(LIB_CHECKED, ["-DSAGE_CHECKED"], force, ptxas_info, verbose)
     return LIB
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, ptxas_info="--ptxas-info" in sys.argv, verbose=True)
+    build(force="--force" in sys.argv, ptxas_info="--ptxas-info" in sys.argv, verbose=True,
+          checked="--no-checked" not in sys.argv)

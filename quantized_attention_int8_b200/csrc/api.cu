@@ -234,6 +234,23 @@ cudaError_t workspace_alloc(void** ptr, size_t bytes, cudaStream_t st) {
   return cudaMallocFromPoolAsync(ptr, bytes, pool, st);
 }
 
+// Store extents of the checked build (-DSAGE_CHECKED): each buffer's size as the header states it.
+Extent extent_of(const void* ptr, size_t bytes) {
+  Extent x;
+  x.base = static_cast<unsigned char*>(const_cast<void*>(ptr));
+  x.bytes = ptr ? bytes : 0;
+  return x;
+}
+
+std::atomic<long long> g_out_limit{0};  // test hook: narrows the output extent when > 0
+
+Extent out_extent(const Dims& m, const void* out) {
+  size_t bytes = (size_t)m.total_q * m.Hq * m.d * 2;  // fp16 / bf16 output
+  const long long lim = g_out_limit.load();
+  if (lim > 0 && (size_t)lim < bytes) bytes = (size_t)lim;
+  return extent_of(out, bytes);
+}
+
 struct QuantBufs {
   const SeqDesc* seqs;  // packed batches: the per-sequence table (else nullptr)
   float* vm;            // V's token mean (read only when V is smoothed)
@@ -267,6 +284,7 @@ sage_status run_fwd(const Dims& m, const QuantBufs& qb, void* out, int dtype, in
   p.nblk_q = m.nblk_q;
   p.G = m.G;
   p.vec_out = (m.d % 8 == 0) && aligned16(out);
+  p.x_out = out_extent(m, out);
   p.scale_log2 = resolve_scale(sm_scale, m.d) * 1.4426950408889634f;
   return from_cuda(launch_fwd(tq, tk, tv, p, dtype, causal, pv_mode, st));
 }
@@ -299,6 +317,25 @@ WsLayout ws_layout(const Dims& m, int pv_mode, const Opts& o) {
   w.seqs = take(m.packed ? (size_t)m.B * sizeof(SeqDesc) : 0);
   w.total = off;
   return w;
+}
+
+// Extents of every buffer the quantize kernels write, from the pointers already in p.
+void set_quant_extents(QuantParams* p, const Dims& m, int pv_mode, const Opts& o) {
+  const size_t per_head = (size_t)m.B * m.Hkv * m.dp * 4;
+  const size_t part = (size_t)m.k_rows / 128 * m.dp * 4;
+  p->x_q8 = extent_of(p->q8, (size_t)m.q_rows * m.dp);
+  p->x_qs = extent_of(p->qs, ((size_t)m.q_rows >> o.q_gran_log2) * 4);
+  p->x_k8 = extent_of(p->k8, (size_t)m.k_rows * m.dp);
+  p->x_ks = extent_of(p->ks, (size_t)m.k_rows / 128 * 4);
+  p->x_km = extent_of(p->km, per_head);
+  p->x_v8t = extent_of(p->v8t, (size_t)m.k_rows * m.dp * (pv_mode_fp16_operands(pv_mode) ? 2 : 1));
+  p->x_vs = extent_of(p->vs, per_head);
+  p->x_vm = extent_of(p->vm, per_head);
+  p->x_vinv = extent_of(p->vinv, per_head);
+  p->x_ksum = extent_of(p->ksum_part, part);
+  p->x_vmax = extent_of(p->vmax_part, part);
+  p->x_vsum = extent_of(p->vsum_part, part);
+  p->x_vmin = extent_of(p->vmin_part, part);
 }
 
 QuantParams quant_params(const Dims& m, const void* q, const void* k, const void* v, int dtype, int layout,
@@ -360,6 +397,7 @@ sage_status attend_on(const Dims& m, unsigned char* ws, const void* q, const voi
   qp.vsum_part = reinterpret_cast<float*>(ws + w.vsum);
   qp.vmin_part = reinterpret_cast<float*>(ws + w.vmin);
   qp.vinv = reinterpret_cast<float*>(ws + w.vinv);
+  set_quant_extents(&qp, m, pv_mode, o);
   sage_status s = from_cuda(launch_quantize(qp, st));
   if (s == SAGE_OK) s = run_fwd(m, qb, out, dtype, layout, causal, sm_scale, pv_mode, o, st);
   return s;
@@ -458,6 +496,7 @@ sage_status sage_quantize(const void* q, const void* k, const void* v, int B, in
   qp.vsum_part = o.smooth_v ? reinterpret_cast<float*>(scratch + 2 * part) : nullptr;
   qp.vmin_part = o.smooth_v ? reinterpret_cast<float*>(scratch + 3 * part) : nullptr;
   qp.vinv = reinterpret_cast<float*>(scratch + nparts * part);
+  set_quant_extents(&qp, m, pv_mode, o);
   s = from_cuda(launch_quantize(qp, st));
   const cudaError_t ef = cudaFreeAsync(scratch, st);
   if (s == SAGE_OK && ef != cudaSuccess) s = from_cuda(ef);
@@ -534,8 +573,12 @@ sage_status sage_check_status(void* stream) {
   cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
   if (e != cudaSuccess) return SAGE_ERR_CUDA;
   int flags = 0;
+  int qflags = 0;
   if (read_clear_device_error(&flags) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (read_clear_quant_error(&qflags) != cudaSuccess) return SAGE_ERR_CUDA;
+  flags |= qflags;
   if (flags & 1) return SAGE_ERR_TIMEOUT;
+  if (flags & SAGE_DEVERR_BOUNDS) return SAGE_ERR_BOUNDS;
   if (flags & 2) return SAGE_ERR_INVALID_ARG;
   return SAGE_OK;
 }
@@ -549,6 +592,7 @@ const char* sage_status_string(sage_status s) {
     case SAGE_ERR_CUDA: return "CUDA error";
     case SAGE_ERR_OOM: return "out of device memory";
     case SAGE_ERR_TIMEOUT: return "a kernel gave up on a bounded wait";
+    case SAGE_ERR_BOUNDS: return "a kernel skipped a store outside its buffer (checked build)";
   }
   return "unknown status";
 }
@@ -558,6 +602,16 @@ int sage_device_supported(void) { return check_device() == SAGE_OK ? 1 : 0; }
 void sage_test_inject(int fake_cc, int fail_allocs) {
   g_fake_cc.store(fake_cc > 0 ? fake_cc : 0);
   g_fail_allocs.store(fail_allocs > 0 ? fail_allocs : 0);
+}
+
+void sage_test_out_limit(long long bytes) { g_out_limit.store(bytes > 0 ? bytes : 0); }
+
+int sage_checked_build(void) {
+#ifdef SAGE_CHECKED
+  return 1;
+#else
+  return 0;
+#endif
 }
 
 }  // extern "C"

@@ -183,7 +183,8 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
   if (n_kv == 0) {
     // no row of this tile sees a key (nk = 0, or the causal offset leaves the tile empty): zeros
     if (warp < 4 && grow < nq)
-      for (int c = 0; c < p.m.d; ++c) store_elem(out + orow + c, 0.f);
+      for (int c = 0; c < p.m.d; ++c)
+        if (SAGE_STORE_OK(p.x_out, out + orow + c, sizeof(OutT), &g_device_error)) store_elem(out + orow + c, 0.f);
     return;
   }
 
@@ -542,12 +543,15 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
 #pragma unroll
             for (int e = 0; e < 16; ++e) w[e] = pack2<OutT>(of[2 * e], of[2 * e + 1]);
             uint4* dst = reinterpret_cast<uint4*>(out + orow + c0);
+            if (SAGE_STORE_OK(p.x_out, dst, 32 * sizeof(OutT), &g_device_error)) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+              for (int e = 0; e < 4; ++e) dst[e] = make_uint4(w[4 * e], w[4 * e + 1], w[4 * e + 2], w[4 * e + 3]);
+            }
           } else {
 #pragma unroll
             for (int e = 0; e < 32; ++e)
-              if (c0 + e < p.m.d) store_elem(out + orow + c0 + e, of[e]);
+              if (c0 + e < p.m.d && SAGE_STORE_OK(p.x_out, out + orow + c0 + e, sizeof(OutT), &g_device_error))
+                store_elem(out + orow + c0 + e, of[e]);
           }
         }
       }

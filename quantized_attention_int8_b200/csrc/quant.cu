@@ -33,6 +33,17 @@
 
 namespace sage {
 
+// Error word of the quantize kernels (store checks of the checked build), read and cleared by
+// sage_check_status() together with the attention kernels' word.
+__device__ int g_quant_error = 0;
+
+cudaError_t read_clear_quant_error(int* value) {
+  cudaError_t e = cudaMemcpyFromSymbol(value, g_quant_error, sizeof(int));
+  if (e != cudaSuccess) return e;
+  const int zero = 0;
+  return cudaMemcpyToSymbol(g_quant_error, &zero, sizeof(int));
+}
+
 // Programmatic dependent launch: the finalize and pass-2 grids are launched while their
 // predecessor still runs; they wait here for it to complete (and its writes to be visible)
 // before reading what it wrote.
@@ -161,7 +172,7 @@ __device__ __forceinline__ float block_max(float v, float* red) {
 // rows at or beyond `rows` (tokens past N) get code 0 whatever `val` returns for them.
 template <typename F, typename G>
 __device__ __forceinline__ void store_int8_tile_rows(int8_t* __restrict__ dst, int dp, const TileCoord& tc, G inv_of,
-                                                     int rows, F val) {
+                                                     int rows, F val, const Extent& x) {
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     const bool valid = tc.g * 16 + r < rows;
@@ -178,14 +189,15 @@ __device__ __forceinline__ void store_int8_tile_rows(int8_t* __restrict__ dst, i
       }
       w[half] = valid ? packed : 0u;
     }
-    *reinterpret_cast<uint2*>(dst + (size_t)(tc.g * 16 + r) * dp + tc.c0) = make_uint2(w[0], w[1]);
+    int8_t* const q = dst + (size_t)(tc.g * 16 + r) * dp + tc.c0;
+    if (SAGE_STORE_OK(x, q, 8, &g_quant_error)) *reinterpret_cast<uint2*>(q) = make_uint2(w[0], w[1]);
   }
 }
 
 // The same with one 127 / amax for the whole tile.
 template <typename F>
 __device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp, const TileCoord& tc, float inv, int rows,
-                                                F val) {
+                                                F val, const Extent& x) {
 #pragma unroll
   for (int r = 0; r < 16; ++r) {
     const bool valid = tc.g * 16 + r < rows;
@@ -201,7 +213,8 @@ __device__ __forceinline__ void store_int8_tile(int8_t* __restrict__ dst, int dp
       }
       w[half] = valid ? packed : 0u;
     }
-    *reinterpret_cast<uint2*>(dst + (size_t)(tc.g * 16 + r) * dp + tc.c0) = make_uint2(w[0], w[1]);
+    int8_t* const q = dst + (size_t)(tc.g * 16 + r) * dp + tc.c0;
+    if (SAGE_STORE_OK(x, q, 8, &g_quant_error)) *reinterpret_cast<uint2*>(q) = make_uint2(w[0], w[1]);
   }
 }
 
@@ -269,8 +282,9 @@ __global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
     if (!FINE_Q) {  // one scale for the 128-token block
       const float am = block_max(tile_absmax<T>(v), red);
       const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
-      store_int8_tile(p.q8 + row * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); });
-      if (threadIdx.x == 0) p.qs[row / 128] = __fdiv_rn(am, 127.f);
+      store_int8_tile(p.q8 + row * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); }, p.x_q8);
+      if (threadIdx.x == 0 && SAGE_STORE_OK(p.x_qs, p.qs + row / 128, 4, &g_quant_error))
+        p.qs[row / 128] = __fdiv_rn(am, 127.f);
     } else {  // one scale per token (q_gran 1) or per 32 tokens (q_gran 32)
       // max |q| of each of this thread's 16 tokens over its 8 channels, then over the dp/8
       // consecutive threads that hold the token's other channels
@@ -293,13 +307,16 @@ __global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
         gm = fmaxf(red[tc.g & ~1], red[tc.g | 1]);
 #pragma unroll
         for (int r = 0; r < 16; ++r) ta[r] = gm;
-        if (tc.cv == 0 && (tc.g & 1) == 0) p.qs[(row + tc.g * 16) / 32] = __fdiv_rn(gm, 127.f);
+        if (tc.cv == 0 && (tc.g & 1) == 0 && SAGE_STORE_OK(p.x_qs, p.qs + (row + tc.g * 16) / 32, 4, &g_quant_error))
+          p.qs[(row + tc.g * 16) / 32] = __fdiv_rn(gm, 127.f);
       } else if (tc.cv == 0) {
 #pragma unroll
-        for (int r = 0; r < 16; ++r) p.qs[row + tc.g * 16 + r] = __fdiv_rn(ta[r], 127.f);
+        for (int r = 0; r < 16; ++r)
+          if (SAGE_STORE_OK(p.x_qs, p.qs + row + tc.g * 16 + r, 4, &g_quant_error))
+            p.qs[row + tc.g * 16 + r] = __fdiv_rn(ta[r], 127.f);
       }
       store_int8_tile_rows(p.q8 + row * dp, dp, tc, [&](int r) { return ta[r] > 0.f ? __fdiv_rn(127.f, ta[r]) : 0.f; },
-                           rows, [&](int r, int e) { return elem<T>(v[r], e); });
+                           rows, [&](int r, int e) { return elem<T>(v[r], e); }, p.x_q8);
     }
   } else if (y < p.m.Hq + p.m.Hkv) {  // ---- K: per-block partial column sums
     const int h = y - p.m.Hq;
@@ -315,7 +332,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
     for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = acc[e];
     __syncthreads();
     const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
-    p.ksum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
+    if (SAGE_STORE_OK(p.x_ksum, p.ksum_part + base + threadIdx.x, 4, &g_quant_error))
+      p.ksum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
   } else if (SMOOTH_V) {  // ---- V, smoothed: per-block partial column sums, max and min
     const int h = y - p.m.Hq - p.m.Hkv;
     float acc[8], hi[8], lo[8];
@@ -335,17 +353,20 @@ __global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
 #pragma unroll
     for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = acc[e];
     __syncthreads();
-    p.vsum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
+    if (SAGE_STORE_OK(p.x_vsum, p.vsum_part + base + threadIdx.x, 4, &g_quant_error))
+      p.vsum_part[base + threadIdx.x] = tree8_sum(part, dp, threadIdx.x);
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = hi[e];
     __syncthreads();
-    p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
+    if (SAGE_STORE_OK(p.x_vmax, p.vmax_part + base + threadIdx.x, 4, &g_quant_error))
+      p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
     __syncthreads();
 #pragma unroll
     for (int e = 0; e < 8; ++e) part[tc.g * dp + tc.c0 + e] = lo[e];
     __syncthreads();
-    p.vmin_part[base + threadIdx.x] = tree8_min(part, dp, threadIdx.x);
+    if (SAGE_STORE_OK(p.x_vmin, p.vmin_part + base + threadIdx.x, 4, &g_quant_error))
+      p.vmin_part[base + threadIdx.x] = tree8_min(part, dp, threadIdx.x);
   } else {  // ---- V: per-block partial column amax
     const int h = y - p.m.Hq - p.m.Hkv;
     uint32_t a[4] = {0, 0, 0, 0};  // channels (2e, 2e+1), |x| as bit patterns
@@ -363,7 +384,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass1_kernel(QuantParams p) {
     }
     __syncthreads();
     const long long base = (sv.k_row0 + h * p.m.k_head_rows + n0) / 128 * dp;
-    p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
+    if (SAGE_STORE_OK(p.x_vmax, p.vmax_part + base + threadIdx.x, 4, &g_quant_error))
+      p.vmax_part[base + threadIdx.x] = tree8_max(part, dp, threadIdx.x);
   }
   __syncthreads();  // `part` and `red` are reused by the next block
   if (blk + 1 < blk1) {
@@ -420,10 +442,11 @@ __global__ void quant_finalize_kernel(QuantParams p) {
   for (int c = threadIdx.x; c < dp; c += blockDim.x) {
     float mean;
     const float am = v_amax_of(p, base, nblk, sv.nk, c, &mean);
-    if (p.vm) p.vm[(size_t)bh * dp + c] = mean;
-    p.km[(size_t)bh * dp + c] = k_mean_of(p, base, nblk, sv.nk, c);
-    p.vs[(size_t)bh * dp + c] = __fdiv_rn(am, p.vmax_code);
-    p.vinv[(size_t)bh * dp + c] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
+    const size_t o = (size_t)bh * dp + c;
+    if (p.vm && SAGE_STORE_OK(p.x_vm, p.vm + o, 4, &g_quant_error)) p.vm[o] = mean;
+    if (SAGE_STORE_OK(p.x_km, p.km + o, 4, &g_quant_error)) p.km[o] = k_mean_of(p, base, nblk, sv.nk, c);
+    if (SAGE_STORE_OK(p.x_vs, p.vs + o, 4, &g_quant_error)) p.vs[o] = __fdiv_rn(am, p.vmax_code);
+    if (SAGE_STORE_OK(p.x_vinv, p.vinv + o, 4, &g_quant_error)) p.vinv[o] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
   }
 }
 
@@ -462,15 +485,15 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
     if (isk) {
       const float km = k_mean_of(p, base, nblk, sv.nk, c);
       hv[0][c] = km;
-      if (blk0 == 0) p.km[bhh * dp + c] = km;
+      if (blk0 == 0 && SAGE_STORE_OK(p.x_km, p.km + bhh * dp + c, 4, &g_quant_error)) p.km[bhh * dp + c] = km;
     } else {
       float mean;
       const float am = v_amax_of(p, base, nblk, sv.nk, c, &mean);
       hv[0][c] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
       hv[1][c] = mean;
       if (blk0 == 0) {
-        p.vs[bhh * dp + c] = __fdiv_rn(am, p.vmax_code);
-        if (p.vm) p.vm[bhh * dp + c] = mean;
+        if (SAGE_STORE_OK(p.x_vs, p.vs + bhh * dp + c, 4, &g_quant_error)) p.vs[bhh * dp + c] = __fdiv_rn(am, p.vmax_code);
+        if (p.vm && SAGE_STORE_OK(p.x_vm, p.vm + bhh * dp + c, 4, &g_quant_error)) p.vm[bhh * dp + c] = mean;
       }
     }
     __syncthreads();
@@ -524,8 +547,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
     am = block_max(am, red);
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
     const long long row = sv.k_row0 + h * p.m.k_head_rows + n0;
-    store_int8_tile(p.k8 + row * dp, dp, tc, inv, rows, x);
-    if (threadIdx.x == 0) p.ks[row / 128] = __fdiv_rn(am, 127.f);
+    store_int8_tile(p.k8 + row * dp, dp, tc, inv, rows, x, p.x_k8);
+    if (threadIdx.x == 0 && SAGE_STORE_OK(p.x_ks, p.ks + row / 128, 4, &g_quant_error)) p.ks[row / 128] = __fdiv_rn(am, 127.f);
   } else {  // ---- V: E4M3 or fp16 codes, transposed to [channel][token]
     const int h = y - p.m.Hkv;
     const size_t bh = (size_t)b * p.m.Hkv + h;
@@ -556,8 +579,10 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
           w[q] = *reinterpret_cast<const uint32_t*>(&h2);
         }
         uint4* dst = reinterpret_cast<uint4*>(vt + (vrow + e) * pitch + vcol);
-        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        if (SAGE_STORE_OK(p.x_v8t, dst, 32, &g_quant_error)) {
+          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+        }
       }
     } else {
 #pragma unroll
@@ -571,7 +596,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
           const float a3 = vx(4 * q + 3, e);
           w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
         }
-        *reinterpret_cast<uint4*>(p.v8t + (vrow + e) * pitch + vcol) = make_uint4(w[0], w[1], w[2], w[3]);
+        uint8_t* const dst = p.v8t + (vrow + e) * pitch + vcol;
+        if (SAGE_STORE_OK(p.x_v8t, dst, 16, &g_quant_error)) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
       }
     }
   }

@@ -10,6 +10,27 @@
 
 namespace sage {
 
+// A buffer the kernels write: [base, base + bytes).  In the checked build (-DSAGE_CHECKED) every
+// global store is tested against the extent of the buffer it targets; a store outside it is
+// skipped and recorded in the kernel's device error word (SAGE_DEVERR_BOUNDS), never made.
+struct Extent {
+  unsigned char* base;
+  unsigned long long bytes;
+};
+enum : int { SAGE_DEVERR_BOUNDS = 4 };
+
+#ifdef SAGE_CHECKED
+__device__ __forceinline__ bool store_in_extent(const Extent& x, const void* ptr, unsigned long long n, int* err) {
+  const unsigned char* q = static_cast<const unsigned char*>(ptr);
+  const bool ok = x.base != nullptr && q >= x.base && q + n <= x.base + x.bytes;
+  if (!ok) atomicOr(err, SAGE_DEVERR_BOUNDS);
+  return ok;
+}
+#define SAGE_STORE_OK(x, ptr, n, err) ::sage::store_in_extent((x), (ptr), (n), (err))
+#else
+#define SAGE_STORE_OK(x, ptr, n, err) true
+#endif
+
 // One sequence of a packed (varlen) batch, as the planning kernel lays it out.
 struct SeqDesc {
   int nq, nk;              // query / key tokens
@@ -103,6 +124,8 @@ struct QuantParams {
   float vmax_code;   // 448 (FP8 P.V, fp32 accumulation) or 1 (the other P.V modes)
   int v_fp16;        // V codes are fp16 (FP16 P.V) instead of E4M3; v8t then holds 2 bytes per code
   int fold;          // pass 2 computes the K mean and V scales itself (no finalize launch)
+  // extents of the buffers above (store checks of the checked build)
+  Extent x_q8, x_qs, x_k8, x_ks, x_km, x_v8t, x_vs, x_vm, x_vinv, x_ksum, x_vmax, x_vsum, x_vmin;
 };
 
 struct FwdParams {
@@ -117,6 +140,7 @@ struct FwdParams {
   int G;          // query heads per kv head
   int vec_out;    // 16-byte output stores allowed (d % 8 == 0 and 16-byte aligned out)
   float scale_log2;  // sm_scale * log2(e)
+  Extent x_out;      // the output tensor (store checks of the checked build)
 };
 
 struct QkDumpParams {
@@ -134,6 +158,7 @@ cudaError_t launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUten
 cudaError_t launch_seq_plan(const int32_t* cu_q, const int32_t* cu_k, int B, int max_q, int max_k,
                             long long total_q, long long total_k, SeqDesc* seqs, cudaStream_t st);
 cudaError_t read_clear_device_error(int* value);
+cudaError_t read_clear_quant_error(int* value);  // the quantize kernels' error word (quant.cu)
 cudaError_t launch_wait_probe(long long budget_cycles, cudaStream_t st);
 // tcgen05.mma issue-rate probe: kind 0 = kind::i8, 1 = kind::f8f6f4, 2 = kind::f16; one CTA per SM.
 cudaError_t launch_mma_probe(int kind, int iters, int n_sm, cudaStream_t st);

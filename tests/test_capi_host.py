@@ -29,9 +29,23 @@ def test_library_exports_every_declared_symbol(lib):
         assert hasattr(raw, n), n
 
 
+def test_checked_build_exports_every_declared_symbol_and_says_so(lib):
+    # the -DSAGE_CHECKED twin is a separate library with the same boundary
+    checked = lib.load_checked()
+    for n in _declared():
+        assert hasattr(checked, n), n
+    assert checked.sage_checked_build() == 1
+    assert lib.capi.sage_checked_build() == 0
+    assert checked.sage_status_string(lib.SAGE_ERR_BOUNDS).decode() == lib.sage_status_string(lib.SAGE_ERR_BOUNDS)
+    # argument checks are the same host code in both
+    assert checked.sage_attn(FAKE, FAKE, FAKE, FAKE, 1, 2, 2, 256, 300, lib.SAGE_FP16, lib.SAGE_HND, 0, 0.0, 0,
+                             None) == lib.SAGE_ERR_INVALID_ARG
+
+
 def test_status_strings(lib):
-    for s in range(7):
+    for s in range(8):
         assert lib.sage_status_string(s)
+    assert "buffer" in lib.sage_status_string(lib.SAGE_ERR_BOUNDS)
     assert "fp16" in lib.sage_status_string(lib.SAGE_ERR_UNSUPPORTED)
 
 

@@ -120,7 +120,12 @@ HEAD_DIM_256 = [Workload("d256_b2_h16_n8192", 2, 16, 16, 8192, 256, "fp16", "HND
                 Workload("d256_b2_h16_n8192_causal", 2, 16, 16, 8192, 256, "fp16", "HND", True, "normal", 0, 6)]
 
 ALL = [TINY, IMAGE_DIT, VIDEO_DIT, LLM_GQA] + list(pad_sweep()) + FP16_PV + OPTIONS + FP32_ACC + HEAD_DIM_256
-BY_NAME = {w.name: w for w in ALL}
+
+# Short video-DiT cases (8192 tokens, inputs still larger than L2) for detailed profiles of the
+# fused kernel, whose counters take dozens of replays per launch.
+PROFILE = [VIDEO_DIT.with_(name="video_dit_b1_h24_n8192_d128_nhd", N=8192),
+           VIDEO_DIT.with_(name="video_dit_b1_h24_n8192_d128_nhd_fp32acc", N=8192, pv_mode=0)]
+BY_NAME = {w.name: w for w in ALL + PROFILE}
 
 
 def _gen(w: Workload, stream: int, seq: int = 0) -> torch.Generator:
