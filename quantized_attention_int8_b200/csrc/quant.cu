@@ -105,10 +105,11 @@ struct TileCoord {
   int g, cv, c0;  // token group, channel vector, first channel
 };
 
-__device__ __forceinline__ TileCoord tile_coord(int dp) {
+__device__ __forceinline__ TileCoord tile_coord_at(int dp, int tid) {
   const int nv = dp / 8;
-  return TileCoord{(int)threadIdx.x / nv, (int)threadIdx.x % nv, ((int)threadIdx.x % nv) * 8};
+  return TileCoord{tid / nv, tid % nv, (tid % nv) * 8};
 }
+__device__ __forceinline__ TileCoord tile_coord(int dp) { return tile_coord_at(dp, (int)threadIdx.x); }
 
 // Load this thread's 16 x 8 register tile of one head: tokens 16g+r (r < 16) of the block that
 // starts at x0 (tokens tok_stride elements apart), channels c0..c0+7.  Tokens >= rows and
@@ -432,19 +433,67 @@ __device__ __forceinline__ float v_amax_of(const QuantParams& p, long long base,
   return am;
 }
 
-__global__ void quant_finalize_kernel(QuantParams p) {
+// One CTA per (batch, kv head, 32 channels).  The partials of a chunk of kFinChunk blocks are
+// staged in shared memory by all eight warps at once (one 128-byte row per block and array, many
+// loads in flight), then warp 0 adds K's sums and warp 1 folds V's statistics, one lane per
+// channel, in block order: the same operations in the same order as k_mean_of / v_amax_of, so
+// the same bits, without a dependent global load per block.
+constexpr int kFinChunk = 64;
+
+__global__ void __launch_bounds__(256) quant_finalize_kernel(QuantParams p) {
+  __shared__ float stage[4][kFinChunk][32];  // ksum, vmax, vsum, vmin
   allow_next_grid();
   wait_for_previous_grid();  // pass 1's partial sums
   const int bh = blockIdx.x, b = bh / p.m.Hkv, h = bh - b * p.m.Hkv;
   const SeqView sv = seq_view(p.m, b);
   const int dp = p.m.dp, nblk = (sv.nk + 127) / 128;
   const long long base = (sv.k_row0 + h * p.m.k_head_rows) / 128 * dp;
-  for (int c = threadIdx.x; c < dp; c += blockDim.x) {
-    float mean;
-    const float am = v_amax_of(p, base, nblk, sv.nk, c, &mean);
-    const size_t o = (size_t)bh * dp + c;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, c = blockIdx.y * 32 + lane;
+  const int narr = p.smooth_v ? 4 : 2;
+  const float* src[4] = {p.ksum_part, p.vmax_part, p.vsum_part, p.vmin_part};
+  float kacc = 0.f, vacc = 0.f, hi = -INFINITY, lo = INFINITY, am = 0.f;
+  for (int b0 = 0; b0 < nblk; b0 += kFinChunk) {
+    const int nb = min(kFinChunk, nblk - b0);
+    // every load of the chunk in flight before the first store (block warp + 8 k of each array)
+    float tmp[4][kFinChunk / 8];
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int k = 0; k < kFinChunk / 8; ++k) {
+        const int i = warp + 8 * k;
+        tmp[a][k] = (a < narr && i < nb) ? src[a][base + (long long)(b0 + i) * dp + c] : 0.f;
+      }
+    __syncthreads();  // the previous chunk has been consumed
+#pragma unroll
+    for (int a = 0; a < 4; ++a)
+#pragma unroll
+      for (int k = 0; k < kFinChunk / 8; ++k) stage[a][warp + 8 * k][lane] = tmp[a][k];
+    __syncthreads();
+    if (warp == 0) {
+      for (int i = 0; i < nb; ++i) kacc = __fadd_rn(kacc, stage[0][i][lane]);
+    } else if (warp == 1) {
+      if (p.smooth_v) {
+        for (int i = 0; i < nb; ++i) {
+          vacc = __fadd_rn(vacc, stage[2][i][lane]);
+          hi = fmaxf(hi, stage[1][i][lane]);
+          lo = fminf(lo, stage[3][i][lane]);
+        }
+      } else {
+        for (int i = 0; i < nb; ++i) am = fmaxf(am, stage[1][i][lane]);
+      }
+    }
+  }
+  const size_t o = (size_t)bh * dp + c;
+  if (warp == 0) {
+    const float km = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(kacc, (float)sv.nk) : 0.f;
+    if (SAGE_STORE_OK(p.x_km, p.km + o, 4, &g_quant_error)) p.km[o] = km;
+  } else if (warp == 1) {
+    float mean = 0.f;
+    if (p.smooth_v) {
+      mean = (c < p.m.d && sv.nk > 0) ? __fdiv_rn(vacc, (float)sv.nk) : 0.f;
+      am = sv.nk > 0 ? fmaxf(fabsf(__fsub_rn(hi, mean)), fabsf(__fsub_rn(lo, mean))) : 0.f;
+    }
     if (p.vm && SAGE_STORE_OK(p.x_vm, p.vm + o, 4, &g_quant_error)) p.vm[o] = mean;
-    if (SAGE_STORE_OK(p.x_km, p.km + o, 4, &g_quant_error)) p.km[o] = k_mean_of(p, base, nblk, sv.nk, c);
     if (SAGE_STORE_OK(p.x_vs, p.vs + o, 4, &g_quant_error)) p.vs[o] = __fdiv_rn(am, p.vmax_code);
     if (SAGE_STORE_OK(p.x_vinv, p.vinv + o, 4, &g_quant_error)) p.vinv[o] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
   }
@@ -455,12 +504,106 @@ __device__ __forceinline__ uint32_t e4m3x2(float a, float b) {
   return __nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3) & 0xFFFFu;
 }
 
+// K - mean(K) of one 128-token block in registers: INT8 codes with the block's scale (rows past
+// the sequence masked), written at q8-layout row `row`.  max_all reduces a float over every
+// thread that holds part of the block; `leader` writes the scale.
+template <typename T, typename MaxAll>
+__device__ __forceinline__ void code_k_block(const QuantParams& p, const uint4 (&v)[16], const TileCoord& tc, int rows,
+                                             const float (&km)[8], long long row, MaxAll max_all, bool leader) {
+  const int dp = p.m.dp, d = p.m.d;
+  // padded channels read 0 and have mean 0; padded rows are masked by store_int8_tile
+  auto x = [&](int r, int e) -> float { return __fsub_rn(elem<T>(v[r], e), km[e]); };
+  // max |k - mean| per channel is reached at the channel's largest or smallest k, since
+  // rounding k - mean to float32 is monotonic in k: take per-channel extremes on the packed
+  // values, then subtract the mean from those two only.
+  using P2 = typename Pair2<T>::type;
+  P2 hi[4], lo[4];
+  bool any = false;
+#pragma unroll
+  for (int r = 0; r < 16; ++r) {
+    if (tc.g * 16 + r < rows) {
+      const P2* w = reinterpret_cast<const P2*>(&v[r]);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hi[e] = any ? __hmax2(hi[e], w[e]) : w[e];
+        lo[e] = any ? __hmin2(lo[e], w[e]) : w[e];
+      }
+      any = true;
+    }
+  }
+  float am = 0.f;
+  if (any) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi[e]);
+      const uint32_t lb = *reinterpret_cast<const uint32_t*>(&lo[e]);
+      if (tc.c0 + 2 * e < d)
+        am = fmaxf(am, fmaxf(fabsf(__fsub_rn(bits_to_f32<T>(hb & 0xFFFFu), km[2 * e])),
+                             fabsf(__fsub_rn(bits_to_f32<T>(lb & 0xFFFFu), km[2 * e]))));
+      if (tc.c0 + 2 * e + 1 < d)
+        am = fmaxf(am, fmaxf(fabsf(__fsub_rn(bits_to_f32<T>(hb >> 16), km[2 * e + 1])),
+                             fabsf(__fsub_rn(bits_to_f32<T>(lb >> 16), km[2 * e + 1]))));
+    }
+  }
+  am = max_all(am);
+  const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
+  store_int8_tile(p.k8 + row * dp, dp, tc, inv, rows, x, p.x_k8);
+  if (leader && SAGE_STORE_OK(p.x_ks, p.ks + row / 128, 4, &g_quant_error)) p.ks[row / 128] = __fdiv_rn(am, 127.f);
+}
+
+// V of one block in registers: E4M3 or fp16 codes of (v - mean) * inv, transposed to V^T (this
+// thread's channels start at V^T row vrow, its 16 tokens at column vcol).
+template <typename T, bool SMOOTH_V>
+__device__ __forceinline__ void code_v_block(const QuantParams& p, const uint4 (&v)[16], const TileCoord& tc, int rows,
+                                             const float (&inv)[8], const float (&mean)[8], long long vrow,
+                                             long long vcol) {
+  // (v - mean) * inv; tokens past N give 0 (with smoothing the subtraction would not)
+  auto vx = [&](int r, int e) -> float {
+    if (!SMOOTH_V) return __fmul_rn(elem<T>(v[r], e), inv[e]);  // tokens past N load as 0 -> code 0
+    const float x = __fsub_rn(elem<T>(v[r], e), mean[e]);
+    return (tc.g * 16 + r < rows) ? __fmul_rn(x, inv[e]) : 0.f;
+  };
+  const long long pitch = p.m.k_head_rows;
+  if (p.v_fp16) {
+    // fp16_rne(v * inv): 16 tokens of one channel = 32 bytes (padded tokens and channels read 0)
+    uint16_t* vt = reinterpret_cast<uint16_t*>(p.v8t);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      uint32_t w[8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        const __half2 h2 = __floats2half2_rn(vx(2 * q, e), vx(2 * q + 1, e));
+        w[q] = *reinterpret_cast<const uint32_t*>(&h2);
+      }
+      uint4* dst = reinterpret_cast<uint4*>(vt + (vrow + e) * pitch + vcol);
+      if (SAGE_STORE_OK(p.x_v8t, dst, 32, &g_quant_error)) {
+        dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+        dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+      }
+    }
+  } else {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      uint32_t w[4];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float a0 = vx(4 * q + 0, e);
+        const float a1 = vx(4 * q + 1, e);
+        const float a2 = vx(4 * q + 2, e);
+        const float a3 = vx(4 * q + 3, e);
+        w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
+      }
+      uint8_t* const dst = p.v8t + (vrow + e) * pitch + vcol;
+      if (SAGE_STORE_OK(p.x_v8t, dst, 16, &g_quant_error)) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
 template <typename T, bool SMOOTH_V>
 __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
   extern __shared__ uint4 stage[];  // p.prefetch: 16 slots per thread
   __shared__ float red[8];
   allow_next_grid();
-  wait_for_previous_grid();  // the finalize kernel's K mean and V scales
   // Last-read-first: pass 1 read V after K and batch B-1 last, so those are the tiles most likely
   // still in L2 when this pass reads them again.
   const int y = gridDim.y - 1 - blockIdx.y, b = gridDim.z - 1 - blockIdx.z;
@@ -473,6 +616,7 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
   const bool vec = isk ? p.vec_k : p.vec_v;
   const int blk0 = (gridDim.x - 1 - blockIdx.x) * p.bpc, blk1 = min((sv.nk + 127) / 128, blk0 + p.bpc);
   if (blk0 >= blk1) return;  // past the end of this sequence (the whole CTA leaves)
+  wait_for_previous_grid();  // pass 1's partials (p.fold), or the finalize kernel's K mean and V scales
   // Short sequences (p.fold): no finalize launch; every CTA computes its head's K mean, or V's
   // scales and mean, from pass 1's partials in the same order, and the head's first CTA writes
   // them out.  Otherwise the finalize kernel has written them.
@@ -510,45 +654,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
     float km[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) km[e] = p.fold ? hv[0][tc.c0 + e] : p.km[bh * dp + tc.c0 + e];
-    // padded channels read 0 and have mean 0; padded rows are masked by store_int8_tile
-    auto x = [&](int r, int e) -> float { return __fsub_rn(elem<T>(v[r], e), km[e]); };
-    // max |k - mean| per channel is reached at the channel's largest or smallest k, since
-    // rounding k - mean to float32 is monotonic in k: take per-channel extremes on the packed
-    // values, then subtract the mean from those two only.
-    using P2 = typename Pair2<T>::type;
-    P2 hi[4], lo[4];
-    bool any = false;
-#pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      if (tc.g * 16 + r < rows) {
-        const P2* w = reinterpret_cast<const P2*>(&v[r]);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          hi[e] = any ? __hmax2(hi[e], w[e]) : w[e];
-          lo[e] = any ? __hmin2(lo[e], w[e]) : w[e];
-        }
-        any = true;
-      }
-    }
-    float am = 0.f;
-    if (any) {
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t hb = *reinterpret_cast<const uint32_t*>(&hi[e]);
-        const uint32_t lb = *reinterpret_cast<const uint32_t*>(&lo[e]);
-        if (tc.c0 + 2 * e < d)
-          am = fmaxf(am, fmaxf(fabsf(__fsub_rn(bits_to_f32<T>(hb & 0xFFFFu), km[2 * e])),
-                               fabsf(__fsub_rn(bits_to_f32<T>(lb & 0xFFFFu), km[2 * e]))));
-        if (tc.c0 + 2 * e + 1 < d)
-          am = fmaxf(am, fmaxf(fabsf(__fsub_rn(bits_to_f32<T>(hb >> 16), km[2 * e + 1])),
-                               fabsf(__fsub_rn(bits_to_f32<T>(lb >> 16), km[2 * e + 1]))));
-      }
-    }
-    am = block_max(am, red);
-    const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
     const long long row = sv.k_row0 + h * p.m.k_head_rows + n0;
-    store_int8_tile(p.k8 + row * dp, dp, tc, inv, rows, x, p.x_k8);
-    if (threadIdx.x == 0 && SAGE_STORE_OK(p.x_ks, p.ks + row / 128, 4, &g_quant_error)) p.ks[row / 128] = __fdiv_rn(am, 127.f);
+    code_k_block<T>(p, v, tc, rows, km, row, [&](float a) { return block_max(a, red); }, threadIdx.x == 0);
   } else {  // ---- V: E4M3 or fp16 codes, transposed to [channel][token]
     const int h = y - p.m.Hkv;
     const size_t bh = (size_t)b * p.m.Hkv + h;
@@ -557,49 +664,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
     for (int e = 0; e < 8; ++e) inv[e] = p.fold ? hv[0][tc.c0 + e] : p.vinv[bh * dp + tc.c0 + e];
 #pragma unroll
     for (int e = 0; e < 8; ++e) mean[e] = SMOOTH_V ? (p.fold ? hv[1][tc.c0 + e] : p.vm[bh * dp + tc.c0 + e]) : 0.f;
-    // (v - mean) * inv; tokens past N give 0 (with smoothing the subtraction would not)
-    auto vx = [&](int r, int e) -> float {
-      if (!SMOOTH_V) return __fmul_rn(elem<T>(v[r], e), inv[e]);  // tokens past N load as 0 -> code 0
-      const float x = __fsub_rn(elem<T>(v[r], e), mean[e]);
-      return (tc.g * 16 + r < rows) ? __fmul_rn(x, inv[e]) : 0.f;
-    };
-    // V^T element (channel c, token t) of this sequence and head: row v_row0 + h*dp + c, column
-    // v_col0 + t, rows k_head_rows codes apart
     const long long vrow = sv.v_row0 + (long long)h * dp + tc.c0, vcol = sv.v_col0 + n0 + tc.g * 16;
-    const long long pitch = p.m.k_head_rows;
-    if (p.v_fp16) {
-      // fp16_rne(v * inv): 16 tokens of one channel = 32 bytes (padded tokens and channels read 0)
-      uint16_t* vt = reinterpret_cast<uint16_t*>(p.v8t);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        uint32_t w[8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          const __half2 h2 = __floats2half2_rn(vx(2 * q, e), vx(2 * q + 1, e));
-          w[q] = *reinterpret_cast<const uint32_t*>(&h2);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(vt + (vrow + e) * pitch + vcol);
-        if (SAGE_STORE_OK(p.x_v8t, dst, 32, &g_quant_error)) {
-          dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
-          dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
-        }
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        uint32_t w[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float a0 = vx(4 * q + 0, e);
-          const float a1 = vx(4 * q + 1, e);
-          const float a2 = vx(4 * q + 2, e);
-          const float a3 = vx(4 * q + 3, e);
-          w[q] = e4m3x2(a0, a1) | (e4m3x2(a2, a3) << 16);
-        }
-        uint8_t* const dst = p.v8t + (vrow + e) * pitch + vcol;
-        if (SAGE_STORE_OK(p.x_v8t, dst, 16, &g_quant_error)) *reinterpret_cast<uint4*>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
-      }
-    }
+    code_v_block<T, SMOOTH_V>(p, v, tc, rows, inv, mean, vrow, vcol);
   }
   __syncthreads();  // `red` is reused by the next block
   if (blk + 1 < blk1) {
@@ -609,6 +675,166 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
       load_tile<T>(v, src + (long long)(n0 + 128) * tstride, tstride, d, min(128, sv.nk - n0 - 128), vec, tc);
   }
   }
+}
+
+// ------------------------------------------------------------------------------------------------
+// Single-launch quantize pass for short dense sequences (at most 32 blocks of 128 tokens, dp <= 128,
+// per-block Q scales, V not smoothed).  A cluster of ceil(nblk / 4) CTAs covers one head; each CTA
+// holds four blocks, one per group of dp threads, in registers.  K and V CTAs exchange their
+// per-block statistics through distributed shared memory, so K and V are read once and no
+// finalize or second pass is launched; every operation, and its order, is that of the two-pass
+// path, so codes, scales and means are the same bits.
+// ------------------------------------------------------------------------------------------------
+constexpr int kClusterGroups = 4;  // blocks (thread groups) per CTA
+constexpr int kClusterMaxBlocks = 32;
+
+__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void cluster_arrive() { asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory"); }
+__device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory"); }
+// `local` in the shared memory of the cluster's CTA `rank`
+__device__ __forceinline__ float ld_cluster(const float* local, int rank) {
+  const uint32_t a = static_cast<uint32_t>(__cvta_generic_to_shared(local));
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(a), "r"(rank));
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(ra) : "memory");
+  return v;
+}
+// max of v over the nthreads threads of group gi (named barrier 1 + gi), as block_max over a CTA
+__device__ __forceinline__ float group_max(float v, float* red, int gi, int tid, int nthreads) {
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  if ((tid & 31) == 0) red[tid >> 5] = v;
+  named_bar_sync(1 + gi, nthreads);
+  float r = 0.f;
+  for (int i = 0; i < (nthreads >> 5); ++i) r = fmaxf(r, red[i]);
+  return r;
+}
+
+template <typename T>
+__global__ void __launch_bounds__(512, 1) quant_cluster_kernel(QuantParams p) {
+  constexpr int G = kClusterGroups;
+  __shared__ float red[G][8];
+  __shared__ float part[G][8 * 128];
+  __shared__ float bstat[G][128];  // this CTA's per-block statistic (K: column sums, V: column amax)
+  __shared__ float hv[128];        // the head's K mean or V 1 / scale
+  allow_next_grid();
+  const int dp = p.m.dp, d = p.m.d;
+  const int gi = threadIdx.x / dp, tid = threadIdx.x - gi * dp;
+  const TileCoord tc = tile_coord_at(dp, tid);
+  const int rank = blockIdx.x;  // the cluster spans x: the CTA's rank in it
+  const int y = blockIdx.y, b = blockIdx.z;
+  const SeqView sv = seq_view<0>(p.m, b);
+  const T* src;
+  long long tstride;
+  int ntok;
+  bool vec;
+  if (y < p.m.Hq) {
+    src = static_cast<const T*>(p.q) + sv.q_in + y * sv.q_head, tstride = sv.q_tok, ntok = sv.nq, vec = p.vec_q;
+  } else if (y < p.m.Hq + p.m.Hkv) {
+    src = static_cast<const T*>(p.k) + sv.k_in + (y - p.m.Hq) * sv.k_head, tstride = sv.k_tok, ntok = sv.nk;
+    vec = p.vec_k;
+  } else {
+    src = static_cast<const T*>(p.v) + sv.k_in + (y - p.m.Hq - p.m.Hkv) * sv.k_head, tstride = sv.k_tok;
+    ntok = sv.nk, vec = p.vec_v;
+  }
+  const int nblk = (ntok + 127) / 128, blk = rank * G + gi;
+  const bool has = blk < nblk;
+  const int n0 = blk * 128, rows = has ? min(128, ntok - n0) : 0;
+  uint4 v[16];
+  if (has) load_tile<T>(v, src + (long long)n0 * tstride, tstride, d, rows, vec, tc);
+  auto gmax = [&](float a) { return group_max(a, red[gi], gi, tid, dp); };
+  if (y < p.m.Hq) {  // ---- Q: codes and per-block scale (a Q cluster takes no cluster barrier)
+    if (has) {
+      const long long row = sv.q_row0 + y * p.m.q_head_rows + n0;
+      const float am = gmax(tile_absmax<T>(v));
+      const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
+      store_int8_tile(p.q8 + row * dp, dp, tc, inv, rows, [&](int r, int e) { return elem<T>(v[r], e); }, p.x_q8);
+      if (tid == 0 && SAGE_STORE_OK(p.x_qs, p.qs + row / 128, 4, &g_quant_error)) p.qs[row / 128] = __fdiv_rn(am, 127.f);
+    }
+    return;
+  }
+  const bool isk = y < p.m.Hq + p.m.Hkv;
+  const int h = isk ? y - p.m.Hq : y - p.m.Hq - p.m.Hkv;
+  const size_t bh = (size_t)b * p.m.Hkv + h;
+  if (has) {  // the block's statistic, as pass 1 computes it
+    float* pg = part[gi];
+    if (isk) {
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+#pragma unroll
+      for (int r = 0; r < 16; ++r)
+        if (tc.g * 16 + r < rows)
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = __fadd_rn(acc[e], elem<T>(v[r], e));
+#pragma unroll
+      for (int e = 0; e < 8; ++e) pg[tc.g * dp + tc.c0 + e] = acc[e];
+      named_bar_sync(1 + gi, dp);
+      bstat[gi][tid] = tree8_sum(pg, dp, tid);
+    } else {
+      uint32_t a[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int r = 0; r < 16; ++r) {
+        a[0] = absmax_bits(a[0], v[r].x);
+        a[1] = absmax_bits(a[1], v[r].y);
+        a[2] = absmax_bits(a[2], v[r].z);
+        a[3] = absmax_bits(a[3], v[r].w);
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        pg[tc.g * dp + tc.c0 + 2 * e] = bits_to_f32<T>(a[e] & 0xFFFFu);
+        pg[tc.g * dp + tc.c0 + 2 * e + 1] = bits_to_f32<T>(a[e] >> 16);
+      }
+      named_bar_sync(1 + gi, dp);
+      bstat[gi][tid] = tree8_max(pg, dp, tid);
+    }
+  }
+  cluster_arrive();
+  cluster_wait();  // every CTA's bstat is written and visible
+  if (gi == 0) {   // the head's statistic, one thread per channel, blocks in order
+    float x[kClusterMaxBlocks];
+#pragma unroll
+    for (int i = 0; i < kClusterMaxBlocks; ++i) x[i] = i < nblk ? ld_cluster(&bstat[i % G][tid], i / G) : 0.f;
+    if (isk) {
+      float acc = 0.f;
+#pragma unroll
+      for (int i = 0; i < kClusterMaxBlocks; ++i)
+        if (i < nblk) acc = __fadd_rn(acc, x[i]);
+      const float km = (tid < d && ntok > 0) ? __fdiv_rn(acc, (float)ntok) : 0.f;
+      hv[tid] = km;
+      if (rank == 0 && SAGE_STORE_OK(p.x_km, p.km + bh * dp + tid, 4, &g_quant_error)) p.km[bh * dp + tid] = km;
+    } else {
+      float am = 0.f;
+#pragma unroll
+      for (int i = 0; i < kClusterMaxBlocks; ++i)
+        if (i < nblk) am = fmaxf(am, x[i]);
+      hv[tid] = am > 0.f ? __fdiv_rn(p.vmax_code, am) : 0.f;
+      if (rank == 0) {
+        if (SAGE_STORE_OK(p.x_vs, p.vs + bh * dp + tid, 4, &g_quant_error)) p.vs[bh * dp + tid] = __fdiv_rn(am, p.vmax_code);
+        if (p.vm && SAGE_STORE_OK(p.x_vm, p.vm + bh * dp + tid, 4, &g_quant_error)) p.vm[bh * dp + tid] = 0.f;
+      }
+    }
+  }
+  cluster_arrive();  // this CTA has read the others' statistics
+  __syncthreads();   // hv for every group
+  if (has) {
+    if (isk) {
+      float km[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) km[e] = hv[tc.c0 + e];
+      const long long row = sv.k_row0 + h * p.m.k_head_rows + n0;
+      code_k_block<T>(p, v, tc, rows, km, row, gmax, tid == 0);
+    } else {
+      float inv[8], mean[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) inv[e] = hv[tc.c0 + e], mean[e] = 0.f;
+      const long long vrow = sv.v_row0 + (long long)h * dp + tc.c0, vcol = sv.v_col0 + n0 + tc.g * 16;
+      code_v_block<T, false>(p, v, tc, rows, inv, mean, vrow, vcol);
+    }
+  }
+  cluster_wait();  // no CTA leaves while another may still read its statistics
 }
 
 // Launch `kern` so that it may start while the previous kernel in the stream still runs (it
@@ -638,6 +864,23 @@ static cudaError_t launch_quant_t(const QuantParams& p_in, cudaStream_t st) {
   // CTA walks a few consecutive blocks of its head, the next block's tile streaming in behind the
   // current one (measured: 328 -> 305 us on a 604 MB pass); below that, one block per CTA (walking
   // four blocks per CTA made a 113 MB pass slower, 60 -> 64 us).
+  // Short dense sequences with the default options: one launch of clusters (see above).
+  if (!p.m.seqs && p.q_gran_log2 == 7 && !p.smooth_v && dp <= 128 && nblk1 <= kClusterMaxBlocks) {
+    const int cs = (nblk1 + kClusterGroups - 1) / kClusterGroups;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(cs, Hq + 2 * Hkv, B);
+    cfg.blockDim = dim3(kClusterGroups * dp);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = st;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = cs;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, quant_cluster_kernel<T>, p);
+  }
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const long long blocks = (long long)nblk1 * (Hq + 2 * Hkv) * B, slots = (long long)sms * 8;
@@ -656,7 +899,7 @@ static cudaError_t launch_quant_t(const QuantParams& p_in, cudaStream_t st) {
   // partials; measured faster than a separate launch there), beyond that a finalize launch.
   p.fold = nblk1 <= 64 ? 1 : 0;
   if (!p.fold) {
-    e = launch_dependent(quant_finalize_kernel, dim3(B * Hkv), dim3(dp), st, p);
+    e = launch_dependent(quant_finalize_kernel, dim3(B * Hkv, dp / 32), dim3(256), st, p);
     if (e != cudaSuccess) return e;
   }
   const int nblk2 = p.nblk_k > 0 ? p.nblk_k : 1;
