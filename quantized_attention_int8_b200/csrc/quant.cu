@@ -685,8 +685,8 @@ __global__ void __launch_bounds__(256, 2) quant_pass2_kernel(QuantParams p) {
 // finalize or second pass is launched; every operation, and its order, is that of the two-pass
 // path, so codes, scales and means are the same bits.
 // ------------------------------------------------------------------------------------------------
-constexpr int kClusterGroups = 4;  // blocks (thread groups) per CTA
 constexpr int kClusterMaxBlocks = 32;
+constexpr int kClusterGroupsUsed = 4;  // blocks per CTA: clusters of ceil(nblk / 4) <= 8 CTAs
 
 __device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
@@ -712,9 +712,8 @@ __device__ __forceinline__ float group_max(float v, float* red, int gi, int tid,
   return r;
 }
 
-template <typename T>
+template <typename T, int G>  // G: blocks (thread groups of dp threads) per CTA
 __global__ void __launch_bounds__(512, 1) quant_cluster_kernel(QuantParams p) {
-  constexpr int G = kClusterGroups;
   __shared__ float red[G][8];
   __shared__ float part[G][8 * 128];
   __shared__ float bstat[G][128];  // this CTA's per-block statistic (K: column sums, V: column amax)
@@ -866,10 +865,16 @@ static cudaError_t launch_quant_t(const QuantParams& p_in, cudaStream_t st) {
   // four blocks per CTA made a 113 MB pass slower, 60 -> 64 us).
   // Short dense sequences with the default options: one launch of clusters (see above).
   if (!p.m.seqs && p.q_gran_log2 == 7 && !p.smooth_v && dp <= 128 && nblk1 <= kClusterMaxBlocks) {
-    const int cs = (nblk1 + kClusterGroups - 1) / kClusterGroups;
+    constexpr int G = kClusterGroupsUsed;
+    const int cs = (nblk1 + G - 1) / G;
+    auto kern = quant_cluster_kernel<T, G>;
+    if (cs > 8) {
+      const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+      if (e != cudaSuccess) return e;
+    }
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(cs, Hq + 2 * Hkv, B);
-    cfg.blockDim = dim3(kClusterGroups * dp);
+    cfg.blockDim = dim3(G * dp);
     cfg.dynamicSmemBytes = 0;
     cfg.stream = st;
     cudaLaunchAttribute attr[1];
@@ -879,7 +884,7 @@ static cudaError_t launch_quant_t(const QuantParams& p_in, cudaStream_t st) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, quant_cluster_kernel<T>, p);
+    return cudaLaunchKernelEx(&cfg, kern, p);
   }
   int dev = 0, sms = 148;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
