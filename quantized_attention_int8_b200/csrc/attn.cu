@@ -374,7 +374,11 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
     const float* ksp = p.ks + (sv.k_row0 + (long long)hkv * p.m.k_head_rows) / 128;
     unsigned char* prow = sP + row * C::ROWB;
     float m = -INFINITY, l = 0.f;  // m: reference max; l accumulates the stored P values' scale
-    float ks_next = DQK == 64 ? ksp[0] : 0.f;  // d = 64: the next tile's K scale
+    // the next key tile's K scale, loaded one tile ahead so that its global-load latency leaves the
+    // tile's critical path (measured +2.8% to +3.2% at d = 128 without a causal mask); the causal
+    // d >= 128 fp32-accumulation instances load it in the loop, measured faster there
+    constexpr bool KS_AHEAD = DQK == 64 || !CAUSAL || MODE == 1;
+    float ks_next = KS_AHEAD ? ksp[0] : 0.f;
     bool ok = true;
     for (int i = 0; i < n_kv; ++i) {
       if (!warp_wait(&bars->s_full, i & 1, abort)) { ok = false; break; }
@@ -387,11 +391,10 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       tmem_wait_ld();
       if (MODE == 0) arm_s();  // S is in registers: re-arm it for the next Q.K^T
 
-      // dequantization factor in the log2 domain, with the K scale of the 128-key block; at d = 64
-      // that scale is loaded one tile ahead (measured +1.3% with FP8 P.V, +3.7% with FP16 P.V;
-      // 5% slower in the causal d = 128 instance, so the others load it here)
+      // dequantization factor in the log2 domain, with the K scale of the 128-key block (loaded one
+      // tile ahead where KS_AHEAD, else here)
       float ksv;
-      if constexpr (DQK == 64) {
+      if constexpr (KS_AHEAD) {
         ksv = ks_next;
         if (i + 1 < n_kv) ks_next = ksp[(i + 1) * BN / 128];
       } else {
@@ -524,34 +527,38 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
         // bits (measured +2.8% on the video-DiT shape, +1.7% with FP16 P.V).
         const bool scaled = i == 0 || __any_sync(0xffffffffu, alpha != 1.f);
         const float am = i == 0 ? 0.f : alpha;
+        // 64 columns of O per batch, both loads in flight before one wait (the merge waits on
+        // tensor-memory loads: measured +1.8% on the video-DiT shape over 32-column batches)
 #pragma unroll
-        for (int cc = 0; cc < DV / 32; ++cc) {
-          uint32_t o[32];
+        for (int cc = 0; cc < DV / 64; ++cc) {
+          uint32_t o[64];
           if (i > 0) {
-            tmem_ld32(ocol + cc * 32, o);
+            tmem_ld32(ocol + cc * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+            tmem_ld32(ocol + cc * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
             tmem_wait_ld();
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = 0u;
+            for (int e = 0; e < 64; ++e) o[e] = 0u;
           }
           if (scaled) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 32; ++e) {
               float a0 = __uint_as_float(o[2 * e]) * am, a1 = __uint_as_float(o[2 * e + 1]) * am;
-              add_f16x2_f32(t[cc * 16 + e], a0, a1);
+              add_f16x2_f32(t[cc * 32 + e], a0, a1);
               o[2 * e] = __float_as_uint(a0);
               o[2 * e + 1] = __float_as_uint(a1);
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
+            for (int e = 0; e < 32; ++e) {
               float a0 = __uint_as_float(o[2 * e]), a1 = __uint_as_float(o[2 * e + 1]);
-              add_f16x2_f32(t[cc * 16 + e], a0, a1);
+              add_f16x2_f32(t[cc * 32 + e], a0, a1);
               o[2 * e] = __float_as_uint(a0);
               o[2 * e + 1] = __float_as_uint(a1);
             }
           }
-          tmem_st32(ocol + cc * 32, o);
+          tmem_st32(ocol + cc * 64, *reinterpret_cast<uint32_t(*)[32]>(&o[0]));
+          tmem_st32(ocol + cc * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&o[32]));
         }
         tmem_wait_st();
       }
