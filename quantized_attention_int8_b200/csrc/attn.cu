@@ -67,6 +67,16 @@ struct FwdCfg {
   // scores are in registers.
   static constexpr uint32_t S_COL = 0, T_COL = 0, O_COL = BN > DV ? BN : DV;
   static constexpr uint32_t TMEM_COLS = O_COL + DV <= 128 ? 128 : (O_COL + DV <= 256 ? 256 : 512);
+  // FP8 P where tensor memory has 32 columns to spare behind O (d = 64; d = 256 at one CTA per SM):
+  // the softmax stores P there with one tcgen05.st and the P.V MMA reads its A operand from tensor
+  // memory, so P neither goes through shared memory nor needs an async-proxy fence (fp32
+  // accumulation only; the fp16+fp32 instances keep P in shared memory, measured to spill).
+  static constexpr bool P_TMEM = !PV16 && (DQK == 64 || DQK == 256);
+  // behind O where it fits, else (d = 256: O at columns 256-511) in the columns between S and O,
+  // which fp32 accumulation leaves unused
+  static constexpr uint32_t P_COL = O_COL + DV + ROWB / 4 <= TMEM_COLS ? O_COL + DV : BN;
+  static_assert(!P_TMEM || (P_COL + ROWB / 4 <= TMEM_COLS && (P_COL >= O_COL + DV || P_COL + ROWB / 4 <= O_COL)),
+                "P in tensor memory");
   static_assert(ROWB == 128, "P and V^T rows are one 128-byte swizzle span");
   static_assert(O_COL + DV <= TMEM_COLS, "TMEM plan");
   static_assert(ST <= 8, "barrier array size");
@@ -299,6 +309,8 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
           const uint64_t ad = smem_desc_kmajor(pa + k * 32, C::ROWB), bd = smem_desc_kmajor(va + k * 32, C::ROWB);
           if (PV16)
             umma_f16(pv_dst, ad, bd, idesc_pv, acc);
+          else if (C::P_TMEM && MODE == 0)
+            umma_f8_ts(pv_dst, tmem + C::P_COL + k * 8, bd, idesc_pv, acc);
           else
             umma_f8(pv_dst, ad, bd, idesc_pv, acc);
         }
@@ -483,13 +495,18 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
       }
       // 16-byte chunk ch of the 128-byte row goes to chunk ch ^ (row & 7): the 128B swizzle the
       // P.V descriptor expects
+      if constexpr (C::P_TMEM && MODE == 0) {
+        tmem_st32(tmem + lane_base + C::P_COL, *reinterpret_cast<const uint32_t(*)[32]>(&pw[0]));
+        tmem_wait_st();
+      } else {
 #pragma unroll
-      for (int ch = 0; ch < C::ROWB / 16; ++ch) {
-        const int sw = row & 7;
-        *reinterpret_cast<uint4*>(prow + ((ch ^ sw) << 4)) =
-            make_uint4(pw[ch * 4 + 0], pw[ch * 4 + 1], pw[ch * 4 + 2], pw[ch * 4 + 3]);
+        for (int ch = 0; ch < C::ROWB / 16; ++ch) {
+          const int sw = row & 7;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ sw) << 4)) =
+              make_uint4(pw[ch * 4 + 0], pw[ch * 4 + 1], pw[ch * 4 + 2], pw[ch * 4 + 3]);
+        }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
       if (rescale) {
         // O *= alpha (rows whose reference did not move have alpha = 1); 64 columns per batch,
         // every TMEM load of a batch in flight before one wait
