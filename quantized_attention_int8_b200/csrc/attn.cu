@@ -66,15 +66,16 @@ struct FwdCfg {
   // per-tile fp16 accumulator T (DV columns) reuses S's columns (and those up to O) once the
   // scores are in registers.
   static constexpr uint32_t S_COL = 0, T_COL = 0, O_COL = BN > DV ? BN : DV;
-  static constexpr uint32_t TMEM_COLS = O_COL + DV <= 128 ? 128 : (O_COL + DV <= 256 ? 256 : 512);
-  // FP8 P where tensor memory has 32 columns to spare behind O (d = 64; d = 256 at one CTA per SM):
-  // the softmax stores P there with one tcgen05.st and the P.V MMA reads its A operand from tensor
-  // memory, so P neither goes through shared memory nor needs an async-proxy fence (fp32
-  // accumulation only; the fp16+fp32 instances keep P in shared memory, measured to spill).
-  static constexpr bool P_TMEM = !PV16 && (DQK == 64 || DQK == 256);
-  // behind O where it fits, else (d = 256: O at columns 256-511) in the columns between S and O,
-  // which fp32 accumulation leaves unused
-  static constexpr uint32_t P_COL = O_COL + DV + ROWB / 4 <= TMEM_COLS ? O_COL + DV : BN;
+  // P (32 columns: 128 E4M3 or 64 fp16 keys per row) in tensor memory for the fp32-accumulation
+  // instances where columns are free: between S and O when they fit there, else behind O.  The
+  // softmax stores P there with one tcgen05.st and the P.V MMA reads its A operand from tensor
+  // memory, so P neither goes through shared memory nor needs an async-proxy fence (the
+  // fp16+fp32 instances keep P in shared memory: their T shares S's columns, and they spilled).
+  // FP8 P at d = 128 has no free columns (S and O fill 256).
+  static constexpr bool P_TMEM = PV16 || DQK == 64 || DQK == 256;
+  static constexpr uint32_t P_COL = BN + ROWB / 4 <= O_COL ? BN : O_COL + DV;
+  static constexpr uint32_t COLS_USED = (P_TMEM && P_COL + ROWB / 4 > O_COL + DV) ? P_COL + ROWB / 4 : O_COL + DV;
+  static constexpr uint32_t TMEM_COLS = COLS_USED <= 128 ? 128 : (COLS_USED <= 256 ? 256 : 512);
   static_assert(!P_TMEM || (P_COL + ROWB / 4 <= TMEM_COLS && (P_COL >= O_COL + DV || P_COL + ROWB / 4 <= O_COL)),
                 "P in tensor memory");
   static_assert(ROWB == 128, "P and V^T rows are one 128-byte swizzle span");
@@ -307,12 +308,16 @@ __global__ void __launch_bounds__(192, FwdCfg<DQK, DV, PV16>::CTAS_PER_SM)
         for (int k = 0; k < C::ROWB / 32; ++k) {
           const uint32_t acc = MODE == 0 ? (uint32_t)(i > 0 || k > 0) : (uint32_t)(k > 0);
           const uint64_t ad = smem_desc_kmajor(pa + k * 32, C::ROWB), bd = smem_desc_kmajor(va + k * 32, C::ROWB);
-          if (PV16)
+          if (C::P_TMEM && MODE == 0) {
+            if (PV16)
+              umma_f16_ts(pv_dst, tmem + C::P_COL + k * 8, bd, idesc_pv, acc);
+            else
+              umma_f8_ts(pv_dst, tmem + C::P_COL + k * 8, bd, idesc_pv, acc);
+          } else if (PV16) {
             umma_f16(pv_dst, ad, bd, idesc_pv, acc);
-          else if (C::P_TMEM && MODE == 0)
-            umma_f8_ts(pv_dst, tmem + C::P_COL + k * 8, bd, idesc_pv, acc);
-          else
+          } else {
             umma_f8(pv_dst, ad, bd, idesc_pv, acc);
+          }
         }
         umma_commit(C::SPLIT_RING ? &bars->v_empty[st] : &bars->k_empty[st]);  // the V (and K) stage
         umma_commit(&bars->pv_done);
