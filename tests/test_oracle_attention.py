@@ -157,7 +157,7 @@ def test_emulation_fp16_pv_modes():
         emc = emulate.emulate(qz, True, 0.35)[0, :N]
         pref = np.cumsum(v[0, 0].astype(np.float64), 0) / np.arange(1, N + 1)[:, None]
         assert np.allclose(emc, pref, rtol=1e-6, atol=1e-7)
-    # and the method stays within the spec cosine on the tiny workload
+    # and the method stays within the target cosine (0.999) on the tiny workload
     w = W.TINY
     q, k, v = W.make_inputs(w)
     for mode in (2, 3):
